@@ -1,0 +1,324 @@
+"""Pins of the CPU oracle against things other than itself (no GPU).
+
+Each test names what fixes the expected value: a value printed on the TQ4_1S
+page ("企业官网建设流程全解析", hotelren.com/news/5458160), a textbook table, a
+closed form, a library routine (numpy / scipy), brute force, or an invariant
+of the method.  Chosen so that a dropped term, a wrong sign or index, or a
+transposed operand in the oracle fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy import integrate
+from scipy.linalg import hadamard
+from scipy.stats import norm
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_table(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([c.strip() for c in line.split("|")])
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# codebook (page: 16 Lloyd-Max centroids of N(0,1); 72.5% error reduction)
+# ---------------------------------------------------------------------------
+def test_lloyd_matches_textbook_tables(oracle_mod):
+    for row in _read_table("lloyd_max_gaussian.txt"):
+        if not row[0].isdigit():
+            continue
+        L = int(row[0])
+        levels = np.array([float(v) for v in row[1].split()])
+        mse_tab = float(row[2])
+        c, mse, _ = oracle_mod.lloyd(L)
+        assert np.all(np.diff(c) > 0)
+        np.testing.assert_allclose(c[L // 2:], levels, atol=6e-4)  # table has 4 digits
+        np.testing.assert_allclose(-c[: L // 2][::-1], levels, atol=6e-4)
+        assert abs(mse - mse_tab) < 1e-3 * mse_tab  # 4 printed digits
+
+
+def test_lloyd_two_level_closed_form(oracle_mod):
+    c, mse, _ = oracle_mod.lloyd(2)
+    assert abs(c[1] - math.sqrt(2 / math.pi)) < 1e-13
+    assert abs(c[0] + math.sqrt(2 / math.pi)) < 1e-13
+    assert abs(mse - (1 - 2 / math.pi)) < 1e-13
+
+
+def test_error_reduction_printed_on_page(oracle_mod):
+    (row,) = [r for r in _read_table("lloyd_max_gaussian.txt") if r[0].startswith("page_")]
+    _, m16, _ = oracle_mod.lloyd(16)
+    _, m8, _ = oracle_mod.lloyd(8)
+    assert abs((1 - m16 / m8) - float(row[1])) < 1e-3
+
+
+def test_lloyd_fixed_point_by_quadrature(oracle_mod):
+    """Centroid = conditional mean of its cell, MSE by numerical integration
+    (scipy quad + scipy.stats.norm), independent of the oracle's closed forms."""
+    c, mse, _ = oracle_mod.lloyd(16)
+    t = np.concatenate(([-np.inf], (c[1:] + c[:-1]) / 2, [np.inf]))
+    total = 0.0
+    for i in range(16):
+        a, b = t[i], t[i + 1]
+        p = norm.cdf(b) - norm.cdf(a)
+        mean = integrate.quad(lambda x: x * norm.pdf(x), a, b, epsabs=1e-14, epsrel=1e-13)[0] / p
+        assert abs(mean - c[i]) < 1e-9
+        total += integrate.quad(lambda x: (x - c[i]) ** 2 * norm.pdf(x), a, b, epsabs=1e-15, epsrel=1e-12)[0]
+    assert abs(total - mse) < 1e-10
+
+
+def test_codebook_tables(oracle_mod):
+    M32, B32, M64 = oracle_mod.codebook()
+    c, _, _ = oracle_mod.lloyd(16)
+    np.testing.assert_array_equal(M64, c[8:])
+    np.testing.assert_array_equal(M32, c[8:].astype(np.float32))
+    np.testing.assert_array_equal(B32, ((c[8:-1] + c[9:]) / 2).astype(np.float32))
+    np.testing.assert_allclose(c[:8], -c[8:][::-1], atol=1e-14)  # symmetric
+
+
+# ---------------------------------------------------------------------------
+# transform and sign pattern (page: 格式原理 item 1)
+# ---------------------------------------------------------------------------
+def test_fwht_is_sylvester_hadamard(oracle_mod):
+    H = hadamard(32).astype(np.float64)
+    cols = oracle_mod.fwht32(np.eye(32))  # row i = H e_i = column i of H
+    np.testing.assert_array_equal(cols.T, H)
+    np.testing.assert_array_equal(H @ H.T, 32 * np.eye(32))
+
+
+def test_fwht_roundtrip_and_fp32_exact_on_integers(oracle_mod):
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((50, 32))
+    back = oracle_mod.fwht32(oracle_mod.fwht32(x)) / 32
+    np.testing.assert_allclose(back, x, rtol=0, atol=1e-13)
+    xi = rng.integers(-1000, 1000, (50, 32)).astype(np.float32)
+    exact = xi.astype(np.float64) @ hadamard(32).T
+    np.testing.assert_array_equal(oracle_mod.fwht32(xi).astype(np.float64), exact)
+
+
+def test_sign_pattern_properties(oracle_mod):
+    k = np.arange(28672)
+    s = oracle_mod.sign(k).astype(np.int64)
+    assert set(np.unique(s)) == {-1, 1}
+    # roughly balanced overall
+    assert abs(s.mean()) < 0.02
+    # per-block coherence with the Walsh functions behaves like random signs
+    # (a random +-1 vector of length 32 has mean max |<s,h_j>|/32 of ~0.42;
+    # the bare golden-ratio bit would sit near 0.71)
+    coh = np.abs(s.reshape(-1, 32) @ hadamard(32)).max(axis=1) / 32
+    assert 0.33 < coh.mean() < 0.5
+    # hash restatement (consistency, not an independent pin)
+    h = (k.astype(np.uint64) * 0x9E3779B9) & 0xFFFFFFFF
+    h ^= h >> 16
+    h = (h * 0x85EBCA6B) & 0xFFFFFFFF
+    h ^= h >> 13
+    np.testing.assert_array_equal(np.where(h >> 31, -1, 1), s)
+
+
+def test_f16_conversion_matches_numpy(oracle_mod):
+    rng = np.random.default_rng(5)
+    vals = np.concatenate([
+        rng.standard_normal(3000).astype(np.float32) * np.float32(10.0) ** rng.integers(-9, 6, 3000),
+        np.array([0.0, -0.0, 65504.0, 65519.996, 65520.0, 1e9, -1e9, 2.0 ** -24, 2.0 ** -25,
+                  2.0 ** -25 * 1.0000001, 3 * 2.0 ** -26, 6.1e-5, 6.0975e-5, 1.0009765625, 1.00048828125,
+                  1.00146484375, np.inf, -np.inf], np.float32),
+    ]).astype(np.float32)
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(oracle_mod.f32_to_f16_bits(vals), ref)
+    back = oracle_mod.f16_bits_to_f32(ref)
+    np.testing.assert_array_equal(back, ref.view(np.float16).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------
+# quantiser (page: 格式原理 items 1-3)
+# ---------------------------------------------------------------------------
+def test_worked_block(oracle_mod):
+    s = oracle_mod.sign(np.arange(32)).astype(np.float32)
+    for row in _read_table("worked_block.txt"):
+        a = float(row[0])
+        code, d = oracle_mod.quantize_block((a * s).astype(np.float32), 0)
+        assert code[0] == int(row[1])
+        assert np.all(code[1:] == 0)
+        assert d[0] == int(row[2], 16) and d[1] == int(row[3], 16)
+        W = np.zeros((1, 32), np.float32)
+        W[0] = a * s
+        c, sc = oracle_mod.quantize(W)
+        ratio = oracle_mod.dequantize(c, sc, 1, 32)[0] / (a * s)
+        special = np.isin(np.arange(32), (0, 16))
+        # fixture ratios come from the 4-digit table values
+        np.testing.assert_allclose(ratio[~special], float(row[4]), rtol=5e-4)
+        np.testing.assert_allclose(ratio[special], float(row[5]), rtol=5e-4)
+
+
+def _rotated_fp64(oracle_mod, W):
+    """y = H (s .* w) per block in fp64 with scipy's Hadamard matrix."""
+    n, k = W.shape
+    s = oracle_mod.sign(np.arange(k)).astype(np.float64)
+    u = (W.astype(np.float64) * s).reshape(n, k // 32, 32)
+    return u @ hadamard(32).T.astype(np.float64)
+
+
+def test_codes_are_nearest_centroid_brute_force(oracle_mod):
+    """fp64 brute-force nearest of y/d among the 16 centroids agrees with the
+    oracle's fp32 threshold search except at counted near-ties."""
+    rng = np.random.default_rng(11)
+    n, k = 64, 512
+    W = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    codes, scales = oracle_mod.quantize(W)
+    code, d = oracle_mod.unpack(codes, scales, n, k)
+    y = _rotated_fp64(oracle_mod, W)
+    # scales: fp16 of the RMS of each half (fp64 reference, at most 1 ulp apart)
+    rms = np.sqrt((y.reshape(n, k // 32, 2, 16) ** 2).mean(axis=3))
+    ref_bits = rms.astype(np.float16).view(np.uint16).astype(np.int64)
+    diff = np.abs(ref_bits - d.astype(np.int64))
+    assert diff.max() <= 1 and (diff > 0).mean() < 0.01
+    D = d.view(np.float16).astype(np.float64)  # [n, nb, 2]
+    Dfull = np.repeat(D, 16, axis=2).reshape(n, k)
+    _, _, M64 = oracle_mod.codebook()
+    cents = np.concatenate((-M64[::-1], M64))  # ascending 16 values
+    q = y.reshape(n, k) / Dfull
+    nearest = np.abs(q[..., None] - cents).argmin(axis=-1)  # index into cents
+    got = np.where(code & 8, 7 - (code & 7), 8 + (code & 7))
+    bad = nearest != got
+    if bad.any():
+        mids = (cents[1:] + cents[:-1]) / 2
+        gap = np.abs(np.abs(q[bad])[:, None] - np.abs(mids)[None, :]).min(axis=1)
+        assert gap.max() < 1e-5, gap.max()
+    assert bad.mean() < 1e-3
+
+
+def test_scale_invariance_and_negation(oracle_mod):
+    rng = np.random.default_rng(12)
+    W = (rng.standard_normal((8, 256)) * 0.02).astype(np.float32)
+    c0, s0 = oracle_mod.quantize(W)
+    for p in (-3, 2, 7):
+        c1, s1 = oracle_mod.quantize((W * np.float32(2.0 ** p)).astype(np.float32))
+        np.testing.assert_array_equal(c1, c0)
+        np.testing.assert_array_equal(s1.view(np.float16), (s0.view(np.float16) * np.float16(2.0 ** p)))
+    cn, sn = oracle_mod.quantize(-W)
+    np.testing.assert_array_equal(sn, s0)
+    code0, _ = oracle_mod.unpack(c0, s0, 8, 256)
+    coden, _ = oracle_mod.unpack(cn, sn, 8, 256)
+    y = _rotated_fp64(oracle_mod, W).reshape(8, 256)
+    nz = y != 0
+    np.testing.assert_array_equal(coden[nz] & 7, code0[nz] & 7)
+    np.testing.assert_array_equal(coden[nz] ^ code0[nz], np.full(nz.sum(), 8, np.uint8))
+
+
+def test_zero_and_underflow_blocks(oracle_mod):
+    W = np.zeros((2, 64), np.float32)
+    W[1, :32] = 1e-30  # rotated RMS far below fp16 range -> d = 0
+    c, s = oracle_mod.quantize(W)
+    code, d = oracle_mod.unpack(c, s, 2, 64)
+    assert np.all(code[0] == 0) and np.all(d == 0)
+    np.testing.assert_array_equal(oracle_mod.dequantize(c, s, 2, 64), 0.0)
+
+
+def test_reconstruction_error_matches_lloyd_mse(oracle_mod):
+    """Gaussian weights: relative L2 error of quantise -> dequantise is close
+    to sqrt(MSE16) ~ 0.0975 (a dropped sign or transposed transform gives ~1.4)."""
+    rng = np.random.default_rng(13)
+    W = (rng.standard_normal((64, 1024)) * 0.02).astype(np.float32)
+    c, s = oracle_mod.quantize(W)
+    Wr = oracle_mod.dequantize(c, s, 64, 1024)
+    rel = np.linalg.norm(Wr - W) / np.linalg.norm(W)
+    assert 0.088 < rel < 0.105, rel
+
+
+def test_dequantize_is_inverse_rotation(oracle_mod):
+    """w~ = s .* (H c) / 32 with scipy's H and the unpacked codes."""
+    rng = np.random.default_rng(14)
+    n, k = 4, 192
+    W = (rng.standard_normal((n, k)) * 0.05).astype(np.float32)
+    c, s = oracle_mod.quantize(W)
+    code, d = oracle_mod.unpack(c, s, n, k)
+    M32, _, _ = oracle_mod.codebook()
+    mag = M32[code & 7].astype(np.float64) * np.where(code & 8, -1.0, 1.0)
+    D = np.repeat(d.view(np.float16).astype(np.float64), 16, axis=2).reshape(n, k)
+    chat = (mag * D).reshape(n, k // 32, 32)
+    sg = oracle_mod.sign(np.arange(k)).astype(np.float64)
+    ref = (chat @ hadamard(32).astype(np.float64)).reshape(n, k) / 32 * sg
+    np.testing.assert_allclose(oracle_mod.dequantize(c, s, n, k), ref, rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# packing (page: nibble packing, 16 centroids, no correction term)
+# ---------------------------------------------------------------------------
+def test_packing_layout_and_bits_per_weight(oracle_mod):
+    rng = np.random.default_rng(15)
+    for k in (32, 96, 128, 160, 4096):
+        n = 3
+        W = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+        c, s = oracle_mod.quantize(W)
+        nsb = (k // 32 + 3) // 4
+        assert c.shape == (n, nsb * 64) and s.shape == (n, nsb * 8)
+        if k % 128 == 0:
+            assert (c.nbytes + s.nbytes) * 8 / (n * k) == 5.0
+        code, d = oracle_mod.unpack(c, s, n, k)
+        for r in range(n):
+            for b in range(k // 32):
+                cb, db = oracle_mod.quantize_block(W[r, 32 * b:32 * b + 32], 32 * b)
+                np.testing.assert_array_equal(code[r, 32 * b:32 * b + 32], cb)
+                np.testing.assert_array_equal(d[r, b], db)
+                # explicit byte positions of the stated layout
+                sb, j = divmod(b, 4)
+                for L in range(16):
+                    byte = c[r, sb * 64 + 16 * (L % 4) + 4 * j + L // 4]
+                    assert byte == cb[2 * L] | (cb[2 * L + 1] << 4)
+                assert s[r, sb * 8 + 2 * j] == db[0] and s[r, sb * 8 + 2 * j + 1] == db[1]
+        # padding blocks are zero
+        nb = k // 32
+        for b in range(nb, nsb * 4):
+            j = b % 4
+            for L in range(16):
+                assert np.all(c[:, (nsb - 1) * 64 + 16 * (L % 4) + 4 * j + L // 4] == 0)
+    # page: 28-42% smaller than Q8_0 (8.5 bits/weight); an all-TQ4_1S tensor is 41.2%
+    assert abs((1 - 5.0 / 8.5) - 0.412) < 1e-3 and 0.28 <= 1 - 5.0 / 8.5 <= 0.42
+
+
+# ---------------------------------------------------------------------------
+# product (page: 解码速度 section, pre-rotated activation)
+# ---------------------------------------------------------------------------
+def test_gemm_equals_prerotated_form(oracle_mod):
+    """sum_k w~[r,k] x[k] = (1/32) sum_b sum_h d * sum_e c_e (H (s .* x))_e."""
+    rng = np.random.default_rng(16)
+    n, k, m = 5, 384, 3
+    W = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    X = rng.standard_normal((m, k))
+    c, s = oracle_mod.quantize(W)
+    Y = oracle_mod.gemm(c, s, n, k, X)
+    code, d = oracle_mod.unpack(c, s, n, k)
+    M32, _, _ = oracle_mod.codebook()
+    cent = M32[code & 7].astype(np.float64) * np.where(code & 8, -1.0, 1.0)
+    D = np.repeat(d.view(np.float16).astype(np.float64), 16, axis=2).reshape(n, k)
+    sg = oracle_mod.sign(np.arange(k)).astype(np.float64)
+    xrot = ((X * sg).reshape(m, k // 32, 32) @ hadamard(32).T.astype(np.float64)).reshape(m, k)
+    Y2 = (xrot @ (cent * D).T) / 32
+    np.testing.assert_allclose(Y, Y2, rtol=1e-12, atol=1e-14)
+    # and the plain matrix product over the dequantised weights
+    np.testing.assert_allclose(Y, X @ oracle_mod.dequantize(c, s, n, k).T, rtol=1e-12, atol=1e-14)
+
+
+def test_gemm_one_hot_reads_a_column(oracle_mod):
+    rng = np.random.default_rng(17)
+    n, k = 6, 96
+    W = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    c, s = oracle_mod.quantize(W)
+    Wd = oracle_mod.dequantize(c, s, n, k)
+    for j in (0, 31, 32, 95):
+        x = np.zeros((1, k))
+        x[0, j] = 1.0
+        np.testing.assert_array_equal(oracle_mod.gemm(c, s, n, k, x)[0], Wd[:, j])
+
+
+def test_quantize_rejects_ragged_k(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.quantize(np.zeros((2, 48), np.float32))
