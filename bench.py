@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the TQ4_1S hot path on B200 (one JSON line on rank 0).
+
+Workload (default): one Llama-3-8B-shaped decoder layer -- q,o 4096x4096,
+k,v 1024x4096, gate,up 14336x4096, down 4096x14336 -- bf16 weights
+~N(0, 0.02^2) with 1% of input columns replaced by 0.02*10*t(4) values,
+batch-1 bf16 activations ~N(0,1).  Synthetic, seeded; no checkpoints.
+
+A step is one pass of the whole path over the layer:
+  quantise all seven matrices -> dequantise all seven (bf16) ->
+  pre-rotate + fused GEMV for all seven (fp32 y).
+The step is captured once in a CUDA graph and replayed.
+
+Reported:
+  value      GEMV weight GB/s = packed layer bytes (codes + scales) / GEMV
+             phase time (the seven pre-rotate + fused-GEMV launches), L2
+             flushed before every timed replay, CUDA events on the stream;
+  quantize   Gweights/s of the quantise phase (same protocol);
+  ms_per_step  the full step (graph replay), inputs resident in HBM;
+  e2e        the same GB/s metric through the public API with host buffers:
+             every step copies the bf16 weights and activations from pinned
+             host memory, runs the path and reads the outputs back;
+  roofline   for the phase with the largest share of the step, against the
+             measured HBM copy bandwidth; rooflines for every phase;
+  cpu_baseline  the CPU oracle (single thread) on a bounded row sample.
+
+Multi-GPU (torchrun): every rank runs its own layer (independent problems,
+no collective on the data path, weak scaling); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "TQ4_1S dequant-GEMV weight GB/s (% of HBM peak) at M=1; quantize Gweights/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", choices=("llama3_8b_layer", "single_matrix", "ffn_70b"), default="llama3_8b_layer")
+    p.add_argument("--skip-cpu-baseline", action="store_true")
+    p.add_argument("--skip-e2e", action="store_true")
+    p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    p.add_argument("--cpu-sample-rows", type=int, default=None,
+                   help="rows per matrix for the CPU oracle sample (default: 1/8 of each matrix)")
+    return p.parse_args(argv)
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+
+    FIELDS = ["index", "pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device: int):
+        props = torch.cuda.get_device_properties(device)
+        self.bus = f"{getattr(props, 'pci_domain_id', 0):08X}:{getattr(props, 'pci_bus_id', 0):02X}:" \
+                   f"{getattr(props, 'pci_device_id', 0):02X}.0"
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.file.read())) if len(r) == len(self.FIELDS)]
+        self.file.close()
+        os.unlink(self.file.name)
+        mine = [r for r in rows if r[1].strip().upper().endswith(self.bus[-12:].upper())] or rows
+        sm = [float(r[2]) for r in mine if r[2].strip().replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in mine if r[3].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in mine for i in range(4) if r[6 + i].strip().lower() == "active"})
+        loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(mine)}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+def make_workload(name: str, rank: int, device):
+    from dequant_gemv_tq4_b200 import inputs
+
+    mats = []  # (label, W, activation name)
+    acts = {}
+    if name == "llama3_8b_layer":
+        weights, acts = inputs.llama3_8b_layer(seed=100 * rank, device=device)
+        for label, W in weights.items():
+            mats.append((label, W, inputs.LLAMA3_8B_INPUTS[label]))
+        desc = {"workload": "llama3_8b_layer", "shapes": {k: list(v) for k, v in inputs.LLAMA3_8B_LAYER.items()},
+                "weights": "bf16 ~N(0,0.02^2), 1% outlier columns 0.2*t(4)", "x": "bf16 ~N(0,1)", "m": 1}
+    elif name == "single_matrix":
+        W, x = inputs.single_matrix(device=device)
+        mats.append(("w", W, "x"))
+        acts = {"x": x}
+        desc = {"workload": "single_matrix_2048", "shapes": {"w": [2048, 2048]}, "weights": "fp32 ~N(0,0.02^2)",
+                "x": "fp32 ~N(0,1)", "m": 1}
+    else:
+        for tid, (label, (n, k)) in enumerate(inputs.FFN_70B.items()):
+            mats.append((label, inputs.gaussian_matrix(2 + 100 * rank, tid, n, k, 0.015, torch.bfloat16, device),
+                         "x_" + label))
+            acts["x_" + label] = inputs.gaussian_matrix(1, 200 + tid, 1, k, 1.0, torch.bfloat16, device)[0]
+        desc = {"workload": "ffn_70b", "shapes": {k: list(v) for k, v in inputs.FFN_70B.items()},
+                "weights": "bf16 ~N(0,0.015^2)", "x": "bf16 ~N(0,1)", "m": 1}
+    return mats, acts, desc
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Path:
+    """Buffers and launches of one step of the hot path."""
+
+    def __init__(self, tq, mats, acts, device):
+        self.tq = tq
+        self.mats = mats
+        self.acts = acts
+        self.items = []
+        ws_bytes = 0
+        for label, W, act in mats:
+            n, k = W.shape
+            nsb = tq.superblocks(k)
+            codes = torch.empty((n, nsb * 64), dtype=torch.uint8, device=device)
+            scales = torch.empty((n, nsb * 8), dtype=torch.int16, device=device)
+            deq = torch.empty((n, k), dtype=torch.bfloat16, device=device)
+            y = torch.empty((n,), dtype=torch.float32, device=device)
+            self.items.append(dict(label=label, W=W, x=acts[act], n=n, k=k, codes=codes, scales=scales, deq=deq, y=y))
+            ws_bytes = max(ws_bytes, tq.tq_gemm_workspace_bytes(1, n, k))
+        self.ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
+
+    def quantize(self):
+        for it in self.items:
+            self.tq.quantize(it["W"], it["codes"], it["scales"])
+
+    def dequantize(self):
+        for it in self.items:
+            self.tq.dequantize(it["codes"], it["scales"], it["n"], it["k"], out=it["deq"])
+
+    def gemv(self):
+        for it in self.items:
+            self.tq.gemv(it["codes"], it["scales"], it["n"], it["k"], it["x"], out=it["y"], ws=self.ws)
+
+    def step(self):
+        self.quantize()
+        self.dequantize()
+        self.gemv()
+
+    # byte / weight accounting (algorithmic)
+    def weights(self):
+        return sum(it["n"] * it["k"] for it in self.items)
+
+    def packed_bytes(self):
+        return sum(it["codes"].numel() + 2 * it["scales"].numel() for it in self.items)
+
+    def in_bytes(self):
+        return sum(it["W"].numel() * it["W"].element_size() for it in self.items)
+
+    def act_bytes(self):
+        return sum(it["x"].numel() * it["x"].element_size() for it in self.items)
+
+    def out_bytes(self):
+        return sum(it["y"].numel() * 4 for it in self.items)
+
+
+def capture(fn, use_graph: bool):
+    if not use_graph:
+        return fn
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g.replay
+
+
+def time_replays(run, reps: int, flush=None):
+    """Sum of CUDA-event durations of `reps` calls on the current stream; the
+    optional flush runs before each call, outside the timed interval."""
+    stream = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        if flush is not None:
+            flush()
+        starts[i].record(stream)
+        run()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+
+
+def max_over_ranks(values, world):
+    if world == 1:
+        return values
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=torch.cuda.current_device())
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def cpu_oracle_sample(path, rows_per_matrix=None):
+    """The CPU oracle, as it stands, on the first rows of every matrix."""
+    import numpy as np
+
+    import oracle
+
+    oracle.build()
+    tq_w = tg = td = 0.0
+    weights = packed = 0
+    for it in path.items:
+        n, k = it["n"], it["k"]
+        r = rows_per_matrix if rows_per_matrix else max(1, n // 8)
+        W = it["W"][:r].float().cpu().numpy()
+        x = it["x"].float().cpu().numpy()[None].astype(np.float64)
+        t0 = time.perf_counter()
+        c, s = oracle.quantize(W)
+        t1 = time.perf_counter()
+        oracle.dequantize(c, s, r, k)
+        t2 = time.perf_counter()
+        oracle.gemm(c, s, r, k, x)
+        t3 = time.perf_counter()
+        tq_w += t1 - t0
+        td += t2 - t1
+        tg += t3 - t2
+        weights += r * k
+        packed += c.nbytes + s.nbytes
+    return {"gemv_gbs": packed / tg / 1e9, "quantize_gweights_per_s": weights / tq_w / 1e9,
+            "dequantize_gweights_per_s": weights / td / 1e9, "seconds": tq_w + td + tg,
+            "sample": f"first {rows_per_matrix or '1/8 of the'} rows of each of the {len(path.items)} matrices "
+                      f"({weights / 1e6:.1f} M weights): quantise, dequantise, GEMV"}
+
+
+def run_ours(args, world, rank, local):
+    import dequant_gemv_tq4_b200 as tq
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    tq.load_library()  # raises: there is no CPU path
+    mats, acts, desc = make_workload(args.workload, rank, device)
+    path = Path(tq, mats, acts, device)
+    nmat = len(path.items)
+    launches_per_step = 4 * nmat  # quantize, dequantize, prerotate, fused gemv per matrix
+    warmup = max(3, args.warmup)
+    steps = max(1, args.steps)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
+
+    def flush():
+        flush_buf.zero_()
+
+    for _ in range(warmup):
+        path.step()
+    torch.cuda.synchronize()
+    use_graph = not args.no_graph
+    try:
+        step_run = capture(path.step, use_graph)
+        q_run = capture(path.quantize, use_graph)
+        d_run = capture(path.dequantize, use_graph)
+        g_run = capture(path.gemv, use_graph)
+    except Exception as e:  # graph capture refused: launch eagerly
+        print(f"[bench] CUDA graph capture failed ({e}); launching eagerly", file=sys.stderr)
+        use_graph = False
+        step_run, q_run, d_run, g_run = path.step, path.quantize, path.dequantize, path.gemv
+    for run in (step_run, q_run, d_run, g_run):
+        for _ in range(warmup):
+            run()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    barrier(world)
+    sampler.start()
+    time.sleep(0.4)
+    barrier(world)
+    t_step = time_replays(step_run, steps)
+    barrier(world)
+    t_q = time_replays(q_run, steps, flush)
+    t_d = time_replays(d_run, steps, flush)
+    t_g = time_replays(g_run, steps, flush)
+    barrier(world)
+    clocks = sampler.stop()
+    t_step, t_q, t_d, t_g = max_over_ranks([t_step, t_q, t_d, t_g], world)
+
+    ms_step = t_step / steps
+    ms_q, ms_d, ms_g = t_q / steps, t_d / steps, t_g / steps
+    packed = path.packed_bytes()
+    weights = path.weights()
+    hbm, hbm_kind = measured_peaks()
+    value = world * packed / (ms_g * 1e-3) / 1e9
+    quant_gw = world * weights / (ms_q * 1e-3) / 1e9
+
+    # algorithmic bytes per phase (one GPU)
+    alg = {
+        "quantize": (path.in_bytes() + packed, ms_q, nmat),
+        "dequantize": (packed + 2 * weights, ms_d, nmat),
+        "gemv": (packed + path.act_bytes() + path.out_bytes(), ms_g, 2 * nmat),
+    }
+    rooflines = {}
+    for ph, (nbytes, ms, nl) in alg.items():
+        ach = nbytes / (ms * 1e-3) / 1e9
+        rooflines[ph] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": None, "bytes_per_step": nbytes,
+                         "ms": round(ms, 5), "launches": nl}
+    dominant = max(("quantize", "dequantize", "gemv"), key=lambda ph: alg[ph][1])
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in, fp16 tensor-core operands, fp32 accumulate",
+        "data": "synthetic (seeded counter-based generator; no checkpoints)",
+        "config": dict(desc, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                       l2="flushed (256 MB write) before every timed phase replay; step loop inputs > L2",
+                       graph=use_graph, hbm_peak_source=hbm_kind),
+        "pct_of_hbm_peak": round(100 * value / world / hbm, 2),
+        "quantize_gweights_per_s": round(quant_gw, 2),
+        "phases_ms": {"quantize": round(ms_q, 5), "dequantize": round(ms_d, 5), "gemv": round(ms_g, 5)},
+        "roofline": dict(rooflines[dominant], kernel=dominant, peak_note=f"{hbm_kind} HBM copy bandwidth"),
+        "rooflines": rooflines,
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * steps,
+    }
+
+    if not args.skip_e2e:
+        line["e2e"] = run_e2e(tq, path, steps=min(steps, 5), world=world)
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        cb = cpu_oracle_sample(path, args.cpu_sample_rows)
+        line["cpu_baseline"] = {"value": round(cb["gemv_gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": cb["sample"],
+                                "quantize_gweights_per_s": round(cb["quantize_gweights_per_s"], 5),
+                                "seconds": round(cb["seconds"], 1)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(tq, path, steps, world):
+    """Public API with host buffers: H2D of weights + activations from pinned
+    memory, quantise/dequantise/GEMV, D2H of every y, per step."""
+    host_w = [it["W"].cpu().pin_memory() for it in path.items]
+    host_x = [it["x"].cpu().pin_memory() for it in path.items]
+    host_y = [torch.empty_like(it["y"], device="cpu").pin_memory() for it in path.items]
+    dev_w = [torch.empty_like(it["W"]) for it in path.items]
+    dev_x = [torch.empty_like(it["x"]) for it in path.items]
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for i, it in enumerate(path.items):
+            dev_w[i].copy_(host_w[i], non_blocking=True)
+            dev_x[i].copy_(host_x[i], non_blocking=True)
+        for i, it in enumerate(path.items):
+            tq.quantize(dev_w[i], it["codes"], it["scales"])
+        for it in path.items:
+            tq.dequantize(it["codes"], it["scales"], it["n"], it["k"], out=it["deq"])
+        for i, it in enumerate(path.items):
+            tq.gemv(it["codes"], it["scales"], it["n"], it["k"], dev_x[i], out=it["y"], ws=path.ws)
+        for i, it in enumerate(path.items):
+            host_y[i].copy_(it["y"], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize()
+    (ms,) = max_over_ranks([start.elapsed_time(end) / steps], world)
+    return {"value": round(world * path.packed_bytes() / (ms * 1e-3) / 1e9, 2), "unit": UNIT,
+            "h2d_bytes_per_step": path.in_bytes() + path.act_bytes(), "d2h_bytes_per_step": path.out_bytes(),
+            "ms_per_step": round(ms, 4), "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from dequant_gemv_tq4_b200 import inputs
+
+    oracle.build()
+    # same workload, one row sample per step: the first 1/64 of every matrix's rows
+    if args.workload == "llama3_8b_layer":
+        shapes = [(lbl, n, k, seed) for seed, (lbl, (n, k)) in enumerate(inputs.LLAMA3_8B_LAYER.items())]
+    elif args.workload == "single_matrix":
+        shapes = [("w", 2048, 2048, 0)]
+    else:
+        shapes = [(lbl, n, k, tid) for tid, (lbl, (n, k)) in enumerate(inputs.FFN_70B.items())]
+    sample = []
+    for lbl, n, k, seed in shapes:
+        r = max(1, n // 64)
+        # the generator is row-major, so r rows are exactly the matrix's first r rows
+        if args.workload == "llama3_8b_layer":
+            W = inputs.llama_weight(seed, 0, r, k)
+        elif args.workload == "single_matrix":
+            W = inputs.gaussian_matrix(0, 0, r, k, 0.02, torch.float32)
+        else:
+            W = inputs.gaussian_matrix(2, seed, r, k, 0.015, torch.bfloat16)
+        x = inputs.gaussian_matrix(1, 7, 1, k, 1.0, torch.bfloat16).float().numpy().astype(np.float64)
+        sample.append((W.float().numpy(), x, r, k))
+
+    def step():
+        tg = 0.0
+        packed = 0
+        for W, x, r, k in sample:
+            c, s = oracle.quantize(W)
+            oracle.dequantize(c, s, r, k)
+            t0 = time.perf_counter()
+            oracle.gemm(c, s, r, k, x)
+            tg += time.perf_counter() - t0
+            packed += c.nbytes + s.nbytes
+        return packed, tg
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    tot_b = tot_t = 0.0
+    t0 = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        b, t = step()
+        tot_b += b
+        tot_t += t
+    wall = time.perf_counter() - t0
+    value = tot_b / tot_t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": max(1, args.steps), "warmup": max(3, args.warmup),
+            "ms_per_step": round(1e3 * wall / max(1, args.steps), 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp32 codec / fp64 product (CPU oracle)",
+            "data": "synthetic (seeded counter-based generator; no checkpoints)",
+            "config": {"workload": args.workload, "sample": "first 1/64 of the rows of every matrix per step"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": "first 1/64 of the rows of every matrix, quantise + dequantise + GEMV"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+        dist.init_process_group("nccl" if args.impl == "ours" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

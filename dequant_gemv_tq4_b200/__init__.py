@@ -1,0 +1,227 @@
+"""TQ4_1S weight codec and fused dequant-GEMV for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/tq.h`` (``libtq.so``, built
+in-tree by ``dequant_gemv_tq4_b200/build.py``).  Every step of the path runs in
+the library's CUDA kernels; this module only marshals arguments.  PyTorch is
+used for device memory and streams.  There is no CPU fallback: if the
+library cannot be loaded, every call raises.
+
+Two layers:
+  * ``tq_*`` functions with the C names and raw integer pointers (what the
+    ABI tests call);
+  * tensor helpers (``quantize``, ``dequantize``, ``prerotate``, ``gemm``,
+    ``gemv``, ``gemm_xrot``) that allocate outputs with torch and pass
+    ``data_ptr()`` and the current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
+_DTYPE_CODE = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}
+STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_INVALID_ARG", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGNMENT",
+                4: "TQ_ERR_DTYPE", 5: "TQ_ERR_WORKSPACE", 6: "TQ_ERR_CUDA", 7: "TQ_ERR_UNSUPPORTED"}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libtq.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libtq.so not built ({LIB_PATH}); run dequant_gemv_tq4_b200/build.py")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I64, SZ, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        sig = {
+            "tq_status_string": ([I], ctypes.c_char_p),
+            "tq_codes_bytes": ([I64, I64], SZ),
+            "tq_scales_bytes": ([I64, I64], SZ),
+            "tq_xrot_bytes": ([I64, I64], SZ),
+            "tq_gemm_workspace_bytes": ([I64, I64, I64], SZ),
+            "tq_quantize": ([P, I, I64, I64, I64, P, P, P], I),
+            "tq_dequantize": ([P, P, I64, I64, P, I, I64, P], I),
+            "tq_prerotate": ([P, I, I64, I64, I64, P, P], I),
+            "tq_gemm": ([P, P, I64, I64, P, I, I64, I64, P, I, I64, P, SZ, P], I),
+            "tq_gemv": ([P, P, I64, I64, P, I, P, I, P, SZ, P], I),
+            "tq_gemm_xrot": ([P, P, I64, I64, P, I64, P, I, I64, P, SZ, P], I),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise TQError(status, where)
+
+
+# ---------------------------------------------------------------------------
+# raw C-ABI layer (integer pointers)
+# ---------------------------------------------------------------------------
+def status_string(status: int) -> str:
+    return load_library().tq_status_string(int(status)).decode()
+
+
+def tq_codes_bytes(n: int, k: int) -> int:
+    return int(load_library().tq_codes_bytes(n, k))
+
+
+def tq_scales_bytes(n: int, k: int) -> int:
+    return int(load_library().tq_scales_bytes(n, k))
+
+
+def tq_xrot_bytes(m: int, k: int) -> int:
+    return int(load_library().tq_xrot_bytes(m, k))
+
+
+def tq_gemm_workspace_bytes(m: int, n: int, k: int) -> int:
+    return int(load_library().tq_gemm_workspace_bytes(m, n, k))
+
+
+def tq_quantize(w, wt, n, k, ldw, codes, scales, stream) -> int:
+    return load_library().tq_quantize(w, wt, n, k, ldw, codes, scales, stream)
+
+
+def tq_dequantize(codes, scales, n, k, w_out, ot, ldo, stream) -> int:
+    return load_library().tq_dequantize(codes, scales, n, k, w_out, ot, ldo, stream)
+
+
+def tq_prerotate(X, xt, m, k, ldx, xrot, stream) -> int:
+    return load_library().tq_prerotate(X, xt, m, k, ldx, xrot, stream)
+
+
+def tq_gemm(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_gemm(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream)
+
+
+def tq_gemv(codes, scales, n, k, x, xt, y, yt, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_gemv(codes, scales, n, k, x, xt, y, yt, workspace, ws_bytes, stream)
+
+
+def tq_gemm_xrot(codes, scales, n, k, xrot, m, Y, yt, ldy, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_gemm_xrot(codes, scales, n, k, xrot, m, Y, yt, ldy, workspace, ws_bytes, stream)
+
+
+# ---------------------------------------------------------------------------
+# tensor helpers
+# ---------------------------------------------------------------------------
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _dt(t: torch.dtype) -> int:
+    if t not in _DTYPE_CODE:
+        raise TypeError(f"unsupported dtype {t}")
+    return _DTYPE_CODE[t]
+
+
+def superblocks(k: int) -> int:
+    return (k // 32 + 3) // 4
+
+
+def _ld(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride")
+    return t.stride(0)
+
+
+def workspace(m: int, n: int, k: int, device=None) -> torch.Tensor:
+    """A workspace tensor for gemm/gemv/gemm_xrot of these sizes (zero-filled)."""
+    nbytes = tq_gemm_workspace_bytes(m, n, k)
+    if nbytes == 0:
+        raise ValueError("invalid sizes for workspace query")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or torch.cuda.current_device())
+
+
+def quantize(w: torch.Tensor, codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+             stream=None):
+    """Encode W (n x k, fp32/bf16/fp16, on the GPU).  Returns (codes uint8 [n, NSB*64],
+    scales int16 [n, NSB*8] holding fp16 bit patterns)."""
+    n, k = w.shape
+    nsb = superblocks(k)
+    if codes is None:
+        codes = torch.empty((n, nsb * 64), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((n, nsb * 8), dtype=torch.int16, device=w.device)
+    _check(tq_quantize(w.data_ptr(), _dt(w.dtype), n, k, _ld(w), codes.data_ptr(), scales.data_ptr(),
+                       _stream(stream)), "tq_quantize")
+    return codes, scales
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, n: int, k: int, dtype=torch.bfloat16,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((n, k), dtype=dtype, device=codes.device)
+    _check(tq_dequantize(codes.data_ptr(), scales.data_ptr(), n, k, out.data_ptr(), _dt(out.dtype), _ld(out),
+                         _stream(stream)), "tq_dequantize")
+    return out
+
+
+def prerotate(X: torch.Tensor, xrot: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    X2 = X.view(1, -1) if X.dim() == 1 else X
+    m, k = X2.shape
+    if xrot is None:
+        xrot = torch.empty(tq_xrot_bytes(m, k) // 2, dtype=torch.int16, device=X.device)
+    _check(tq_prerotate(X2.data_ptr(), _dt(X2.dtype), m, k, _ld(X2), xrot.data_ptr(), _stream(stream)),
+           "tq_prerotate")
+    return xrot
+
+
+def gemm(codes, scales, n: int, k: int, X: torch.Tensor, dtype=torch.float32, out=None, ws=None,
+         stream=None) -> torch.Tensor:
+    """Y[m, n] = X[m, k] @ w~[n, k]^T (w~ = the dequantised weights), fused."""
+    X2 = X.view(1, -1) if X.dim() == 1 else X
+    m = X2.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=dtype, device=X.device)
+    if ws is None:
+        ws = workspace(m, n, k, X.device)
+    _check(tq_gemm(codes.data_ptr(), scales.data_ptr(), n, k, X2.data_ptr(), _dt(X2.dtype), m, _ld(X2),
+                   out.data_ptr(), _dt(out.dtype), _ld(out), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "tq_gemm")
+    return out
+
+
+def gemv(codes, scales, n: int, k: int, x: torch.Tensor, dtype=torch.float32, out=None, ws=None,
+         stream=None) -> torch.Tensor:
+    """y[n] = w~[n, k] @ x[k], fused (m = 1)."""
+    if out is None:
+        out = torch.empty((n,), dtype=dtype, device=x.device)
+    if ws is None:
+        ws = workspace(1, n, k, x.device)
+    _check(tq_gemv(codes.data_ptr(), scales.data_ptr(), n, k, x.data_ptr(), _dt(x.dtype), out.data_ptr(),
+                   _dt(out.dtype), ws.data_ptr(), ws.numel(), _stream(stream)), "tq_gemv")
+    return out
+
+
+def gemm_xrot(codes, scales, n: int, k: int, xrot: torch.Tensor, m: int, dtype=torch.float32, out=None,
+              ws=None, stream=None) -> torch.Tensor:
+    """The fused product with an activation pre-rotated by ``prerotate`` (m <= 32)."""
+    if out is None:
+        out = torch.empty((m, n), dtype=dtype, device=xrot.device)
+    if ws is None:
+        ws = workspace(m, n, k, xrot.device)
+    _check(tq_gemm_xrot(codes.data_ptr(), scales.data_ptr(), n, k, xrot.data_ptr(), m, out.data_ptr(),
+                        _dt(out.dtype), _ld(out), ws.data_ptr(), ws.numel(), _stream(stream)), "tq_gemm_xrot")
+    return out

@@ -1,0 +1,187 @@
+// tq_device.cuh -- device-side building blocks shared by the TQ4_1S kernels.
+//
+// Method: TQ4_1S page ("企业官网建设流程全解析", hotelren.com/news/5458160),
+// paragraph 格式原理 (sign flip + 32-point Walsh-Hadamard rotation per block,
+// 16 Lloyd-Max centroids, two half-block scales) and section 解码速度：分硬件汇总
+// (the activation is pre-rotated once; decode is centroid lookup x scale).
+//
+// Floating-point rule for everything that decides a code or a scale: one
+// IEEE fp32 operation per step, round-to-nearest-even, in the order the codec
+// defines (explicit __fadd_rn/__fmul_rn/__fsqrt_rn so nothing is contracted
+// into an FMA); this file is compiled without fast-math, so no flush-to-zero.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "tq_codebook.h"
+
+namespace tq {
+
+constexpr int kBlock = 32;        // elements per block
+constexpr int kSbBlocks = 4;      // blocks per superblock
+constexpr int kSbElems = 128;     // elements per superblock
+constexpr int kSbCodeBytes = 64;  // code bytes per superblock
+constexpr int kSbScaleBytes = 16; // scale bytes per superblock (4 blocks x 2 fp16)
+constexpr unsigned kFull = 0xffffffffu;
+
+// Element dtypes, same numbering as tq_dtype in tq.h.
+enum Dtype : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
+
+__device__ __forceinline__ uint32_t f32_bits(float v) { return __float_as_uint(v); }
+
+// Sign pattern of global column k: golden-ratio multiplicative hash followed by
+// one MurmurHash3-style mixing round; -1 where bit 31 is set.  Returned as the
+// mask to XOR into an fp32 bit pattern (0x80000000 = negate, 0 = keep).
+__device__ __forceinline__ uint32_t sign_mask(uint32_t k) {
+    uint32_t h = k * 0x9E3779B9u;
+    h ^= h >> 16;
+    h *= 0x85EBCA6Bu;
+    h ^= h >> 13;
+    return h & 0x80000000u;
+}
+
+__device__ __forceinline__ float flip(float v, uint32_t mask) { return __uint_as_float(__float_as_uint(v) ^ mask); }
+
+// One butterfly stage across lanes: this lane holds element i, the partner lane
+// (lane ^ lane_xor) holds element i ^ h.  The lower index becomes a + b, the
+// upper a - b, exactly as the sequential transform computes them (fp32 add is
+// commutative, and partner - own == a - b for the upper element).
+__device__ __forceinline__ float butterfly_xlane(float v, int lane_xor, bool upper) {
+    float o = __shfl_xor_sync(kFull, v, lane_xor);
+    return upper ? __fsub_rn(o, v) : __fadd_rn(v, o);
+}
+
+// In-register stages h = 1 and h = 2 on four consecutive elements v[0..3].
+__device__ __forceinline__ void butterfly_local4(float (&v)[4]) {
+    float a0 = __fadd_rn(v[0], v[1]), a1 = __fsub_rn(v[0], v[1]);
+    float a2 = __fadd_rn(v[2], v[3]), a3 = __fsub_rn(v[2], v[3]);
+    v[0] = __fadd_rn(a0, a2);
+    v[2] = __fsub_rn(a0, a2);
+    v[1] = __fadd_rn(a1, a3);
+    v[3] = __fsub_rn(a1, a3);
+}
+
+// Loads of 4 consecutive elements converted (exactly) to fp32.
+template <int DT>
+__device__ __forceinline__ void load4(const void *p, float (&v)[4]);
+
+template <>
+__device__ __forceinline__ void load4<kF32>(const void *p, float (&v)[4]) {
+    float4 q = __ldg(reinterpret_cast<const float4 *>(p));
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+}
+
+template <>
+__device__ __forceinline__ void load4<kBF16>(const void *p, float (&v)[4]) {
+    uint2 q = __ldg(reinterpret_cast<const uint2 *>(p));
+    v[0] = __uint_as_float(q.x << 16);
+    v[1] = __uint_as_float(q.x & 0xffff0000u);
+    v[2] = __uint_as_float(q.y << 16);
+    v[3] = __uint_as_float(q.y & 0xffff0000u);
+}
+
+template <>
+__device__ __forceinline__ void load4<kF16>(const void *p, float (&v)[4]) {
+    uint2 q = __ldg(reinterpret_cast<const uint2 *>(p));
+    __half2 h0 = *reinterpret_cast<__half2 *>(&q.x), h1 = *reinterpret_cast<__half2 *>(&q.y);
+    float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+    v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+}
+
+// Stores of 4 consecutive fp32 values rounded (nearest-even) to the dtype.
+template <int DT>
+__device__ __forceinline__ void store4(void *p, const float (&v)[4]);
+
+template <>
+__device__ __forceinline__ void store4<kF32>(void *p, const float (&v)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+
+template <>
+__device__ __forceinline__ void store4<kBF16>(void *p, const float (&v)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 q;
+    q.x = *reinterpret_cast<uint32_t *>(&a);
+    q.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = q;
+}
+
+template <>
+__device__ __forceinline__ void store4<kF16>(void *p, const float (&v)[4]) {
+    __half2 a = __floats2half2_rn(v[0], v[1]), b = __floats2half2_rn(v[2], v[3]);
+    uint2 q;
+    q.x = *reinterpret_cast<uint32_t *>(&a);
+    q.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = q;
+}
+
+template <int DT>
+__device__ __forceinline__ void store1(void *p, float v);
+
+template <>
+__device__ __forceinline__ void store1<kF32>(void *p, float v) { *reinterpret_cast<float *>(p) = v; }
+
+template <>
+__device__ __forceinline__ void store1<kBF16>(void *p, float v) {
+    *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(v);
+}
+
+template <>
+__device__ __forceinline__ void store1<kF16>(void *p, float v) { *reinterpret_cast<__half *>(p) = __float2half_rn(v); }
+
+template <int DT>
+struct ElemSize {
+    static constexpr int value = DT == kF32 ? 4 : 2;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+
+// Streaming 128-bit global load: read-only, not kept in L1.
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// 128-bit global load that may stay in L1 (small, reused operands).
+__device__ __forceinline__ uint4 ldg_keep(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+// Byte permute: result byte i = byte sel_i of the 8-byte value {b, a}.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
+
+// D = A(16x16 f16, row) * B(16x8 f16, col) with a zero accumulator; fp32 out.
+__device__ __forceinline__ void mma_16816_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// Programmatic dependent launch: wait for the preceding grid's results / let
+// the next grid start its prologue.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+}  // namespace tq

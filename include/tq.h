@@ -1,0 +1,177 @@
+/*
+ * tq.h -- C ABI of libtq: the TQ4_1S weight codec and its fused dequant-GEMV
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: the web page titled "企业官网建设流程全解析"
+ * (hotelren.com/news/5458160; below "TQ page"), which describes TQ4_1S weight
+ * compression: paragraph 格式原理 items 1-3 (sign flip + 32-point Walsh-Hadamard
+ * rotation per block, nearest of 16 Lloyd-Max N(0,1) centroids, separate
+ * scales d0/d1 for elements 0-15 and 16-31), the paragraph after them (16
+ * centroids, nibble packing, no correction term; the reference dequantiser
+ * inverse-rotates and rescales) and section 解码速度：分硬件汇总 (decode
+ * pre-rotates the activation once, so dequantisation becomes centroid
+ * lookup times scale).
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions shared by every entry point
+ * ---------------------------------------------------------------------------
+ *  - W is N x K (out_features x in_features), row-major; y = W x.  Blocks of
+ *    32 run along K; K must be a positive multiple of 32.
+ *  - Pointers named codes/scales/w/x/y/workspace/xrot are DEVICE pointers on
+ *    the current CUDA device; the caller owns and allocates all of them.
+ *    The library allocates no memory and keeps no state beyond constant
+ *    tables.  stream is a cudaStream_t (NULL = legacy default stream).
+ *  - Calls are asynchronous on `stream` and never synchronise.  Argument
+ *    errors are detected on the host before any launch and nothing is
+ *    launched; a launch failure returns TQ_ERR_CUDA.
+ *  - n == 0 or m == 0 is an empty problem: TQ_OK, nothing launched.
+ *  - All results are deterministic run to run (no floating-point atomics).
+ *
+ * Packed format (5.0 bits per weight when K % 128 == 0):
+ *  - code: 4 bits; bit 3 = sign (1 = negative), bits 0-2 = magnitude rank
+ *    0..7 into the eight positive Lloyd-Max centroids.
+ *  - superblock = four consecutive 32-element blocks of one row (128
+ *    columns).  Row r has NSB = ceil(K/128) superblocks; blocks past K/32 in
+ *    the last one are padding (zero codes, zero scales).
+ *  - codes plane: uint8 [N][NSB][64].  Within a superblock, logical byte L
+ *    (0..15) of block j (0..3) holds the codes of elements 2L (low nibble)
+ *    and 2L+1 (high nibble) and is stored at byte 16*(L%4) + 4*j + L/4.
+ *  - scales plane: uint16 [N][NSB][4][2], IEEE fp16 bit patterns d0, d1 of
+ *    each block: d_h = fp16(sqrt(mean of the 16 squared rotated values)).
+ *  - rotation: y = H (s .* w) per block, H the unnormalised 32x32 Sylvester
+ *    Hadamard matrix; s_k = -1 where bit 31 of hash(k) is set, with
+ *    hash(k) = g(k * 0x9E3779B9) and g(h) = ((h ^ h>>16) * 0x85EBCA6B) ^ (...>>13)
+ *    on 32-bit words, k = global column index (same for every row).
+ *  - dequantisation: w~ = s .* (H c) / 32, c_e = +-M[mag_e] * d_h(e).
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1, /* null pointer, bad leading dimension, negative size */
+    TQ_ERR_SHAPE = 2,       /* k <= 0, k % 32 != 0, or a size above the supported maximum */
+    TQ_ERR_ALIGNMENT = 3,   /* a pointer or leading dimension breaks the alignment rule */
+    TQ_ERR_DTYPE = 4,       /* unknown tq_dtype value */
+    TQ_ERR_WORKSPACE = 5,   /* workspace null or smaller than the *_workspace_bytes query */
+    TQ_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    TQ_ERR_UNSUPPORTED = 7  /* valid request that this build does not implement */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* Largest supported sizes (checked; TQ_ERR_SHAPE above them). */
+#define TQ_MAX_N ((int64_t)1 << 30)
+#define TQ_MAX_K ((int64_t)1 << 26)
+
+/* Human-readable name of a status code (static string, never NULL). */
+TQ_API const char *tq_status_string(tq_status s);
+
+/* Bytes of the codes plane / of the scales plane for an N x K matrix
+ * (n * ceil(k/128) * 64 and n * ceil(k/128) * 16).  0 for invalid sizes. */
+TQ_API size_t tq_codes_bytes(int64_t n, int64_t k);
+TQ_API size_t tq_scales_bytes(int64_t n, int64_t k);
+
+/*
+ * tq_quantize -- encode W into the packed TQ4_1S planes.
+ * TQ page, 格式原理 items 1-3 and the paragraph after them: per 32-block,
+ * sign flip + Walsh-Hadamard rotation, two fp16 RMS half-block scales, then
+ * for every rotated value y the code sign(y) / #{j : |y| > B_j * d} with the
+ * seven Lloyd-Max decision thresholds B_j (ties go to the smaller magnitude,
+ * +0 and -0 count as positive).  Every step is IEEE fp32 in a fixed order,
+ * so codes and scales are bit-reproducible by a CPU implementation.
+ *   w      device, n x k of dtype wt (F32, BF16 or F16), row stride ldw
+ *          elements (ldw >= k, ldw % 8 == 0, w 16-byte aligned)
+ *   codes  device, tq_codes_bytes(n, k) bytes, 16-byte aligned (written)
+ *   scales device, tq_scales_bytes(n, k) bytes, 16-byte aligned (written)
+ * Inputs with |w| large enough to overflow fp16 scales (RMS >= 65520) or
+ * containing NaN/Inf are outside the contract.
+ */
+TQ_API tq_status tq_quantize(const void *w, tq_dtype wt, int64_t n, int64_t k, int64_t ldw, uint8_t *codes,
+                      uint16_t *scales, void *stream);
+
+/*
+ * tq_dequantize -- reconstruct w~ = s .* (H c) / 32 (TQ page, paragraph after
+ * 格式原理: inverse rotation and rescale).  fp32 arithmetic, output rounded
+ * to ot (nearest-even).
+ *   codes, scales  device, as written by tq_quantize for the same n, k
+ *   w_out  device, n x k of dtype ot, row stride ldo (ldo >= k, ldo % 8 == 0,
+ *          16-byte aligned)
+ */
+TQ_API tq_status tq_dequantize(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, void *w_out,
+                        tq_dtype ot, int64_t ldo, void *stream);
+
+/*
+ * Pre-rotated activations (TQ page, 解码速度 section: the activation is
+ * rotated once and shared, so the per-weight work is lookup x scale).
+ * xrot holds fp16 values H(s .* x)/32 per 32-block, in the order the fused
+ * kernel's tensor-core fragments read them: [m][NSB][4 blocks][4][8], where
+ * entry [t][q] of a block is element (q/2)*8 + 2t + (q%2).  Padding blocks
+ * are zero.  |x| must stay below 65504 (fp16 range).
+ */
+TQ_API size_t tq_xrot_bytes(int64_t m, int64_t k);
+
+/*
+ * tq_prerotate -- xrot = fragment-ordered fp16(H (s .* x) / 32) for each of the
+ * m rows of X.
+ *   X     device, m x k of dtype xt, row stride ldx (ldx >= k, ldx % 8 == 0,
+ *         16-byte aligned)
+ *   xrot  device, tq_xrot_bytes(m, k) bytes, 16-byte aligned (written)
+ */
+TQ_API tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
+                       void *stream);
+
+/* Workspace bytes needed by tq_gemm / tq_gemv (and tq_gemm_xrot, which needs
+ * the same minus the xrot area) on the CURRENT device for these sizes. */
+TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/*
+ * tq_gemm -- Y[i][r] = sum_k w~[r][k] X[i][k] for i < m, r < n, computed as
+ * (1/32) sum_blocks sum_halves d * sum_e c_e xrot_e with the activation
+ * pre-rotated once per call (TQ page, 解码速度 section).  Centroids and xrot
+ * enter the tensor cores as fp16; products accumulate in fp32.
+ *   X          device, m x k of dtype xt, row stride ldx (as tq_prerotate)
+ *   Y          device, m x n of dtype yt (F32, BF16 or F16), row stride ldy
+ *              (ldy >= n)
+ *   workspace  device, >= tq_gemm_workspace_bytes(m, n, k) bytes, 256-byte
+ *              aligned, exclusively owned by this call until it completes
+ *              on `stream` (no zero-fill needed)
+ * m <= 32 runs the skinny kernel in one pass; larger m runs it once per
+ * 32-row slice of X (weights re-read per slice).
+ */
+TQ_API tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X, tq_dtype xt,
+                  int64_t m, int64_t ldx, void *Y, tq_dtype yt, int64_t ldy, void *workspace, size_t ws_bytes,
+                  void *stream);
+
+/* tq_gemv -- tq_gemm with m = 1 (x: k elements, y: n elements). */
+TQ_API tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *x, tq_dtype xt,
+                  void *y, tq_dtype yt, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * tq_gemm_xrot -- the product with an activation already pre-rotated by
+ * tq_prerotate (one xrot shared by every matrix that consumes the same
+ * input, e.g. q/k/v).  m <= 32.  Same workspace rules as tq_gemm (no
+ * zero-fill needed: the call clears its split-K counters with one
+ * cudaMemsetAsync on `stream` before the kernel).
+ */
+TQ_API tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const uint16_t *xrot,
+                       int64_t m, void *Y, tq_dtype yt, int64_t ldy, void *workspace, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

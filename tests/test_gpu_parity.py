@@ -1,0 +1,283 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bars (TQ4_1S page "企业官网建设流程全解析": 格式原理 items 1-3, 解码速度 section):
+  * quantise: codes and fp16 scale bits identical (integer / byte work);
+  * dequantise: within a bound derived from the fp32 arithmetic (product
+    rounding + five butterfly stages, plus rounding to the output type);
+  * pre-rotation: fp16 values within 1 ulp of the fp64 transform;
+  * GEMV / GEMM: relative L2 error <= 1e-3 per output row against the fp64
+    product over the oracle's own dequantised weights.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dequant_gemv_tq4_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+REL_L2_TOL = 1e-3
+DEV = "cuda:0"
+F32, BF16, F16 = torch.float32, torch.bfloat16, torch.float16
+
+
+def _w(n, k, dtype, seed=0, std=0.02):
+    return inputs.gaussian_matrix(seed, n * 7919 + k, n, k, std, dtype)
+
+
+def _host_f32(t):
+    return t.detach().to("cpu").float().numpy()
+
+
+def _oracle_quantize(W):
+    return oracle.quantize(_host_f32(W))
+
+
+def _gpu_quantize(tq, W):
+    codes, scales = tq.quantize(W.to(DEV))
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16)
+
+
+def _rel_l2(y, ref):
+    y = np.atleast_2d(y).astype(np.float64)
+    ref = np.atleast_2d(ref)
+    num = np.linalg.norm(y - ref, axis=1)
+    den = np.maximum(np.linalg.norm(ref, axis=1), 1e-300)
+    return num / den
+
+
+QUANT_SHAPES = [(1, 32), (3, 64), (17, 96), (16, 128), (33, 160), (5, 4096), (64, 1056), (100, 384)]
+
+
+@pytest.mark.parametrize("dtype", [F32, BF16, F16])
+@pytest.mark.parametrize("n,k", QUANT_SHAPES)
+def test_quantize_bit_exact(cuda_lib, n, k, dtype):
+    W = _w(n, k, dtype)
+    c_ref, s_ref = _oracle_quantize(W)
+    c, s = _gpu_quantize(cuda_lib, W)
+    np.testing.assert_array_equal(s, s_ref)
+    np.testing.assert_array_equal(c, c_ref)
+
+
+def test_quantize_strided_and_special_values(cuda_lib):
+    n, k, ld = 12, 256, 264
+    base = torch.zeros((n, ld), dtype=F32)
+    base[:, :k] = _w(n, k, F32, seed=3)
+    base[0, :k] = 0.0                                   # all-zero row
+    base[1, :k] = 1e-30                                 # scale underflows to 0
+    base[2, :k] = 1000.0 * torch.sign(_w(1, k, F32)[0]) # large values
+    s = torch.tensor(oracle.sign(np.arange(k)).astype(np.float32))
+    base[3, :k] = -0.5 * s                              # worked block, every block
+    base[4, :k] = 3.0                                   # constant row
+    base[5, :k] = -0.0
+    W = base[:, :k]
+    c_ref, s_ref = oracle.quantize(W.numpy().copy())
+    Wd = base.to(DEV)
+    codes, scales = cuda_lib.quantize(Wd[:, :k])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
+    np.testing.assert_array_equal(scales.cpu().numpy().view(np.uint16), s_ref)
+
+
+def _dequant_bound(codes, scales, n, k, w64, out_dtype):
+    code, d = oracle.unpack(codes, scales, n, k)
+    M32, _, _ = oracle.codebook()
+    absc = M32[code & 7].astype(np.float64) * np.repeat(d.view(np.float16).astype(np.float64), 16, axis=2).reshape(n, k)
+    blk = absc.reshape(n, k // 32, 32).sum(axis=2, keepdims=True) / 32
+    arith = 8 * 2.0 ** -24 * np.broadcast_to(blk, (n, k // 32, 32)).reshape(n, k)
+    rel = {F32: 2.0 ** -24, BF16: 2.0 ** -8, F16: 2.0 ** -11}[out_dtype]
+    floor = {F32: 2.0 ** -149, BF16: 2.0 ** -133, F16: 2.0 ** -25}[out_dtype]
+    return arith * (1 + rel) + np.abs(w64) * rel + floor
+
+
+@pytest.mark.parametrize("out_dtype", [F32, BF16, F16])
+@pytest.mark.parametrize("n,k", [(3, 64), (17, 96), (33, 160), (64, 1056)])
+def test_dequantize_within_arithmetic_bound(cuda_lib, n, k, out_dtype):
+    W = _w(n, k, BF16, seed=5)
+    c_ref, s_ref = _oracle_quantize(W)
+    w64 = oracle.dequantize(c_ref, s_ref, n, k)
+    codes = torch.tensor(c_ref, device=DEV)
+    scales = torch.tensor(s_ref.view(np.int16), device=DEV)
+    out = cuda_lib.dequantize(codes, scales, n, k, dtype=out_dtype)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().astype(np.float64)
+    bound = _dequant_bound(c_ref, s_ref, n, k, w64, out_dtype)
+    err = np.abs(got - w64)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+def test_dequantize_strided_output(cuda_lib):
+    n, k, ld = 9, 128, 136
+    W = _w(n, k, F32, seed=6)
+    c_ref, s_ref = _oracle_quantize(W)
+    codes = torch.tensor(c_ref, device=DEV)
+    scales = torch.tensor(s_ref.view(np.int16), device=DEV)
+    out = torch.full((n, ld), 7.0, device=DEV)
+    cuda_lib.dequantize(codes, scales, n, k, out=out[:, :k])
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    assert np.all(o[:, k:] == 7.0)  # nothing written past k
+    w64 = oracle.dequantize(c_ref, s_ref, n, k)
+    assert np.all(np.abs(o[:, :k] - w64) <= _dequant_bound(c_ref, s_ref, n, k, w64, F32))
+
+
+@pytest.mark.parametrize("m,k", [(1, 32), (1, 4096), (3, 96), (5, 160)])
+def test_prerotate_values_and_layout(cuda_lib, m, k):
+    X = _w(m, k, BF16, seed=7, std=1.0)
+    xr = cuda_lib.prerotate(X.to(DEV))
+    torch.cuda.synchronize()
+    got = xr.cpu().numpy().view(np.float16).astype(np.float64)
+    nsb = (k // 32 + 3) // 4
+    got = got.reshape(m, nsb * 4, 4, 8)  # [row][block][t][q]
+    s = oracle.sign(np.arange(k)).astype(np.float64)
+    ref = oracle.fwht32((_host_f32(X).astype(np.float64) * s).reshape(m, k // 32, 32)) / 32
+    # entry [t][q] of a block is element (q//2)*8 + 2t + q%2
+    t_idx, q_idx = np.meshgrid(np.arange(4), np.arange(8), indexing="ij")
+    elem = (q_idx // 2) * 8 + 2 * t_idx + q_idx % 2
+    unperm = np.zeros((m, nsb * 4, 32))
+    unperm[:, :, elem] = got
+    assert np.all(unperm[:, k // 32:, :] == 0)  # padding blocks
+    r16 = ref.astype(np.float16).astype(np.float64)
+    ulp = np.spacing(np.abs(r16).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(unperm[:, : k // 32, :] - ref) <= ulp + 1e-12)
+
+
+GEMM_CASES = [
+    (1, 1, 32), (1, 15, 96), (1, 16, 128), (1, 17, 4096), (1, 1024, 4096), (2, 33, 256), (3, 64, 160),
+    (5, 40, 1024), (8, 16, 8192), (9, 48, 512), (16, 100, 384), (31, 17, 1024), (32, 64, 2048),
+    (33, 20, 256), (40, 64, 128), (4, 3, 16384),
+]
+
+
+@pytest.mark.parametrize("m,n,k", GEMM_CASES)
+def test_gemm_rel_l2(cuda_lib, m, n, k):
+    W = _w(n, k, BF16, seed=8)
+    X = _w(m, k, BF16, seed=9, std=1.0)
+    c_ref, s_ref = _oracle_quantize(W)
+    Y_ref = oracle.gemm(c_ref, s_ref, n, k, _host_f32(X))
+    codes, scales = cuda_lib.quantize(W.to(DEV))
+    Y = cuda_lib.gemm(codes, scales, n, k, X.to(DEV))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
+    assert _rel_l2(Y.cpu().numpy(), Y_ref).max() <= REL_L2_TOL
+
+
+@pytest.mark.parametrize("out_dtype", [BF16, F16])
+def test_gemv_low_precision_outputs(cuda_lib, out_dtype):
+    n, k = 300, 1024
+    W = _w(n, k, BF16, seed=10)
+    x = _w(1, k, F32, seed=11, std=1.0)[0]
+    c_ref, s_ref = _oracle_quantize(W)
+    y_ref = oracle.gemm(c_ref, s_ref, n, k, _host_f32(x)[None])[0]
+    codes, scales = cuda_lib.quantize(W.to(DEV))
+    y = cuda_lib.gemv(codes, scales, n, k, x.to(DEV), dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert _rel_l2(y.float().cpu().numpy(), y_ref).max() <= REL_L2_TOL
+
+
+def test_gemv_single_matrix_workload(cuda_lib):
+    """2048x2048 fp32 ~N(0, 0.02^2), x fp32 ~N(0,1): quantise, dequantise, GEMV."""
+    W, x = inputs.single_matrix()
+    n, k = W.shape
+    c_ref, s_ref = oracle.quantize(W.numpy())
+    Wd = W.to(DEV)
+    codes, scales = cuda_lib.quantize(Wd)
+    deq = cuda_lib.dequantize(codes, scales, n, k, dtype=F32)
+    y = cuda_lib.gemv(codes, scales, n, k, x.to(DEV))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
+    np.testing.assert_array_equal(scales.cpu().numpy().view(np.uint16), s_ref)
+    w64 = oracle.dequantize(c_ref, s_ref, n, k)
+    assert np.all(np.abs(deq.cpu().numpy() - w64) <= _dequant_bound(c_ref, s_ref, n, k, w64, F32))
+    y_ref = oracle.gemm(c_ref, s_ref, n, k, x.numpy()[None])[0]
+    assert _rel_l2(y.cpu().numpy(), y_ref)[0] <= REL_L2_TOL
+
+
+def test_gemv_deterministic_and_workspace_reuse(cuda_lib):
+    n, k = 4096, 4096
+    W = inputs.gaussian_matrix(0, 1, n, k, 0.02, BF16, DEV)
+    x = inputs.gaussian_matrix(1, 1, 1, k, 1.0, BF16, DEV)[0]
+    codes, scales = cuda_lib.quantize(W)
+    ws = cuda_lib.workspace(1, n, k)
+    y1 = cuda_lib.gemv(codes, scales, n, k, x, ws=ws).clone()
+    for _ in range(3):
+        y2 = cuda_lib.gemv(codes, scales, n, k, x, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_shared_prerotation_matches_gemm(cuda_lib):
+    """One pre-rotated activation shared by three matrices (q/k/v style)."""
+    k = 1024
+    x = _w(1, k, BF16, seed=12, std=1.0).to(DEV)
+    xr = cuda_lib.prerotate(x)
+    for n in (256, 64, 64):
+        W = _w(n, k, BF16, seed=n).to(DEV)
+        codes, scales = cuda_lib.quantize(W)
+        ws = cuda_lib.workspace(1, n, k)
+        a = cuda_lib.gemm_xrot(codes, scales, n, k, xr, 1, ws=ws)
+        b = cuda_lib.gemm(codes, scales, n, k, x)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b)
+
+
+def test_workspace_errors(cuda_lib):
+    n, k = 64, 256
+    codes, scales = cuda_lib.quantize(_w(n, k, BF16).to(DEV))
+    x = torch.zeros(k, dtype=BF16, device=DEV)
+    y = torch.zeros(n, dtype=F32, device=DEV)
+    need = cuda_lib.tq_gemm_workspace_bytes(1, n, k)
+    ws = torch.zeros(need + 512, dtype=torch.uint8, device=DEV)
+    st = cuda_lib.tq_gemv(codes.data_ptr(), scales.data_ptr(), n, k, x.data_ptr(), 1, y.data_ptr(), 0,
+                          ws.data_ptr(), need - 1, torch.cuda.current_stream().cuda_stream)
+    assert st == 5
+    st = cuda_lib.tq_gemv(codes.data_ptr(), scales.data_ptr(), n, k, x.data_ptr(), 1, y.data_ptr(), 0,
+                          ws.data_ptr() + 16, need, torch.cuda.current_stream().cuda_stream)
+    assert st == 5
+    st = cuda_lib.tq_gemv(codes.data_ptr(), scales.data_ptr(), n, k, x.data_ptr(), 1, y.data_ptr(), 0,
+                          0, need, torch.cuda.current_stream().cuda_stream)
+    assert st == 5
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, checked on sampled rows (rows are independent)
+# ---------------------------------------------------------------------------
+def _sample_rows(n, count=24, seed=0):
+    rng = np.random.default_rng(seed + n)
+    rows = np.unique(np.concatenate(([0, n - 1], rng.choice(n, count, replace=False))))
+    return rows
+
+
+def test_llama3_8b_layer_full_size(cuda_lib):
+    weights, acts = inputs.llama3_8b_layer(device=DEV)
+    for name, W in weights.items():
+        n, k = W.shape
+        x = acts[inputs.LLAMA3_8B_INPUTS[name]]
+        codes, scales = cuda_lib.quantize(W)
+        y = cuda_lib.gemv(codes, scales, n, k, x)
+        torch.cuda.synchronize()
+        rows = _sample_rows(n)
+        Wr = W[torch.tensor(rows, device=DEV)]
+        c_ref, s_ref = oracle.quantize(_host_f32(Wr))
+        np.testing.assert_array_equal(codes[torch.tensor(rows, device=DEV)].cpu().numpy(), c_ref, err_msg=name)
+        np.testing.assert_array_equal(
+            scales[torch.tensor(rows, device=DEV)].cpu().numpy().view(np.uint16), s_ref, err_msg=name)
+        y_ref = oracle.gemm(c_ref, s_ref, len(rows), k, _host_f32(x)[None])[0]
+        assert _rel_l2(y.cpu().numpy()[rows], y_ref)[0] <= REL_L2_TOL, name
+
+
+@pytest.mark.parametrize("m", [1, 2, 4, 8, 16, 32])
+def test_ffn_70b_skinny_sweep_full_size(cuda_lib, m):
+    n, k = inputs.FFN_70B["gate"]
+    W = inputs.gaussian_matrix(2, 0, n, k, 0.015, BF16, DEV)
+    X = inputs.gaussian_matrix(1, 100 + m, m, k, 1.0, BF16, DEV)
+    codes, scales = cuda_lib.quantize(W)
+    Y = cuda_lib.gemm(codes, scales, n, k, X)
+    torch.cuda.synchronize()
+    rows = _sample_rows(n, 12)
+    c_ref, s_ref = oracle.quantize(_host_f32(W[torch.tensor(rows, device=DEV)]))
+    Y_ref = oracle.gemm(c_ref, s_ref, len(rows), k, _host_f32(X))
+    assert _rel_l2(Y.cpu().numpy()[:, rows], Y_ref).max() <= REL_L2_TOL
