@@ -85,6 +85,9 @@ __global__ void __launch_bounds__(kThreads, 1) skinny_kernel(const SkinnyParams 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int gw = blockIdx.x * kWarps + warp;
+    // total_warps <= units, so every participating warp owns >= 1 unit and the
+    // contributors of a tile are exactly the warps owner(first)..owner(last)
+    if (gw >= p.total_warps) return;
     const int64_t U = p.units;
     const int64_t u0 = (int64_t)gw * U / p.total_warps;
     const int64_t u1 = (int64_t)(gw + 1) * U / p.total_warps;
@@ -276,7 +279,7 @@ SkinnyPlan plan_skinny(int64_t m, int64_t n, int64_t k, int sm_count) {
     if (want > sm_count) want = sm_count;
     if (want < 1) want = 1;
     pl.grid = (int)want;
-    pl.total_warps = pl.grid * kWarps;
+    pl.total_warps = (int)(pl.units < (int64_t)pl.grid * kWarps ? pl.units : (int64_t)pl.grid * kWarps);
     const int64_t mm = m < 1 ? 1 : (m > 32 ? 32 : m);
     pl.mcap = (int)(8 * ((mm + 7) / 8));
     pl.counter_bytes = round_up((size_t)pl.tiles * 4u, 256);

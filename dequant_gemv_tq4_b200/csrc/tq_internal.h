@@ -31,7 +31,7 @@ struct SkinnyPlan {
     int64_t tiles;        // ceil(n / 16)
     int64_t units;        // tiles * nsb
     int grid;             // CTAs
-    int total_warps;      // grid * warps per CTA
+    int total_warps;      // min(grid * warps per CTA, units): warps that own work
     int mcap;             // 8 * ceil(m / 8)
     size_t counter_bytes; // tiles * 4, rounded up to 256
     size_t partial_bytes; // (tiles + total_warps) * 16 * mcap * 4
