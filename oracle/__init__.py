@@ -68,6 +68,8 @@ def _load():
             lib.tqo_quantize_block.argtypes = [P, ctypes.c_uint32, P, P, P]
             lib.tqo_superblocks.argtypes = [I64]
             lib.tqo_superblocks.restype = I64
+            lib.tqo_tiles.argtypes = [I64]
+            lib.tqo_tiles.restype = I64
             lib.tqo_quantize.argtypes = [P, I64, I64, I64, P, P]
             lib.tqo_quantize.restype = ctypes.c_int
             lib.tqo_unpack.argtypes = [P, P, I64, I64, P, P]
@@ -155,12 +157,25 @@ def superblocks(k: int) -> int:
     return int(_load().tqo_superblocks(int(k)))
 
 
+def tiles(n: int) -> int:
+    return int(_load().tqo_tiles(int(n)))
+
+
 def codes_bytes(n: int, k: int) -> int:
-    return n * superblocks(k) * 64
+    return tiles(n) * superblocks(k) * 1024
 
 
 def scales_count(n: int, k: int) -> int:
-    return n * superblocks(k) * 8
+    return tiles(n) * superblocks(k) * 128
+
+
+def row_view(codes: np.ndarray, scales: np.ndarray, n: int, k: int):
+    """Row-major views of the tiled planes: (codes [n, NSB*64], scales [n, NSB*8]).
+    Pure re-indexing of the stored bytes (no arithmetic)."""
+    T, nsb = tiles(n), superblocks(k)
+    c = np.asarray(codes).reshape(T, nsb, 16, 64).transpose(0, 2, 1, 3).reshape(T * 16, nsb * 64)[:n]
+    s = np.asarray(scales).reshape(T, nsb, 16, 8).transpose(0, 2, 1, 3).reshape(T * 16, nsb * 8)[:n]
+    return c, s
 
 
 def quantize_block(w32: np.ndarray, k0: int):
@@ -176,13 +191,15 @@ def quantize_block(w32: np.ndarray, k0: int):
 
 
 def quantize(W: np.ndarray):
-    """W: float32 [n, k] (k % 32 == 0).  Returns (codes uint8 [n, NSB*64], scales uint16 [n, NSB*8])."""
+    """W: float32 [n, k] (k % 32 == 0).  Returns the tiled planes
+    (codes uint8 [T*NSB*1024], scales uint16 [T*NSB*128]), T = ceil(n/16)."""
     lib = _load()
     W = np.ascontiguousarray(W, dtype=np.float32)
     n, k = W.shape
-    nsb = superblocks(k)
-    codes = np.zeros((n, nsb * 64), np.uint8)
-    scales = np.zeros((n, nsb * 8), np.uint16)
+    if k % 32 != 0:
+        raise ValueError("k must be a multiple of 32")
+    codes = np.zeros(codes_bytes(n, k), np.uint8)
+    scales = np.zeros(scales_count(n, k), np.uint16)
     if lib.tqo_quantize(_ptr(W), n, k, k, _ptr(codes), _ptr(scales)) != 0:
         raise ValueError("k must be a multiple of 32")
     return codes, scales

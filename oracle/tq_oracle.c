@@ -250,34 +250,43 @@ void tqo_quantize_block(const float *w, uint32_t k0, const float *B32, uint8_t *
 /* ------------------------------------------------------------------------ */
 /* Packed layout (the repository's stated format; the pages fix only "16     */
 /* optimal centroids + clean nibble packing + no correction term", TQ page).  */
-/*   row n has NSB = ceil(K/128) superblocks; superblock sb holds blocks      */
-/*   4sb..4sb+3.  codes: 64 bytes per superblock; logical byte L (0..15) of    */
-/*   block j is code[2L] | code[2L+1] << 4 and sits at byte                   */
-/*   16*(L % 4) + 4*j + L / 4.  scales: 8 uint16 per superblock, [j][h].      */
-/*   Blocks past K/32 are zero codes with zero scales.                        */
+/*   Rows are grouped in tiles of 16 (T = ceil(N/16)); each row has           */
+/*   NSB = ceil(K/128) superblocks of four blocks.  A unit = (tile, sb) is     */
+/*   stored contiguously, units in tile-major order:                           */
+/*     codes  [T][NSB][16 rows][64 B]   scales [T][NSB][16 rows][4 blocks][2]  */
+/*   Inside a row's 64-byte superblock, logical byte L (0..15) of block j is   */
+/*   code[2L] | code[2L+1] << 4 and sits at byte 16*(L % 4) + 4*j + L / 4.     */
+/*   Blocks past K/32 and rows past N are zero codes with zero scales.        */
 /* ------------------------------------------------------------------------ */
 int64_t tqo_superblocks(int64_t k) { return (k / TQO_BLOCK + TQO_SB_BLOCKS - 1) / TQO_SB_BLOCKS; }
 
+int64_t tqo_tiles(int64_t n) { return (n + 15) / 16; }
+
+static int64_t tqo_unit_row(int64_t nsb, int64_t row, int64_t blk) {
+    int64_t sb = blk / TQO_SB_BLOCKS;
+    return ((row / 16) * nsb + sb) * 16 + row % 16; /* index of the row's 64-byte slot */
+}
+
 static int64_t tqo_code_offset(int64_t nsb, int64_t row, int64_t blk, int L) {
-    int64_t sb = blk / TQO_SB_BLOCKS, j = blk % TQO_SB_BLOCKS;
-    return (row * nsb + sb) * 64 + 16 * (L % 4) + 4 * j + L / 4;
+    int64_t j = blk % TQO_SB_BLOCKS;
+    return tqo_unit_row(nsb, row, blk) * 64 + 16 * (L % 4) + 4 * j + L / 4;
 }
 
 static int64_t tqo_scale_offset(int64_t nsb, int64_t row, int64_t blk, int h) {
-    int64_t sb = blk / TQO_SB_BLOCKS, j = blk % TQO_SB_BLOCKS;
-    return (row * nsb + sb) * 8 + 2 * j + h;
+    int64_t j = blk % TQO_SB_BLOCKS;
+    return tqo_unit_row(nsb, row, blk) * 8 + 2 * j + h;
 }
 
-/* W: fp32, n x k, leading dimension ldw (elements).  codes: n*NSB*64 bytes,
- * scales: n*NSB*8 uint16.  Returns 0, or 1 if k % 32 != 0. */
+/* W: fp32, n x k, leading dimension ldw (elements).  codes: T*NSB*1024 bytes,
+ * scales: T*NSB*128 uint16.  Returns 0, or 1 if k % 32 != 0. */
 int tqo_quantize(const float *W, int64_t n, int64_t k, int64_t ldw, uint8_t *codes, uint16_t *scales) {
     if (k % TQO_BLOCK != 0 || n < 0) return 1;
     float M32[8], B32[7];
     double M64[8];
     tqo_codebook(M32, B32, M64);
     int64_t nsb = tqo_superblocks(k), nb = k / TQO_BLOCK;
-    memset(codes, 0, (size_t)(n * nsb * 64));
-    memset(scales, 0, (size_t)(n * nsb * 8) * sizeof(uint16_t));
+    memset(codes, 0, (size_t)(tqo_tiles(n) * nsb * 1024));
+    memset(scales, 0, (size_t)(tqo_tiles(n) * nsb * 128) * sizeof(uint16_t));
     for (int64_t r = 0; r < n; ++r)
         for (int64_t b = 0; b < nb; ++b) {
             uint8_t code[TQO_BLOCK];
@@ -350,10 +359,13 @@ void tqo_dequantize(const uint8_t *codes, const uint16_t *scales, int64_t n, int
  */
 void tqo_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const double *X, int64_t m,
               int64_t ldx, double *Y, int64_t ldy) {
-    double *w = (double *)malloc((size_t)k * sizeof(double));
+    double *w = (double *)malloc((size_t)(k > 0 ? k : 1) * sizeof(double));
+    double *tile = (double *)malloc((size_t)16 * (size_t)(k > 0 ? k : 1) * sizeof(double));
     int64_t nsb = tqo_superblocks(k);
     for (int64_t r = 0; r < n; ++r) {
-        tqo_dequantize(codes + r * nsb * 64, scales + r * nsb * 8, 1, k, w, k);
+        /* dequantise the row's 16-row tile, keep row r */
+        if (r % 16 == 0) tqo_dequantize(codes + (r / 16) * nsb * 1024, scales + (r / 16) * nsb * 128, 16, k, tile, k);
+        memcpy(w, tile + (r % 16) * k, (size_t)k * sizeof(double));
         for (int64_t i = 0; i < m; ++i) {
             double acc = 0.0;
             for (int64_t c = 0; c < k; ++c) acc += w[c] * X[i * ldx + c];
@@ -361,4 +373,5 @@ void tqo_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k
         }
     }
     free(w);
+    free(tile);
 }

@@ -254,13 +254,12 @@ def test_dequantize_is_inverse_rotation(oracle_mod):
 # ---------------------------------------------------------------------------
 def test_packing_layout_and_bits_per_weight(oracle_mod):
     rng = np.random.default_rng(15)
-    for k in (32, 96, 128, 160, 4096):
-        n = 3
+    for n, k in ((3, 32), (17, 96), (16, 128), (5, 160), (20, 4096)):
         W = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
         c, s = oracle_mod.quantize(W)
-        nsb = (k // 32 + 3) // 4
-        assert c.shape == (n, nsb * 64) and s.shape == (n, nsb * 8)
-        if k % 128 == 0:
+        nsb, T = (k // 32 + 3) // 4, (n + 15) // 16
+        assert c.shape == (T * nsb * 1024,) and s.shape == (T * nsb * 128,)
+        if k % 128 == 0 and n % 16 == 0:
             assert (c.nbytes + s.nbytes) * 8 / (n * k) == 5.0
         code, d = oracle_mod.unpack(c, s, n, k)
         for r in range(n):
@@ -268,18 +267,22 @@ def test_packing_layout_and_bits_per_weight(oracle_mod):
                 cb, db = oracle_mod.quantize_block(W[r, 32 * b:32 * b + 32], 32 * b)
                 np.testing.assert_array_equal(code[r, 32 * b:32 * b + 32], cb)
                 np.testing.assert_array_equal(d[r, b], db)
-                # explicit byte positions of the stated layout
+                # explicit byte positions of the stated tiled layout
                 sb, j = divmod(b, 4)
+                slot = ((r // 16) * nsb + sb) * 16 + r % 16
                 for L in range(16):
-                    byte = c[r, sb * 64 + 16 * (L % 4) + 4 * j + L // 4]
-                    assert byte == cb[2 * L] | (cb[2 * L + 1] << 4)
-                assert s[r, sb * 8 + 2 * j] == db[0] and s[r, sb * 8 + 2 * j + 1] == db[1]
-        # padding blocks are zero
+                    assert c[slot * 64 + 16 * (L % 4) + 4 * j + L // 4] == cb[2 * L] | (cb[2 * L + 1] << 4)
+                assert s[slot * 8 + 2 * j] == db[0] and s[slot * 8 + 2 * j + 1] == db[1]
+        # padding: blocks past k/32 and rows past n hold zeros
+        rc, rs = oracle_mod.row_view(c, s, T * 16, k)
         nb = k // 32
-        for b in range(nb, nsb * 4):
-            j = b % 4
-            for L in range(16):
-                assert np.all(c[:, (nsb - 1) * 64 + 16 * (L % 4) + 4 * j + L // 4] == 0)
+        full = np.zeros((T * 16, nsb * 4), bool)
+        full[:n, :nb] = True
+        for b in range(nsb * 4):
+            sb, j = divmod(b, 4)
+            cols = [sb * 64 + 16 * (L % 4) + 4 * j + L // 4 for L in range(16)]
+            assert np.all(rc[~full[:, b]][:, cols] == 0)
+            assert np.all(rs[~full[:, b]][:, [sb * 8 + 2 * j, sb * 8 + 2 * j + 1]] == 0)
     # page: 28-42% smaller than Q8_0 (8.5 bits/weight); an all-TQ4_1S tensor is 41.2%
     assert abs((1 - 5.0 / 8.5) - 0.412) < 1e-3 and 0.28 <= 1 - 5.0 / 8.5 <= 0.42
 
