@@ -171,20 +171,19 @@ class Path:
 
     def __init__(self, tq, mats, acts, device):
         self.tq = tq
-        self.mats = mats
-        self.acts = acts
         self.items = []
-        ws_bytes = 0
         for label, W, act in mats:
             n, k = W.shape
-            nsb = tq.superblocks(k)
-            codes = torch.empty((n, nsb * 64), dtype=torch.uint8, device=device)
-            scales = torch.empty((n, nsb * 8), dtype=torch.int16, device=device)
+            codes = torch.empty(tq.tq_codes_bytes(n, k), dtype=torch.uint8, device=device)
+            scales = torch.empty(tq.tq_scales_bytes(n, k) // 2, dtype=torch.int16, device=device)
             deq = torch.empty((n, k), dtype=torch.bfloat16, device=device)
-            y = torch.empty((n,), dtype=torch.float32, device=device)
-            self.items.append(dict(label=label, W=W, x=acts[act], n=n, k=k, codes=codes, scales=scales, deq=deq, y=y))
-            ws_bytes = max(ws_bytes, tq.tq_gemm_workspace_bytes(1, n, k))
-        self.ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
+            y = torch.empty((1, n), dtype=torch.float32, device=device)
+            x = acts[act].view(1, -1)
+            self.items.append(dict(label=label, W=W, x=x, n=n, k=k, codes=codes, scales=scales, deq=deq, y=y,
+                                   ws=tq.workspace(1, n, k, device)))
+        self.batch = [(it["codes"], it["scales"], it["n"], it["k"], it["x"], it["y"]) for it in self.items]
+        self.descs = tq.batch_descs(self.batch)
+        self.ws = tq.batch_workspace(self.batch, 1, device)
 
     def quantize(self):
         for it in self.items:
@@ -195,8 +194,14 @@ class Path:
             self.tq.dequantize(it["codes"], it["scales"], it["n"], it["k"], out=it["deq"])
 
     def gemv(self):
-        for it in self.items:
-            self.tq.gemv(it["codes"], it["scales"], it["n"], it["k"], it["x"], out=it["y"], ws=self.ws)
+        """All matrices in one batch: one pre-rotation launch for the distinct
+        inputs, one fused-product launch."""
+        self.tq.gemm_batch(self.batch, m=1, ws=self.ws, descs=self.descs)
+
+    def gemv_one(self, i):
+        it = self.items[i]
+        return lambda: self.tq.gemv(it["codes"], it["scales"], it["n"], it["k"], it["x"][0], out=it["y"][0],
+                                    ws=it["ws"])
 
     def step(self):
         self.quantize()
@@ -207,14 +212,20 @@ class Path:
     def weights(self):
         return sum(it["n"] * it["k"] for it in self.items)
 
-    def packed_bytes(self):
-        return sum(it["codes"].numel() + 2 * it["scales"].numel() for it in self.items)
+    def packed_bytes(self, i=None):
+        its = self.items if i is None else [self.items[i]]
+        return sum(it["codes"].numel() + 2 * it["scales"].numel() for it in its)
 
     def in_bytes(self):
         return sum(it["W"].numel() * it["W"].element_size() for it in self.items)
 
     def act_bytes(self):
-        return sum(it["x"].numel() * it["x"].element_size() for it in self.items)
+        seen, total = set(), 0
+        for it in self.items:
+            if it["x"].data_ptr() not in seen:
+                seen.add(it["x"].data_ptr())
+                total += it["x"].numel() * it["x"].element_size()
+        return total
 
     def out_bytes(self):
         return sum(it["y"].numel() * 4 for it in self.items)
@@ -282,7 +293,7 @@ def cpu_oracle_sample(path, rows_per_matrix=None):
         n, k = it["n"], it["k"]
         r = rows_per_matrix if rows_per_matrix else max(1, n // 8)
         W = it["W"][:r].float().cpu().numpy()
-        x = it["x"].float().cpu().numpy()[None].astype(np.float64)
+        x = it["x"].float().cpu().numpy().reshape(1, -1).astype(np.float64)
         t0 = time.perf_counter()
         c, s = oracle.quantize(W)
         t1 = time.perf_counter()
@@ -310,7 +321,7 @@ def run_ours(args, world, rank, local):
     mats, acts, desc = make_workload(args.workload, rank, device)
     path = Path(tq, mats, acts, device)
     nmat = len(path.items)
-    launches_per_step = 4 * nmat  # quantize, dequantize, prerotate, fused gemv per matrix
+    launches_per_step = 2 * nmat + 2  # quantize + dequantize per matrix; one pre-rotation + one fused product
     warmup = max(3, args.warmup)
     steps = max(1, args.steps)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
@@ -346,6 +357,14 @@ def run_ours(args, world, rank, local):
     t_q = time_replays(q_run, steps, flush)
     t_d = time_replays(d_run, steps, flush)
     t_g = time_replays(g_run, steps, flush)
+    per_matrix = {}
+    for i, it in enumerate(path.items):
+        run_i = capture(path.gemv_one(i), use_graph)
+        for _ in range(warmup):
+            run_i()
+        ms_i = time_replays(run_i, steps, flush) / steps
+        per_matrix[it["label"]] = {"n": it["n"], "k": it["k"], "us": round(1e3 * ms_i, 2),
+                                   "gbs": round(path.packed_bytes(i) / (ms_i * 1e-3) / 1e9, 1)}
     barrier(world)
     clocks = sampler.stop()
     t_step, t_q, t_d, t_g = max_over_ranks([t_step, t_q, t_d, t_g], world)
@@ -362,7 +381,7 @@ def run_ours(args, world, rank, local):
     alg = {
         "quantize": (path.in_bytes() + packed, ms_q, nmat),
         "dequantize": (packed + 2 * weights, ms_d, nmat),
-        "gemv": (packed + path.act_bytes() + path.out_bytes(), ms_g, 2 * nmat),
+        "gemv": (packed + path.act_bytes() + path.out_bytes(), ms_g, 2),
     }
     rooflines = {}
     for ph, (nbytes, ms, nl) in alg.items():
@@ -383,6 +402,7 @@ def run_ours(args, world, rank, local):
         "pct_of_hbm_peak": round(100 * value / world / hbm, 2),
         "quantize_gweights_per_s": round(quant_gw, 2),
         "phases_ms": {"quantize": round(ms_q, 5), "dequantize": round(ms_d, 5), "gemv": round(ms_g, 5)},
+        "gemv_single_matrix": per_matrix,
         "roofline": dict(rooflines[dominant], kernel=dominant, peak_note=f"{hbm_kind} HBM copy bandwidth"),
         "rooflines": rooflines,
         "clocks": clocks,
@@ -405,22 +425,26 @@ def run_e2e(tq, path, steps, world):
     """Public API with host buffers: H2D of weights + activations from pinned
     memory, quantise/dequantise/GEMV, D2H of every y, per step."""
     host_w = [it["W"].cpu().pin_memory() for it in path.items]
-    host_x = [it["x"].cpu().pin_memory() for it in path.items]
     host_y = [torch.empty_like(it["y"], device="cpu").pin_memory() for it in path.items]
     dev_w = [torch.empty_like(it["W"]) for it in path.items]
-    dev_x = [torch.empty_like(it["x"]) for it in path.items]
+    # one host/device buffer per distinct activation (matrices share inputs)
+    xs = {}
+    for it in path.items:
+        xs.setdefault(it["x"].data_ptr(), (it["x"].cpu().pin_memory(), torch.empty_like(it["x"])))
+    batch = [(it["codes"], it["scales"], it["n"], it["k"], xs[it["x"].data_ptr()][1], it["y"]) for it in path.items]
+    descs = tq.batch_descs(batch)
     stream = torch.cuda.current_stream()
 
     def one():
         for i, it in enumerate(path.items):
             dev_w[i].copy_(host_w[i], non_blocking=True)
-            dev_x[i].copy_(host_x[i], non_blocking=True)
+        for hx, dx in xs.values():
+            dx.copy_(hx, non_blocking=True)
         for i, it in enumerate(path.items):
             tq.quantize(dev_w[i], it["codes"], it["scales"])
         for it in path.items:
             tq.dequantize(it["codes"], it["scales"], it["n"], it["k"], out=it["deq"])
-        for i, it in enumerate(path.items):
-            tq.gemv(it["codes"], it["scales"], it["n"], it["k"], dev_x[i], out=it["y"], ws=path.ws)
+        tq.gemm_batch(batch, m=1, ws=path.ws, descs=descs)
         for i, it in enumerate(path.items):
             host_y[i].copy_(it["y"], non_blocking=True)
 

@@ -27,7 +27,16 @@ LIB_PATH = os.path.join(_HERE, "libtq.so")
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 _DTYPE_CODE = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16, torch.float16: TQ_F16}
 STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_INVALID_ARG", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGNMENT",
-                4: "TQ_ERR_DTYPE", 5: "TQ_ERR_WORKSPACE", 6: "TQ_ERR_CUDA", 7: "TQ_ERR_UNSUPPORTED"}
+                4: "TQ_ERR_DTYPE", 5: "TQ_ERR_WORKSPACE", 6: "TQ_ERR_CUDA", 7: "TQ_ERR_UNSUPPORTED",
+                8: "TQ_ERR_TIMEOUT"}
+TQ_MAX_BATCH = 8
+
+
+class GemmDesc(ctypes.Structure):
+    """Mirror of ``tq_gemm_desc`` in include/tq.h."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("n", ctypes.c_int64),
+                ("k", ctypes.c_int64), ("X", ctypes.c_void_p), ("ldx", ctypes.c_int64), ("Y", ctypes.c_void_p),
+                ("ldy", ctypes.c_int64)]
 
 _lock = threading.Lock()
 _lib = None
@@ -61,6 +70,10 @@ def load_library() -> ctypes.CDLL:
             "tq_gemm": ([P, P, I64, I64, P, I, I64, I64, P, I, I64, P, SZ, P], I),
             "tq_gemv": ([P, P, I64, I64, P, I, P, I, P, SZ, P], I),
             "tq_gemm_xrot": ([P, P, I64, I64, P, I64, P, I, I64, P, SZ, P], I),
+            "tq_gemm_batch_workspace_bytes": ([ctypes.POINTER(GemmDesc), I, I64], SZ),
+            "tq_gemm_batch": ([ctypes.POINTER(GemmDesc), I, I64, I, I, P, SZ, P], I),
+            "tq_workspace_status": ([P, I, P], I),
+            "tq_debug_set_flags": ([ctypes.c_uint32], None),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -122,6 +135,22 @@ def tq_gemm_xrot(codes, scales, n, k, xrot, m, Y, yt, ldy, workspace, ws_bytes, 
     return load_library().tq_gemm_xrot(codes, scales, n, k, xrot, m, Y, yt, ldy, workspace, ws_bytes, stream)
 
 
+def tq_gemm_batch_workspace_bytes(descs, count, m) -> int:
+    return int(load_library().tq_gemm_batch_workspace_bytes(descs, count, m))
+
+
+def tq_gemm_batch(descs, count, m, xt, yt, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_gemm_batch(descs, count, m, xt, yt, workspace, ws_bytes, stream)
+
+
+def tq_workspace_status(workspace, clear, stream) -> int:
+    return load_library().tq_workspace_status(workspace, clear, stream)
+
+
+def tq_debug_set_flags(flags: int) -> None:
+    load_library().tq_debug_set_flags(flags)
+
+
 # ---------------------------------------------------------------------------
 # tensor helpers
 # ---------------------------------------------------------------------------
@@ -154,16 +183,20 @@ def workspace(m: int, n: int, k: int, device=None) -> torch.Tensor:
     return torch.zeros(nbytes, dtype=torch.uint8, device=device or torch.cuda.current_device())
 
 
+def tiles(n: int) -> int:
+    return (n + 15) // 16
+
+
 def quantize(w: torch.Tensor, codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
              stream=None):
-    """Encode W (n x k, fp32/bf16/fp16, on the GPU).  Returns (codes uint8 [n, NSB*64],
-    scales int16 [n, NSB*8] holding fp16 bit patterns)."""
+    """Encode W (n x k, fp32/bf16/fp16, on the GPU).  Returns the packed planes
+    (codes uint8 [T*NSB*1024], scales int16 [T*NSB*128] holding fp16 bit
+    patterns), T = ceil(n/16), in the tile-major layout of include/tq.h."""
     n, k = w.shape
-    nsb = superblocks(k)
     if codes is None:
-        codes = torch.empty((n, nsb * 64), dtype=torch.uint8, device=w.device)
+        codes = torch.empty(tq_codes_bytes(n, k), dtype=torch.uint8, device=w.device)
     if scales is None:
-        scales = torch.empty((n, nsb * 8), dtype=torch.int16, device=w.device)
+        scales = torch.empty(tq_scales_bytes(n, k) // 2, dtype=torch.int16, device=w.device)
     _check(tq_quantize(w.data_ptr(), _dt(w.dtype), n, k, _ld(w), codes.data_ptr(), scales.data_ptr(),
                        _stream(stream)), "tq_quantize")
     return codes, scales
@@ -225,3 +258,40 @@ def gemm_xrot(codes, scales, n: int, k: int, xrot: torch.Tensor, m: int, dtype=t
     _check(tq_gemm_xrot(codes.data_ptr(), scales.data_ptr(), n, k, xrot.data_ptr(), m, out.data_ptr(),
                         _dt(out.dtype), _ld(out), ws.data_ptr(), ws.numel(), _stream(stream)), "tq_gemm_xrot")
     return out
+
+
+def batch_descs(items):
+    """items: sequence of (codes, scales, n, k, X [m, k], Y [m, n]) -> ctypes array."""
+    arr = (GemmDesc * len(items))()
+    for i, (codes, scales, n, k, X, Y) in enumerate(items):
+        X2 = X.view(1, -1) if X.dim() == 1 else X
+        Y2 = Y.view(1, -1) if Y.dim() == 1 else Y
+        arr[i] = GemmDesc(codes.data_ptr(), scales.data_ptr(), n, k, X2.data_ptr(), _ld(X2), Y2.data_ptr(), _ld(Y2))
+    return arr
+
+
+def batch_workspace(items, m: int, device=None) -> torch.Tensor:
+    descs = batch_descs(items)
+    nbytes = tq_gemm_batch_workspace_bytes(descs, len(items), m)
+    if nbytes == 0:
+        raise ValueError("invalid batch for workspace query")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or torch.cuda.current_device())
+
+
+def gemm_batch(items, m: int = 1, ws=None, stream=None, descs=None):
+    """Fused products for several matrices in two launches (one pre-rotation
+    per distinct input, one product launch).  items as in ``batch_descs``;
+    the outputs Y are written in place.  All X share one dtype, all Y too."""
+    if descs is None:
+        descs = batch_descs(items)
+    X0, Y0 = items[0][4], items[0][5]
+    if ws is None:
+        ws = batch_workspace(items, m, X0.device)
+    _check(tq_gemm_batch(descs, len(items), m, _dt(X0.dtype), _dt(Y0.dtype), ws.data_ptr(), ws.numel(),
+                         _stream(stream)), "tq_gemm_batch")
+    return [it[5] for it in items]
+
+
+def workspace_status(ws: torch.Tensor, clear: bool = True, stream=None) -> int:
+    """0 (TQ_OK) or 8 (TQ_ERR_TIMEOUT) for the last product that used ``ws``."""
+    return tq_workspace_status(ws.data_ptr(), 1 if clear else 0, _stream(stream))

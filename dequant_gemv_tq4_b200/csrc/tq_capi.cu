@@ -54,22 +54,34 @@ tq_status check_planes(const uint8_t *codes, const uint16_t *scales) {
 
 tq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 
-struct GemmLayout {
-    size_t xrot_off, xrot_bytes, counter_off, partial_off, total;
-    tq::SkinnyPlan plan;
+// Workspace of a fused-product call:
+//   [0, 256)           status word (timeout flag of the last call)
+//   [256, ...)         split-K arrival counters, one per 16-row tile
+//   partial slots      (tiles + warps) * 16 * mcap floats
+//   pre-rotated inputs one area per distinct activation (calls that rotate)
+struct Layout {
+    size_t counter_off, partial_off, xrot_off[tq::kMaxInputs], total;
+    int inputs;
+    tq::GroupPlan plan;
 };
 
-// Workspace: [xrot for <= 32 rows][split-K counters][partial slots].
-tq_status gemm_layout(int64_t m, int64_t n, int64_t k, bool with_xrot, GemmLayout *lay) {
+constexpr size_t kStatusBytes = 256;
+
+tq_status make_layout(const int64_t *n, const int64_t *k, int count, const int64_t *input_k, int inputs, int64_t m,
+                      Layout *lay) {
     tq::DeviceInfo di;
     if (tq::device_info(&di) != cudaSuccess) return TQ_ERR_CUDA;
-    const int64_t ms = m > 32 ? 32 : m;
-    lay->plan = tq::plan_skinny(ms, n, k, di.sm_count);
-    lay->xrot_off = 0;
-    lay->xrot_bytes = with_xrot ? tq::round_up(tq_xrot_bytes(ms, k), 256) : 0;
-    lay->counter_off = lay->xrot_bytes;
+    const int64_t ms = m > 32 ? 32 : (m < 1 ? 1 : m);
+    lay->plan = tq::plan_group(n, k, count, ms, di.sm_count);
+    lay->counter_off = kStatusBytes;
     lay->partial_off = lay->counter_off + lay->plan.counter_bytes;
-    lay->total = lay->partial_off + lay->plan.partial_bytes;
+    size_t off = lay->partial_off + lay->plan.partial_bytes;
+    lay->inputs = inputs;
+    for (int i = 0; i < inputs; ++i) {
+        lay->xrot_off[i] = off;
+        off += tq::round_up(tq_xrot_bytes(ms, input_k[i]), 256);
+    }
+    lay->total = off;
     return TQ_OK;
 }
 
@@ -87,18 +99,19 @@ const char *tq_status_string(tq_status s) {
         case TQ_ERR_WORKSPACE: return "TQ_ERR_WORKSPACE: workspace missing, misaligned or too small";
         case TQ_ERR_CUDA: return "TQ_ERR_CUDA: a CUDA call or kernel launch failed";
         case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED: request not implemented by this build";
+        case TQ_ERR_TIMEOUT: return "TQ_ERR_TIMEOUT: a kernel's bounded wait expired (see tq_workspace_status)";
     }
     return "unknown tq_status";
 }
 
 size_t tq_codes_bytes(int64_t n, int64_t k) {
     if (check_nk(n, k) != TQ_OK) return 0;
-    return (size_t)n * (size_t)tq::superblocks(k) * 64u;
+    return (size_t)tq::tiles(n) * (size_t)tq::superblocks(k) * 1024u;
 }
 
 size_t tq_scales_bytes(int64_t n, int64_t k) {
     if (check_nk(n, k) != TQ_OK) return 0;
-    return (size_t)n * (size_t)tq::superblocks(k) * 16u;
+    return (size_t)tq::tiles(n) * (size_t)tq::superblocks(k) * 256u;
 }
 
 size_t tq_xrot_bytes(int64_t m, int64_t k) {
@@ -137,13 +150,14 @@ tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t
     if ((st = check_matrix_operand(X, ldx, k)) != TQ_OK) return st;
     if (!xrot) return TQ_ERR_INVALID_ARG;
     if (!aligned(xrot, 16)) return TQ_ERR_ALIGNMENT;
-    return from_cuda(tq::launch_prerotate(X, xt, m, k, ldx, xrot, nullptr, 0, (cudaStream_t)stream));
+    tq::RotJob job = {X, ldx, k, xrot};
+    return from_cuda(tq::launch_prerotate(&job, 1, xt, m, nullptr, 0, (cudaStream_t)stream));
 }
 
 size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 0 || check_nk(n, k) != TQ_OK) return 0;
-    GemmLayout lay;
-    if (gemm_layout(m < 1 ? 1 : m, n, k, true, &lay) != TQ_OK) return 0;
+    Layout lay;
+    if (make_layout(&n, &k, 1, &k, 1, m, &lay) != TQ_OK) return 0;
     return lay.total;
 }
 
@@ -163,6 +177,11 @@ static tq_status check_gemm_common(const uint8_t *codes, const uint16_t *scales,
     return TQ_OK;
 }
 
+static tq_status check_workspace(void *workspace, size_t ws_bytes, size_t need) {
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < need) return TQ_ERR_WORKSPACE;
+    return TQ_OK;
+}
+
 tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const uint16_t *xrot,
                        int64_t m, void *Y, tq_dtype yt, int64_t ldy, void *workspace, size_t ws_bytes, void *stream) {
     tq_status st = check_gemm_common(codes, scales, n, k, m, Y, yt, ldy);
@@ -170,17 +189,18 @@ tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, 
     if (m > 32) return TQ_ERR_SHAPE;
     if (!xrot) return TQ_ERR_INVALID_ARG;
     if (!aligned(xrot, 16)) return TQ_ERR_ALIGNMENT;
-    GemmLayout lay;
-    if ((st = gemm_layout(m, n, k, false, &lay)) != TQ_OK) return st;
-    if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return TQ_ERR_WORKSPACE;
+    Layout lay;
+    if ((st = make_layout(&n, &k, 1, nullptr, 0, m, &lay)) != TQ_OK) return st;
+    if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
     char *ws = static_cast<char *>(workspace);
-    auto *counters = reinterpret_cast<unsigned *>(ws + lay.counter_off);
-    // the arrival counters must start at zero; the workspace may have held
-    // anything (another call's partial sums or pre-rotated activations)
-    cudaError_t e = cudaMemsetAsync(counters, 0, (size_t)lay.plan.tiles * sizeof(unsigned), (cudaStream_t)stream);
-    if (e != cudaSuccess) return TQ_ERR_CUDA;
-    return from_cuda(tq::launch_skinny(codes, scales, n, k, xrot, m, Y, yt, ldy, lay.plan, counters,
-                                       reinterpret_cast<float *>(ws + lay.partial_off), true, (cudaStream_t)stream));
+    cudaStream_t s = (cudaStream_t)stream;
+    // status word and arrival counters must start at zero; the workspace may
+    // have held anything (another call's partial sums or activations)
+    if (cudaMemsetAsync(ws, 0, lay.partial_off, s) != cudaSuccess) return TQ_ERR_CUDA;
+    tq::GemvProblem pb = {codes, scales, xrot, Y, ldy, n, k};
+    return from_cuda(tq::launch_group(&pb, 1, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
+                                      reinterpret_cast<float *>(ws + lay.partial_off),
+                                      reinterpret_cast<unsigned *>(ws), true, s));
 }
 
 tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X, tq_dtype xt,
@@ -190,22 +210,23 @@ tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64
     if (st != TQ_OK || n == 0 || m == 0) return st;
     if (!valid_dtype(xt)) return TQ_ERR_DTYPE;
     if ((st = check_matrix_operand(X, ldx, k)) != TQ_OK) return st;
-    GemmLayout lay;
-    if ((st = gemm_layout(m, n, k, true, &lay)) != TQ_OK) return st;
-    if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return TQ_ERR_WORKSPACE;
+    Layout lay;
+    if ((st = make_layout(&n, &k, 1, &k, 1, m, &lay)) != TQ_OK) return st;
+    if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
     char *ws = static_cast<char *>(workspace);
-    auto *xrot = reinterpret_cast<uint16_t *>(ws + lay.xrot_off);
-    auto *counters = reinterpret_cast<unsigned *>(ws + lay.counter_off);
-    auto *partials = reinterpret_cast<float *>(ws + lay.partial_off);
+    auto *xrot = reinterpret_cast<uint16_t *>(ws + lay.xrot_off[0]);
     const size_t xsize = xt == TQ_F32 ? 4 : 2, ysize = yt == TQ_F32 ? 4 : 2;
     cudaStream_t s = (cudaStream_t)stream;
     for (int64_t i0 = 0; i0 < m; i0 += 32) {
         const int64_t ms = (m - i0) < 32 ? (m - i0) : 32;
-        const char *Xs = static_cast<const char *>(X) + (size_t)i0 * (size_t)ldx * xsize;
-        char *Ys = static_cast<char *>(Y) + (size_t)i0 * (size_t)ldy * ysize;
-        cudaError_t e = tq::launch_prerotate(Xs, xt, ms, k, ldx, xrot, counters, lay.plan.tiles, s);
+        tq::RotJob job = {static_cast<const char *>(X) + (size_t)i0 * (size_t)ldx * xsize, ldx, k, xrot};
+        // zeroes the status word and the counters that follow it
+        cudaError_t e = tq::launch_prerotate(&job, 1, xt, ms, reinterpret_cast<unsigned *>(ws),
+                                             (int64_t)(lay.partial_off / 4), s);
         if (e != cudaSuccess) return TQ_ERR_CUDA;
-        e = tq::launch_skinny(codes, scales, n, k, xrot, ms, Ys, yt, ldy, lay.plan, counters, partials, true, s);
+        tq::GemvProblem pb = {codes, scales, xrot, static_cast<char *>(Y) + (size_t)i0 * (size_t)ldy * ysize, ldy, n, k};
+        e = tq::launch_group(&pb, 1, ms, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
+                             reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true, s);
         if (e != cudaSuccess) return TQ_ERR_CUDA;
     }
     return TQ_OK;
@@ -215,5 +236,88 @@ tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n, int64
                   void *y, tq_dtype yt, void *workspace, size_t ws_bytes, void *stream) {
     return tq_gemm(codes, scales, n, k, x, xt, 1, k, y, yt, n, workspace, ws_bytes, stream);
 }
+
+// ---- batch: several matrices, one pre-rotation per distinct input ----------
+static tq_status batch_layout(const tq_gemm_desc *descs, int count, int64_t m, Layout *lay, int *input_of) {
+    int64_t n[tq::kMaxProblems], k[tq::kMaxProblems], ik[tq::kMaxInputs];
+    int inputs = 0;
+    for (int i = 0; i < count; ++i) {
+        n[i] = descs[i].n;
+        k[i] = descs[i].k;
+        int found = -1;
+        for (int j = 0; j < i; ++j)
+            if (descs[j].X == descs[i].X && descs[j].k == descs[i].k && descs[j].ldx == descs[i].ldx) {
+                found = input_of[j];
+                break;
+            }
+        if (found < 0) {
+            found = inputs;
+            ik[inputs++] = descs[i].k;
+        }
+        input_of[i] = found;
+    }
+    return make_layout(n, k, count, ik, inputs, m, lay);
+}
+
+size_t tq_gemm_batch_workspace_bytes(const tq_gemm_desc *descs, int count, int64_t m) {
+    if (!descs || count < 1 || count > TQ_MAX_BATCH || m < 0 || m > 32) return 0;
+    for (int i = 0; i < count; ++i)
+        if (check_nk(descs[i].n, descs[i].k) != TQ_OK) return 0;
+    Layout lay;
+    int input_of[tq::kMaxProblems];
+    if (batch_layout(descs, count, m, &lay, input_of) != TQ_OK) return 0;
+    return lay.total;
+}
+
+tq_status tq_gemm_batch(const tq_gemm_desc *descs, int count, int64_t m, tq_dtype xt, tq_dtype yt, void *workspace,
+                        size_t ws_bytes, void *stream) {
+    if (!descs) return TQ_ERR_INVALID_ARG;
+    if (count < 1 || count > TQ_MAX_BATCH) return TQ_ERR_SHAPE;
+    if (m < 0) return TQ_ERR_INVALID_ARG;
+    if (m > 32) return TQ_ERR_SHAPE;
+    if (!valid_dtype(xt) || !valid_dtype(yt)) return TQ_ERR_DTYPE;
+    tq_status st;
+    for (int i = 0; i < count; ++i) {
+        const tq_gemm_desc &d = descs[i];
+        if ((st = check_gemm_common(d.codes, d.scales, d.n, d.k, m, d.Y, yt, d.ldy)) != TQ_OK) return st;
+        if (d.n == 0) return TQ_ERR_SHAPE;  /* every matrix of a batch must be non-empty */
+        if (m > 0 && (st = check_matrix_operand(d.X, d.ldx, d.k)) != TQ_OK) return st;
+    }
+    if (m == 0) return TQ_OK;
+    Layout lay;
+    int input_of[tq::kMaxProblems];
+    if ((st = batch_layout(descs, count, m, &lay, input_of)) != TQ_OK) return st;
+    if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
+    char *ws = static_cast<char *>(workspace);
+    tq::RotJob jobs[tq::kMaxInputs];
+    tq::GemvProblem pbs[tq::kMaxProblems];
+    for (int i = 0; i < count; ++i) {
+        const int q = input_of[i];
+        auto *xrot = reinterpret_cast<uint16_t *>(ws + lay.xrot_off[q]);
+        jobs[q] = {descs[i].X, descs[i].ldx, descs[i].k, xrot};
+        pbs[i] = {descs[i].codes, descs[i].scales, xrot, descs[i].Y, descs[i].ldy, descs[i].n, descs[i].k};
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws),
+                                         (int64_t)(lay.partial_off / 4), s);
+    if (e != cudaSuccess) return TQ_ERR_CUDA;
+    e = tq::launch_group(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
+                         reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true, s);
+    return from_cuda(e);
+}
+
+tq_status tq_workspace_status(void *workspace, int clear, void *stream) {
+    if (!workspace) return TQ_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TQ_ERR_CUDA;
+    if (clear && word != 0) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return TQ_ERR_CUDA;
+    }
+    return word ? TQ_ERR_TIMEOUT : TQ_OK;
+}
+
+void tq_debug_set_flags(uint32_t flags) { tq::set_debug_flags(flags); }
 
 }  // extern "C"

@@ -35,6 +35,12 @@ __device__ __forceinline__ void fwht32_warp(float (&v)[4], int p) {
     }
 }
 
+// Index of a row's 64-byte code slot (and 16-byte scale slot) for superblock
+// sb in the tile-major layout [tile][sb][16 rows].
+__device__ __forceinline__ size_t unit_row(int row, int sb, int nsb) {
+    return ((size_t)(row >> 4) * nsb + sb) * 16 + (row & 15);
+}
+
 // #{j : a > t_j} for ascending t (binary search over the seven thresholds).
 __device__ __forceinline__ uint32_t magnitude_rank(float a, const float (&t)[7]) {
     const bool b2 = a > t[3];
@@ -71,9 +77,10 @@ __global__ void __launch_bounds__(kCodecThreads) quantize_kernel(const char *__r
     const int o = lane & 15, tw = o >> 2, jw = o & 3;
     const int byte_shift = 8 * (tw & 1);
 
-    for (int row = blockIdx.y * kCodecWarps + warp; row < n; row += gridDim.y * kCodecWarps) {
+    const int rows_padded = (n + 15) & ~15;  // rows past n are written as zeros
+    for (int row = blockIdx.y * kCodecWarps + warp; row < rows_padded; row += gridDim.y * kCodecWarps) {
         float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) load4<DT>(w + ((int64_t)row * ldw + col0) * ElemSize<DT>::value, v);
+        if (valid && row < n) load4<DT>(w + ((int64_t)row * ldw + col0) * ElemSize<DT>::value, v);
 #pragma unroll
         for (int i = 0; i < 4; ++i) v[i] = flip(v[i], smask[i]);
         fwht32_warp(v, p);
@@ -103,7 +110,7 @@ __global__ void __launch_bounds__(kCodecThreads) quantize_kernel(const char *__r
             const uint32_t src = __shfl_sync(kFull, c16, 8 * jw + 2 * i + (tw >> 1));
             word |= ((src >> byte_shift) & 0xffu) << (8 * i);
         }
-        const size_t sb_index = (size_t)row * nsb + sb;
+        const size_t sb_index = unit_row(row, sb, nsb);
         if (lane < 16) codes[sb_index * 16 + o] = word;
 
         const uint32_t hbits = __half_as_ushort(hd);
@@ -140,7 +147,7 @@ __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_
     const int half = p >> 2;
 
     for (int row = blockIdx.y * kCodecWarps + warp; row < n; row += gridDim.y * kCodecWarps) {
-        const size_t sb_index = (size_t)row * nsb + sb;
+        const size_t sb_index = unit_row(row, sb, nsb);
         const uint32_t cw = __ldg(codes + sb_index * 16 + (lane & 15));
         const uint32_t sw = __ldg(scales + sb_index * 4 + j);
         const uint32_t b0 = (__shfl_sync(kFull, cw, src0) >> bsh) & 0xffu;
@@ -163,43 +170,45 @@ __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_
 // -------------------------------------------------------------------------
 // Pre-rotation of activations into the fused kernel's fragment order:
 // element e of a block goes to slot t*8 + q with t = (e%8)/2, q = 2*(e/8) + e%2.
-// Also zeroes the split-K arrival counters of the product that follows.
+// Handles a list of inputs (one warp per (input, row, superblock)) and zeroes
+// the split-K arrival counters of the product that follows.
 // -------------------------------------------------------------------------
 template <int DT>
-__global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const char *__restrict__ x, int64_t ldx, int m,
-                                                                    int nb, int nsb, uint32_t *__restrict__ xrot,
-                                                                    unsigned *__restrict__ counters,
-                                                                    int64_t counters_count) {
+__global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_constant__ RotParams prm) {
     grid_dependents_launch();
     const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (int64_t i = gtid; i < counters_count; i += (int64_t)gridDim.x * blockDim.x) counters[i] = 0u;
+    for (int64_t i = gtid; i < prm.counters_count; i += (int64_t)gridDim.x * blockDim.x) prm.counters[i] = 0u;
 
     const int lane = threadIdx.x & 31;
     const int j = lane >> 3, p = lane & 7;
     const int64_t unit = (int64_t)blockIdx.x * kCodecWarps + (threadIdx.x >> 5);
-    if (unit >= (int64_t)m * nsb) return;
-    const int row = (int)(unit / nsb), sb = (int)(unit % nsb);
-    const bool valid = sb * kSbBlocks + j < nb;
+    if (unit >= prm.units) return;
+    int q = 0;
+    while (q + 1 < prm.count && unit >= prm.in[q + 1].unit_begin) ++q;
+    const RotInput &in = prm.in[q];
+    const int64_t local = unit - in.unit_begin;
+    const int row = (int)(local / in.nsb), sb = (int)(local % in.nsb);
+    const bool valid = sb * kSbBlocks + j < in.nb;
     const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (valid) load4<DT>(x + ((int64_t)row * ldx + col0) * ElemSize<DT>::value, v);
+    if (valid) load4<DT>(in.x + ((int64_t)row * in.ldx + col0) * ElemSize<DT>::value, v);
 #pragma unroll
     for (int i = 0; i < 4; ++i) v[i] = flip(v[i], sign_mask(col0 + i));
     fwht32_warp(v, p);
     const __half2 lo = __floats2half2_rn(__fmul_rn(v[0], 0.03125f), __fmul_rn(v[1], 0.03125f));
     const __half2 hi = __floats2half2_rn(__fmul_rn(v[2], 0.03125f), __fmul_rn(v[3], 0.03125f));
     // elements 4p, 4p+1 -> t = 2(p&1), q = 2(p>>1) + {0,1}; 4p+2, 4p+3 -> t + 1
-    const size_t blk_words = ((size_t)unit * kSbBlocks + j) * 16;  // 32 halves per block
+    const size_t blk_words = ((size_t)local * kSbBlocks + j) * 16;  // 32 halves per block
     const int t0 = 2 * (p & 1), q0 = 2 * (p >> 1);
-    xrot[blk_words + (t0 * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&lo);
-    xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
+    in.xrot[blk_words + (t0 * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&lo);
+    in.xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
 }
 
 int rows_grid(int64_t n, int64_t nsb, int sm_count) {
     // aim for ~8 resident CTAs per SM in total, at least one warp-row per CTA
     int64_t target = (int64_t)sm_count * 8;
     int64_t gy = (target + nsb - 1) / nsb;
-    int64_t max_gy = (n + kCodecWarps - 1) / kCodecWarps;
+    int64_t max_gy = (((n + 15) & ~(int64_t)15) + kCodecWarps - 1) / kCodecWarps;
     if (gy > max_gy) gy = max_gy;
     if (gy > 65535) gy = 65535;
     if (gy < 1) gy = 1;
@@ -246,19 +255,31 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int6
     return cudaGetLastError();
 }
 
-cudaError_t launch_prerotate(const void *X, int dtype, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
-                             unsigned *counters, int64_t counters_count, cudaStream_t stream) {
-    const int64_t nb = k / 32, nsb = superblocks(k);
-    int64_t units = m * nsb;
+cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *counters,
+                             int64_t counters_count, cudaStream_t stream) {
+    if (count < 1 || count > kMaxInputs) return cudaErrorInvalidValue;
+    RotParams prm = {};
+    int64_t units = 0;
+    for (int i = 0; i < count; ++i) {
+        RotInput &in = prm.in[i];
+        in.x = static_cast<const char *>(jobs[i].x);
+        in.xrot = reinterpret_cast<uint32_t *>(jobs[i].xrot);
+        in.ldx = jobs[i].ldx;
+        in.unit_begin = units;
+        in.nb = (int)(jobs[i].k / 32);
+        in.nsb = (int)superblocks(jobs[i].k);
+        units += m * in.nsb;
+    }
+    prm.count = count;
+    prm.units = units;
+    prm.counters = counters;
+    prm.counters_count = counters ? counters_count : 0;
     int64_t grid = (units + kCodecWarps - 1) / kCodecWarps;
     if (grid < 1) grid = 1;
-    auto *xr = reinterpret_cast<uint32_t *>(xrot);
-    const char *xp = static_cast<const char *>(X);
-    if (!counters) counters_count = 0;
     switch (dtype) {
-        case kF32: prerotate_kernel<kF32><<<(unsigned)grid, kCodecThreads, 0, stream>>>(xp, ldx, (int)m, (int)nb, (int)nsb, xr, counters, counters_count); break;
-        case kBF16: prerotate_kernel<kBF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(xp, ldx, (int)m, (int)nb, (int)nsb, xr, counters, counters_count); break;
-        case kF16: prerotate_kernel<kF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(xp, ldx, (int)m, (int)nb, (int)nsb, xr, counters, counters_count); break;
+        case kF32: prerotate_kernel<kF32><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
+        case kBF16: prerotate_kernel<kBF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
+        case kF16: prerotate_kernel<kF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

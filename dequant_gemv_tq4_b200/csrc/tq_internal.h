@@ -8,6 +8,9 @@
 
 namespace tq {
 
+constexpr int kMaxInputs = 8;    // distinct activations pre-rotated by one launch
+constexpr int kMaxProblems = 8;  // matrices in one fused-product launch
+
 struct DeviceInfo {
     int device;
     int sm_count;
@@ -16,34 +19,74 @@ struct DeviceInfo {
 // Current device and its SM count (cached per device).
 cudaError_t device_info(DeviceInfo *out);
 
+inline int64_t superblocks(int64_t k) { return (k / 32 + 3) / 4; }
+inline int64_t tiles(int64_t n) { return (n + 15) / 16; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
 cudaError_t launch_quantize(const void *w, int dtype, int64_t n, int64_t k, int64_t ldw, uint8_t *codes,
                             uint16_t *scales, cudaStream_t stream);
 
 cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, void *w_out,
                               int dtype, int64_t ldo, cudaStream_t stream);
 
-// xrot for m rows; also zeroes `counters` (count entries) when non-null.
-cudaError_t launch_prerotate(const void *X, int dtype, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
-                             unsigned *counters, int64_t counters_count, cudaStream_t stream);
+// ---- pre-rotation ----------------------------------------------------------
+struct RotInput {  // device-side description of one activation matrix
+    const char *x;
+    uint32_t *xrot;
+    int64_t ldx;
+    int64_t unit_begin;  // first warp unit (row, superblock) of this input
+    int nb;
+    int nsb;
+};
 
-// Skinny product for m <= 32 rows of pre-rotated activations.
-struct SkinnyPlan {
-    int64_t tiles;        // ceil(n / 16)
-    int64_t units;        // tiles * nsb
-    int grid;             // CTAs
+struct RotParams {
+    RotInput in[kMaxInputs];
+    int count;
+    int64_t units;
+    unsigned *counters;
+    int64_t counters_count;
+};
+
+struct RotJob {  // host-side request
+    const void *x;
+    int64_t ldx;
+    int64_t k;
+    uint16_t *xrot;
+};
+
+// xrot for m rows of every job (same dtype); also zeroes `counters`.
+cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *counters,
+                             int64_t counters_count, cudaStream_t stream);
+
+// ---- fused product ---------------------------------------------------------
+struct GemvProblem {  // host-side request, m <= 32 rows of pre-rotated activations
+    const uint8_t *codes;
+    const uint16_t *scales;
+    const uint16_t *xrot;
+    void *y;
+    int64_t ldy;
+    int64_t n;
+    int64_t k;
+};
+
+struct GroupPlan {
+    int64_t units;        // sum over problems of tiles * nsb
+    int64_t tiles;        // sum over problems of ceil(n / 16)
+    int grid;             // CTAs (<= SM count)
     int total_warps;      // min(grid * warps per CTA, units): warps that own work
     int mcap;             // 8 * ceil(m / 8)
     size_t counter_bytes; // tiles * 4, rounded up to 256
-    size_t partial_bytes; // (tiles + total_warps) * 16 * mcap * 4
+    size_t partial_bytes; // (tiles + total_warps) * 16 * mcap * 4, rounded up to 256
 };
 
-SkinnyPlan plan_skinny(int64_t m, int64_t n, int64_t k, int sm_count);
+GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, int sm_count);
 
-cudaError_t launch_skinny(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const uint16_t *xrot,
-                          int64_t m, void *Y, int dtype, int64_t ldy, const SkinnyPlan &plan, unsigned *counters,
-                          float *partials, bool programmatic, cudaStream_t stream);
+// Debug hooks (tq_debug_set_flags): bit 0 makes one bulk copy go missing so
+// the kernel's bounded wait expires and reports a timeout.
+void set_debug_flags(uint32_t flags);
 
-inline int64_t superblocks(int64_t k) { return (k / 32 + 3) / 4; }
-inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
+                         unsigned *counters, float *partials, unsigned *status, bool programmatic,
+                         cudaStream_t stream);
 
 }  // namespace tq

@@ -27,17 +27,20 @@
  *  - n == 0 or m == 0 is an empty problem: TQ_OK, nothing launched.
  *  - All results are deterministic run to run (no floating-point atomics).
  *
- * Packed format (5.0 bits per weight when K % 128 == 0):
+ * Packed format (5.0 bits per weight when N % 16 == 0 and K % 128 == 0):
  *  - code: 4 bits; bit 3 = sign (1 = negative), bits 0-2 = magnitude rank
  *    0..7 into the eight positive Lloyd-Max centroids.
  *  - superblock = four consecutive 32-element blocks of one row (128
- *    columns).  Row r has NSB = ceil(K/128) superblocks; blocks past K/32 in
- *    the last one are padding (zero codes, zero scales).
- *  - codes plane: uint8 [N][NSB][64].  Within a superblock, logical byte L
- *    (0..15) of block j (0..3) holds the codes of elements 2L (low nibble)
- *    and 2L+1 (high nibble) and is stored at byte 16*(L%4) + 4*j + L/4.
- *  - scales plane: uint16 [N][NSB][4][2], IEEE fp16 bit patterns d0, d1 of
- *    each block: d_h = fp16(sqrt(mean of the 16 squared rotated values)).
+ *    columns); NSB = ceil(K/128).  Rows are grouped in tiles of 16
+ *    (T = ceil(N/16)).  A unit = (tile, superblock) is stored contiguously and
+ *    units are tile-major, so the fused kernel streams 1024 + 256 contiguous
+ *    bytes per unit.  Blocks past K/32 and rows past N are zero.
+ *  - codes plane: uint8 [T][NSB][16 rows][64].  Within a row's 64 bytes,
+ *    logical byte L (0..15) of block j (0..3) holds the codes of elements 2L
+ *    (low nibble) and 2L+1 (high nibble) and is stored at byte
+ *    16*(L%4) + 4*j + L/4.
+ *  - scales plane: uint16 [T][NSB][16 rows][4 blocks][2], IEEE fp16 bit
+ *    patterns d0, d1: d_h = fp16(sqrt(mean of the 16 squared rotated values)).
  *  - rotation: y = H (s .* w) per block, H the unnormalised 32x32 Sylvester
  *    Hadamard matrix; s_k = -1 where bit 31 of hash(k) is set, with
  *    hash(k) = g(k * 0x9E3779B9) and g(h) = ((h ^ h>>16) * 0x85EBCA6B) ^ (...>>13)
@@ -68,7 +71,8 @@ typedef enum {
     TQ_ERR_DTYPE = 4,       /* unknown tq_dtype value */
     TQ_ERR_WORKSPACE = 5,   /* workspace null or smaller than the *_workspace_bytes query */
     TQ_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
-    TQ_ERR_UNSUPPORTED = 7  /* valid request that this build does not implement */
+    TQ_ERR_UNSUPPORTED = 7, /* valid request that this build does not implement */
+    TQ_ERR_TIMEOUT = 8      /* a kernel's bounded wait expired (tq_workspace_status) */
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
@@ -76,12 +80,14 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 /* Largest supported sizes (checked; TQ_ERR_SHAPE above them). */
 #define TQ_MAX_N ((int64_t)1 << 30)
 #define TQ_MAX_K ((int64_t)1 << 26)
+#define TQ_MAX_BATCH 8
 
 /* Human-readable name of a status code (static string, never NULL). */
 TQ_API const char *tq_status_string(tq_status s);
 
 /* Bytes of the codes plane / of the scales plane for an N x K matrix
- * (n * ceil(k/128) * 64 and n * ceil(k/128) * 16).  0 for invalid sizes. */
+ * (ceil(n/16) * ceil(k/128) * 1024 and ceil(n/16) * ceil(k/128) * 256).
+ * 0 for invalid sizes. */
 TQ_API size_t tq_codes_bytes(int64_t n, int64_t k);
 TQ_API size_t tq_scales_bytes(int64_t n, int64_t k);
 
@@ -134,8 +140,10 @@ TQ_API size_t tq_xrot_bytes(int64_t m, int64_t k);
 TQ_API tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
                        void *stream);
 
-/* Workspace bytes needed by tq_gemm / tq_gemv (and tq_gemm_xrot, which needs
- * the same minus the xrot area) on the CURRENT device for these sizes. */
+/* Workspace bytes needed by tq_gemm / tq_gemv / tq_gemm_xrot on the CURRENT
+ * device for these sizes (the split-K partition depends on its SM count).
+ * Layout: a status word (256 bytes), split-K counters, partial sums and the
+ * pre-rotated activation. */
 TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -148,7 +156,8 @@ TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *              (ldy >= n)
  *   workspace  device, >= tq_gemm_workspace_bytes(m, n, k) bytes, 256-byte
  *              aligned, exclusively owned by this call until it completes
- *              on `stream` (no zero-fill needed)
+ *              on `stream` (no zero-fill needed; calls that overlap on the
+ *              GPU must use different workspaces)
  * m <= 32 runs the skinny kernel in one pass; larger m runs it once per
  * 32-row slice of X (weights re-read per slice).
  */
@@ -169,6 +178,52 @@ TQ_API tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n
  */
 TQ_API tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const uint16_t *xrot,
                        int64_t m, void *Y, tq_dtype yt, int64_t ldy, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Several matrices in one launch (TQ page, paragraph 适用前提与边界: the
+ * attention tensors of a layer share one in-place rotation, i.e. matrices
+ * that consume the same input can share one pre-rotated activation).
+ * Every descriptor is one product Y = X w~^T with its own codes/scales;
+ * descriptors with the same X pointer, k and ldx share one pre-rotation.
+ * One launch pre-rotates every distinct input, one launch computes every
+ * product (no per-matrix launch overhead).
+ */
+typedef struct {
+    const uint8_t *codes;   /* device, packed planes of an n x k matrix */
+    const uint16_t *scales;
+    int64_t n;              /* >= 1 */
+    int64_t k;              /* positive multiple of 32 */
+    const void *X;          /* device, m x k activations (dtype xt), row stride ldx */
+    int64_t ldx;
+    void *Y;                /* device, m x n outputs (dtype yt), row stride ldy */
+    int64_t ldy;
+} tq_gemm_desc;
+
+/* Workspace bytes for tq_gemm_batch on the current device (0 if invalid). */
+TQ_API size_t tq_gemm_batch_workspace_bytes(const tq_gemm_desc *descs, int count, int64_t m);
+
+/* tq_gemm_batch -- count (1..TQ_MAX_BATCH) products with m <= 32 activation
+ * rows each; the same argument rules as tq_gemm per descriptor. */
+TQ_API tq_status tq_gemm_batch(const tq_gemm_desc *descs, int count, int64_t m, tq_dtype xt, tq_dtype yt,
+                               void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * tq_workspace_status -- synchronises `stream`, then reports whether the last
+ * product that used this workspace hit a bounded wait (TQ_ERR_TIMEOUT: the
+ * kernel gave up on a bulk copy after ~1 s, recorded it and returned; its
+ * outputs are then incomplete).  clear != 0 resets the flag.  The flag is
+ * also reset by the next tq_gemm / tq_gemv / tq_gemm_xrot / tq_gemm_batch
+ * on the workspace.
+ */
+TQ_API tq_status tq_workspace_status(void *workspace, int clear, void *stream);
+
+/*
+ * tq_debug_set_flags -- test hook, process-wide, 0 by default.  Bit 0: in
+ * later fused-product launches one bulk copy of the first warp is never
+ * issued, so its bounded wait expires after ~5 ms and the timeout path runs
+ * (status word set, kernel returns normally; no fault, no trap).
+ */
+TQ_API void tq_debug_set_flags(uint32_t flags);
 
 #ifdef __cplusplus
 }

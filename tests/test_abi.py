@@ -12,7 +12,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "tq.h")
 
-OK, INVALID, SHAPE, ALIGN, DTYPE, WORKSPACE, CUDA, UNSUP = range(8)
+OK, INVALID, SHAPE, ALIGN, DTYPE, WORKSPACE, CUDA, UNSUP, TIMEOUT = range(9)
 FAKE = 1 << 20  # never dereferenced: every call using it fails validation first
 
 
@@ -35,7 +35,8 @@ def test_header_declares_the_boundary():
     names = declared_symbols()
     for required in ("tq_quantize", "tq_dequantize", "tq_gemv", "tq_gemm", "tq_prerotate", "tq_gemm_xrot",
                      "tq_codes_bytes", "tq_scales_bytes", "tq_xrot_bytes", "tq_gemm_workspace_bytes",
-                     "tq_status_string"):
+                     "tq_status_string", "tq_gemm_batch", "tq_gemm_batch_workspace_bytes", "tq_workspace_status",
+                     "tq_debug_set_flags"):
         assert required in names
 
 
@@ -52,17 +53,17 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         s = lib.tq_status_string(code).decode()
         assert s.startswith("TQ_")
     assert lib.tq_status_string(99).decode() == "unknown tq_status"
 
 
 def test_size_queries(lib):
-    assert lib.tq_codes_bytes(3, 128) == 3 * 64
-    assert lib.tq_scales_bytes(3, 128) == 3 * 16
-    assert lib.tq_codes_bytes(2, 160) == 2 * 2 * 64  # ragged last superblock is padded
-    assert lib.tq_scales_bytes(2, 160) == 2 * 2 * 16
+    assert lib.tq_codes_bytes(3, 128) == 1024      # rows padded to a 16-row tile
+    assert lib.tq_scales_bytes(3, 128) == 256
+    assert lib.tq_codes_bytes(17, 160) == 2 * 2 * 1024  # two tiles, ragged last superblock padded
+    assert lib.tq_scales_bytes(17, 160) == 2 * 2 * 256
     assert lib.tq_codes_bytes(14336, 4096) + lib.tq_scales_bytes(14336, 4096) == 14336 * 4096 * 5 // 8
     assert lib.tq_xrot_bytes(1, 4096) == 4096 * 2
     assert lib.tq_xrot_bytes(3, 96) == 3 * 128 * 2
@@ -123,6 +124,33 @@ def test_gemm_argument_errors(lib):
     assert x(FAKE, FAKE, 8, 64, FAKE, 33, FAKE, 0, 8, FAKE, 1 << 20, None) == SHAPE
     assert x(FAKE, FAKE, 8, 64, None, 2, FAKE, 0, 8, FAKE, 1 << 20, None) == INVALID
     assert x(FAKE, FAKE, 8, 64, FAKE + 2, 2, FAKE, 0, 8, FAKE, 1 << 20, None) == ALIGN
+
+
+def test_batch_argument_errors(lib):
+    import dequant_gemv_tq4_b200 as tq
+
+    def descs(*specs):
+        arr = (tq.GemmDesc * max(1, len(specs)))()
+        for i, (codes, scales, n, k, X, ldx, Y, ldy) in enumerate(specs):
+            arr[i] = tq.GemmDesc(codes, scales, n, k, X, ldx, Y, ldy)
+        return arr
+
+    good = (FAKE, FAKE, 64, 128, FAKE, 128, FAKE, 64)
+    b = lib.tq_gemm_batch
+    assert b(None, 1, 1, 1, 0, FAKE, 1 << 20, None) == INVALID
+    assert b(descs(good), 0, 1, 1, 0, FAKE, 1 << 20, None) == SHAPE
+    assert b(descs(*[good] * 9), 9, 1, 1, 0, FAKE, 1 << 20, None) == SHAPE
+    assert b(descs(good), 1, 33, 1, 0, FAKE, 1 << 20, None) == SHAPE
+    assert b(descs(good), 1, -1, 1, 0, FAKE, 1 << 20, None) == INVALID
+    assert b(descs(good), 1, 1, 5, 0, FAKE, 1 << 20, None) == DTYPE
+    assert b(descs(good, (FAKE, FAKE, 64, 100, FAKE, 128, FAKE, 64)), 2, 1, 1, 0, FAKE, 1 << 20, None) == SHAPE
+    assert b(descs(good, (FAKE, FAKE, 0, 128, FAKE, 128, FAKE, 64)), 2, 1, 1, 0, FAKE, 1 << 20, None) == SHAPE
+    assert b(descs((None, FAKE, 64, 128, FAKE, 128, FAKE, 64)), 1, 1, 1, 0, FAKE, 1 << 20, None) == INVALID
+    assert b(descs((FAKE, FAKE, 64, 128, FAKE + 4, 128, FAKE, 64)), 1, 1, 1, 0, FAKE, 1 << 20, None) == ALIGN
+    assert b(descs(good), 1, 0, 1, 0, FAKE, 1 << 20, None) == OK  # m = 0: nothing launched
+    assert lib.tq_gemm_batch_workspace_bytes(None, 1, 1) == 0
+    assert lib.tq_gemm_batch_workspace_bytes(descs(good), 1, 33) == 0
+    assert lib.tq_workspace_status(None, 0, None) == INVALID
 
 
 def test_binding_has_no_cpu_fallback(monkeypatch, tmp_path):

@@ -265,9 +265,10 @@ def test_llama3_8b_layer_full_size(cuda_lib):
         rows = _sample_rows(n)
         Wr = W[torch.tensor(rows, device=DEV)]
         c_ref, s_ref = oracle.quantize(_host_f32(Wr))
-        np.testing.assert_array_equal(codes[torch.tensor(rows, device=DEV)].cpu().numpy(), c_ref, err_msg=name)
-        np.testing.assert_array_equal(
-            scales[torch.tensor(rows, device=DEV)].cpu().numpy().view(np.uint16), s_ref, err_msg=name)
+        gc, gs = oracle.row_view(codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16), n, k)
+        rc, rs = oracle.row_view(c_ref, s_ref, len(rows), k)
+        np.testing.assert_array_equal(gc[rows], rc, err_msg=name)
+        np.testing.assert_array_equal(gs[rows], rs, err_msg=name)
         y_ref = oracle.gemm(c_ref, s_ref, len(rows), k, _host_f32(x)[None])[0]
         assert _rel_l2(y.cpu().numpy()[rows], y_ref)[0] <= REL_L2_TOL, name
 
@@ -284,3 +285,49 @@ def test_ffn_70b_skinny_sweep_full_size(cuda_lib, m):
     c_ref, s_ref = oracle.quantize(_host_f32(W[torch.tensor(rows, device=DEV)]))
     Y_ref = oracle.gemm(c_ref, s_ref, len(rows), k, _host_f32(X))
     assert _rel_l2(Y.cpu().numpy()[:, rows], Y_ref).max() <= REL_L2_TOL
+
+
+@pytest.mark.parametrize("m", [1, 5])
+def test_gemm_batch_shares_prerotation(cuda_lib, m):
+    """Six matrices with three distinct inputs in one batch (q/k/v-style and
+    gate/up-style sharing) against the oracle and the one-matrix path."""
+    shapes = [(256, 1024, "a"), (64, 1024, "a"), (64, 1024, "a"), (300, 512, "b"), (300, 512, "b"), (40, 2048, "c")]
+    Xs = {name: _w(m, k, BF16, seed=20 + i, std=1.0) for i, (_, k, name) in enumerate(shapes)}
+    items, refs, singles = [], [], []
+    for i, (n, k, name) in enumerate(shapes):
+        W = _w(n, k, BF16, seed=30 + i)
+        c_ref, s_ref = _oracle_quantize(W)
+        refs.append(oracle.gemm(c_ref, s_ref, n, k, _host_f32(Xs[name])))
+        codes, scales = cuda_lib.quantize(W.to(DEV))
+        X = Xs[name]
+        Xd = X.to(DEV) if name not in [it[6] for it in items] else [it[4] for it in items if it[6] == name][0]
+        Y = torch.empty((m, n), dtype=F32, device=DEV)
+        items.append((codes, scales, n, k, Xd, Y, name))
+        singles.append(cuda_lib.gemm(codes, scales, n, k, Xd))
+    cuda_lib.gemm_batch([it[:6] for it in items], m=m)
+    torch.cuda.synchronize()
+    for (codes, scales, n, k, Xd, Y, name), ref, single in zip(items, refs, singles):
+        assert _rel_l2(Y.cpu().numpy(), ref).max() <= REL_L2_TOL
+        np.testing.assert_allclose(Y.cpu().numpy(), single.cpu().numpy(), rtol=1e-5, atol=1e-6)
+
+
+def test_timeout_path_reports_and_recovers(cuda_lib):
+    """Fault injection on the host side of the contract: one bulk copy is never
+    issued, the kernel's bounded wait (5 ms under injection) expires, it sets
+    the workspace status word and returns; the context stays usable."""
+    n, k = 4096, 4096
+    W = inputs.gaussian_matrix(0, 3, n, k, 0.02, BF16, DEV)
+    x = inputs.gaussian_matrix(1, 3, 1, k, 1.0, BF16, DEV)[0]
+    codes, scales = cuda_lib.quantize(W)
+    ws = cuda_lib.workspace(1, n, k)
+    y_good = cuda_lib.gemv(codes, scales, n, k, x, ws=ws).clone()
+    assert cuda_lib.workspace_status(ws) == 0
+    try:
+        cuda_lib.tq_debug_set_flags(1)
+        cuda_lib.gemv(codes, scales, n, k, x, ws=ws)
+        assert cuda_lib.workspace_status(ws) == 8  # TQ_ERR_TIMEOUT
+    finally:
+        cuda_lib.tq_debug_set_flags(0)
+    y = cuda_lib.gemv(codes, scales, n, k, x, ws=ws)
+    assert cuda_lib.workspace_status(ws) == 0
+    assert torch.equal(y, y_good)
