@@ -48,15 +48,28 @@ constexpr int kStages = 6;
 constexpr int kUnitCodeBytes = 1024;
 constexpr int kUnitScaleBytes = 256;
 constexpr int kUnitBytes = kUnitCodeBytes + kUnitScaleBytes;
-constexpr int kLutBytes = 256 * 256;  // 256 entries x 256 B (32 lanes x 4 B used)
-constexpr int kRingBytes = kWarps * kStages * kUnitBytes;
-constexpr int kBarBytes = kWarps * kStages * 8;
-constexpr int kSmemBytes = kLutBytes + kRingBytes + kBarBytes;
+constexpr int kRingWarpBytes = kStages * kUnitBytes;  // 7680
+// Shared-memory map (addresses in the CTA's shared window; the dynamic
+// allocation starts at a small base B <= kMaxSmemBase):
+//   [B, B + 8 rings)            rings of warps 0..7
+//   [0x10000, 0x20000)          lookup table, 64 KB aligned so that one PRMT
+//                               yields the full address of an entry
+//   [0x20000, + 8 rings)        rings of warps 8..15
+//   then the mbarriers
+constexpr uint32_t kLutAddr = 0x10000;
+constexpr uint32_t kMaxSmemBase = 0x10000 - 8 * kRingWarpBytes;  // 4096
+constexpr uint32_t kHighRings = 0x20000;
+constexpr uint32_t kBarAddr = kHighRings + 8 * kRingWarpBytes;
+constexpr uint32_t kBarBytes = kWarps * kStages * 8;
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusLayout = 2u;
 constexpr uint64_t kTimeoutNs = 1000000000ull;     // 1 s
 constexpr uint64_t kDebugTimeoutNs = 5000000ull;   // 5 ms under fault injection
 
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert(kWarps == 16, "the shared-memory map places 8 rings below and 8 above the table");
+
+// Dynamic shared memory to request for a dynamic base of `base` bytes.
+inline uint32_t smem_bytes_for_base(uint32_t base) { return kBarAddr + kBarBytes - base; }
 
 __constant__ uint16_t c_mag_f16[8] = TQ_MAG_F16_INIT;
 
@@ -100,8 +113,6 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -121,8 +132,7 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Wait for phase `parity` of the barrier; false after `timeout_ns` (or 2^30 polls).
-__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
-    if (mbar_try(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
     const uint64_t t0 = global_ns();
     for (uint32_t it = 0; it < (1u << 30); ++it) {
         if (mbar_try(bar, parity)) return true;
@@ -131,21 +141,20 @@ __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, ui
     return false;
 }
 
-// One unit (1024 code bytes + 256 scale bytes) into a ring stage.
-__device__ __forceinline__ void issue_unit(const GroupParams &P, int64_t v, uint32_t dst, uint32_t bar) {
-    int q = 0;
-    while (q + 1 < P.count && v >= P.prob[q + 1].unit_begin) ++q;
-    const int64_t local = v - P.prob[q].unit_begin;
-    const uint8_t *src_c = P.prob[q].codes + local * kUnitCodeBytes;
-    const uint8_t *src_s = P.prob[q].scales + local * kUnitScaleBytes;
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kUnitBytes) : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src_c), "r"(kUnitCodeBytes), "r"(bar)
-                 : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     dst + kUnitCodeBytes),
-                 "l"(src_s), "r"(kUnitScaleBytes), "r"(bar)
-                 : "memory");
+// One unit (1024 code bytes + 256 scale bytes) into a ring stage, issued by
+// the lanes for which `pred` is set (one lane), without a branch.
+__device__ __forceinline__ void issue_unit_pred(uint32_t pred, const uint8_t *src_c, const uint8_t *src_s,
+                                                uint32_t dst, uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %0, 0;\n\t"
+        "@p fence.proxy.async.shared::cta;\n\t"
+        "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n\t"
+        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%3], [%4], %5, [%1];\n\t"
+        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%6], [%7], %8, [%1];\n\t}" ::"r"(pred),
+        "r"(bar), "r"(kUnitBytes), "r"(dst), "l"(src_c), "r"(kUnitCodeBytes), "r"(dst + kUnitCodeBytes), "l"(src_s),
+        "r"(kUnitScaleBytes)
+        : "memory");
 }
 
 __device__ __forceinline__ float h2f_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
@@ -156,15 +165,51 @@ __device__ __forceinline__ int owner_warp(int64_t x, int64_t units, int warps) {
     return (int)(((x + 1) * (int64_t)warps - 1) / units);
 }
 
+// Producer cursor: the next unit this warp will copy, walked incrementally.
+struct Cursor {
+    const uint8_t *c;
+    const uint8_t *s;
+    int64_t left;  // units left in the current problem
+    int q;
+};
+
+__device__ __forceinline__ Cursor cursor_at(const GroupParams &P, int64_t v) {
+    int q = 0;
+    while (q + 1 < P.count && v >= P.prob[q + 1].unit_begin) ++q;
+    const int64_t local = v - P.prob[q].unit_begin;
+    const int64_t end = (q + 1 < P.count) ? P.prob[q + 1].unit_begin : P.units;
+    Cursor cu;
+    cu.c = P.prob[q].codes + local * kUnitCodeBytes;
+    cu.s = P.prob[q].scales + local * kUnitScaleBytes;
+    cu.left = end - v;
+    cu.q = q;
+    return cu;
+}
+
+__device__ __forceinline__ void cursor_next(const GroupParams &P, Cursor &cu) {
+    cu.c += kUnitCodeBytes;
+    cu.s += kUnitScaleBytes;
+    if (--cu.left == 0 && cu.q + 1 < P.count) {
+        ++cu.q;
+        cu.c = P.prob[cu.q].codes;
+        cu.s = P.prob[cu.q].scales;
+        const int64_t end = (cu.q + 1 < P.count) ? P.prob[cu.q + 1].unit_begin : P.units;
+        cu.left = end - P.prob[cu.q].unit_begin;
+    }
+}
+
 template <int NT, bool M1, int OT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gw = blockIdx.x * kWarps + warp;
-    const uint32_t smem_base = (uint32_t)__cvta_generic_to_shared(smem);
-    const uint32_t ring = smem_base + kLutBytes + warp * (kStages * kUnitBytes);
-    const uint32_t bars = smem_base + kLutBytes + kRingBytes + warp * (kStages * 8);
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(smem);
+    if (base > kMaxSmemBase) {  // layout precondition (checked, never expected)
+        if (threadIdx.x == 0) atomicOr(P.status, kStatusLayout);
+        return;
+    }
+    const uint32_t ring = (warp < 8 ? base : kHighRings) + (warp & 7) * kRingWarpBytes;
+    const uint32_t bars = kBarAddr + warp * (kStages * 8);
     const bool active = gw < P.total_warps;
     const int64_t U = P.units;
     const int64_t u0 = active ? (int64_t)gw * U / P.total_warps : 0;
@@ -173,193 +218,224 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     // ---- prologue: barriers, first bulk copies, lookup table -------------
     // (the packed weights never depend on the preceding grid, so the copies
     // start before the programmatic-dependency wait)
-    if (active && lane == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(bars + 8 * i, 1);
-        fence_mbar_init();
-        for (int i = 0; i < kStages; ++i) {
-            const int64_t v = u0 + i;
-            if (v < u1 && !(P.inject_skip && gw == 0 && i == 1))
-                issue_unit(P, v, ring + i * kUnitBytes, bars + 8 * i);
+    Cursor cu = {nullptr, nullptr, 0, 0};
+    int64_t pv = u0;  // next unit to copy
+    if (active) {
+        if (lane == 0) {
+            for (int i = 0; i < kStages; ++i) mbar_init(bars + 8 * i, 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        cu = cursor_at(P, u0);
+        for (int i = 0; i < kStages && pv < u1; ++i, ++pv) {
+            const bool skip = P.inject_skip && gw == 0 && i == 1;
+            issue_unit_pred(lane == 0 && !skip, cu.c, cu.s, ring + i * kUnitBytes, bars + 8 * i);
+            cursor_next(P, cu);
         }
     }
-    for (int idx = threadIdx.x; idx < 256 * 32; idx += kThreads) {
-        const int v = idx >> 5, l = idx & 31;
-        const uint32_t lo = c_mag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
-        const uint32_t hi = c_mag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
-        lut[v * 64 + l] = lo | (hi << 16);
+    {
+        uint32_t *lut = reinterpret_cast<uint32_t *>(smem + (kLutAddr - base));
+        for (int idx = threadIdx.x; idx < 256 * 32; idx += kThreads) {
+            const int v = idx >> 5, l = idx & 31;
+            const uint32_t lo = c_mag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
+            const uint32_t hi = c_mag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
+            lut[v * 64 + l] = lo | (hi << 16);
+        }
     }
     __syncthreads();
     grid_dependency_wait();  // pre-rotated activations and counters are ready
     if (!active) return;
 
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t lane4 = (uint32_t)lane * 4u;
+    // PRMT operand: byte 0 = lane*4, bytes 2..3 = table base >> 16
+    const uint32_t lut_lane = kLutAddr | ((uint32_t)lane * 4u);
     constexpr int kMcap = 8 * NT;
 
     int q = 0;
     while (q + 1 < P.count && u0 >= P.prob[q + 1].unit_begin) ++q;
-    int nsb = P.prob[q].nsb;
-    int64_t r;
-    int sb;
-    {
-        const int64_t local = u0 - P.prob[q].unit_begin;
-        r = local / nsb;
-        sb = (int)(local % nsb);
-    }
-    int64_t prob_end = (q + 1 < P.count) ? P.prob[q + 1].unit_begin : U;
-
-    float acc[NT][4];
-#pragma unroll
-    for (int a = 0; a < NT; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-
+    int64_t u = u0;
     int stage = 0;
     uint32_t parity = 0;
-    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-    for (int64_t u = u0; u < u1; ++u) {
-        const uint32_t st = ring + stage * kUnitBytes, bar = bars + 8 * stage;
-        const bool ok = mbar_wait_bounded(bar, parity, P.timeout_ns);
-        if (!__all_sync(kFull, ok)) {
-            // report, then let the copies still in flight land before leaving
-            if (lane == 0) {
-                atomicOr(P.status, kStatusTimeout);
-                int s2 = stage;
-                uint32_t p2 = parity;
-                for (int64_t v = u + 1; v < u1 && v < u + kStages; ++v) {
-                    if (++s2 == kStages) { s2 = 0; p2 ^= 1u; }
-                    mbar_wait_bounded(bars + 8 * s2, p2, P.timeout_ns);
+
+    while (u < u1) {
+        // ---- one tile segment: units u .. seg_end-1 share the 16 rows --------
+        const DevProblem &pr = P.prob[q];
+        const int nsb = pr.nsb;
+        const int64_t local = u - pr.unit_begin;
+        const int64_t r = local / nsb;
+        const int sb0 = (int)(local % nsb);
+        const int64_t tile_lo = pr.unit_begin + r * nsb, tile_hi = tile_lo + nsb;
+        const int64_t seg_end = tile_hi < u1 ? tile_hi : u1;
+        // activation fragments: rows past m repeat row m-1 (their outputs are
+        // never stored), so every lane loads without a predicate
+        const uint16_t *xbase[NT];
+#pragma unroll
+        for (int a = 0; a < NT; ++a) {
+            const int xrow = min(8 * a + g, P.m - 1);
+            xbase[a] = pr.xrot + (int64_t)xrow * nsb * 128 + t * 8;
+        }
+
+        float acc[NT][4];
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+
+        int sb = sb0;
+        for (; u < seg_end; ++u, ++sb) {
+            const uint32_t st = ring + stage * kUnitBytes, bar = bars + 8 * stage;
+            bool ok = mbar_try(bar, parity);
+            if (!__all_sync(kFull, ok)) {
+                ok = ok || mbar_wait_slow(bar, parity, P.timeout_ns);
+                if (!__all_sync(kFull, ok)) {
+                    // report, then let the copies still in flight land before leaving
+                    if (lane == 0) {
+                        atomicOr(P.status, kStatusTimeout);
+                        int s2 = stage;
+                        uint32_t p2 = parity;
+                        for (int64_t v = u + 1; v < pv; ++v) {
+                            if (++s2 == kStages) { s2 = 0; p2 ^= 1u; }
+                            mbar_wait_slow(bars + 8 * s2, p2, P.timeout_ns);
+                        }
+                    }
+                    __syncwarp();
+                    return;
                 }
             }
+            const uint4 c0 = lds128(st + g * 64 + t * 16);
+            const uint4 c1 = lds128(st + (g + 8) * 64 + t * 16);
+            const uint4 s0 = lds128(st + kUnitCodeBytes + g * 16);
+            const uint4 s1 = lds128(st + kUnitCodeBytes + (g + 8) * 16);
             __syncwarp();
-            return;
-        }
-        const uint4 c0 = lds128(st + g * 64 + t * 16);
-        const uint4 c1 = lds128(st + (g + 8) * 64 + t * 16);
-        const uint4 s0 = lds128(st + kUnitCodeBytes + g * 16);
-        const uint4 s1 = lds128(st + kUnitCodeBytes + (g + 8) * 16);
-        __syncwarp();
-        if (lane == 0 && u + kStages < u1) {
-            fence_proxy_async();
-            issue_unit(P, u + kStages, st, bar);
-        }
-        if (++stage == kStages) { stage = 0; parity ^= 1u; }
-
-        const uint16_t *xr = P.prob[q].xrot;
-        const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
-        const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
-        const uint32_t sw0[4] = {s0.x, s0.y, s0.z, s0.w};
-        const uint32_t sw1[4] = {s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-        for (int j = 0; j < kSbBlocks; ++j) {
-            uint4 xb[NT];
-#pragma unroll
-            for (int a = 0; a < NT; ++a) {
-                const int xrow = 8 * a + g;
-                xb[a] = (xrow < P.m) ? ldg_keep(xr + (((int64_t)xrow * nsb + sb) * kSbBlocks + j) * 32 + t * 8) : z4;
+            if (pv < u1) {  // warp-uniform
+                issue_unit_pred(lane == 0, cu.c, cu.s, st, bar);
+                cursor_next(P, cu);
+                ++pv;
             }
-            // code byte b of word cw: logical byte t + 4b of the block
-            const uint32_t a00 = lds_u32(smem_base + prmt(cw0[j], lane4, 0x5504u));
-            const uint32_t a01 = lds_u32(smem_base + prmt(cw1[j], lane4, 0x5504u));
-            const uint32_t a02 = lds_u32(smem_base + prmt(cw0[j], lane4, 0x5514u));
-            const uint32_t a03 = lds_u32(smem_base + prmt(cw1[j], lane4, 0x5514u));
-            const uint32_t a10 = lds_u32(smem_base + prmt(cw0[j], lane4, 0x5524u));
-            const uint32_t a11 = lds_u32(smem_base + prmt(cw1[j], lane4, 0x5524u));
-            const uint32_t a12 = lds_u32(smem_base + prmt(cw0[j], lane4, 0x5534u));
-            const uint32_t a13 = lds_u32(smem_base + prmt(cw1[j], lane4, 0x5534u));
-            const float d0g = h2f_lo(sw0[j]), d1g = h2f_hi(sw0[j]);
-            const float d0g8 = h2f_lo(sw1[j]), d1g8 = h2f_hi(sw1[j]);
+            if (++stage == kStages) { stage = 0; parity ^= 1u; }
+
+            const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
+            const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+            const uint32_t sw0[4] = {s0.x, s0.y, s0.z, s0.w};
+            const uint32_t sw1[4] = {s1.x, s1.y, s1.z, s1.w};
+            const int xoff = sb * 128;
 #pragma unroll
-            for (int a = 0; a < NT; ++a) {
-                float d[4];
-                mma_16816_zero(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
-                acc[a][0] = fmaf(d[0], d0g, acc[a][0]);
-                acc[a][2] = fmaf(d[2], d0g8, acc[a][2]);
-                if (!M1) {
-                    acc[a][1] = fmaf(d[1], d0g, acc[a][1]);
-                    acc[a][3] = fmaf(d[3], d0g8, acc[a][3]);
-                }
-                mma_16816_zero(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
-                acc[a][0] = fmaf(d[0], d1g, acc[a][0]);
-                acc[a][2] = fmaf(d[2], d1g8, acc[a][2]);
-                if (!M1) {
-                    acc[a][1] = fmaf(d[1], d1g, acc[a][1]);
-                    acc[a][3] = fmaf(d[3], d1g8, acc[a][3]);
+            for (int j = 0; j < kSbBlocks; ++j) {
+                uint4 xb[NT];
+#pragma unroll
+                for (int a = 0; a < NT; ++a) xb[a] = ldg_keep(xbase[a] + xoff + j * 32);
+                // code byte b of word cw: logical byte t + 4b of the block
+                const uint32_t a00 = lds_u32(prmt(cw0[j], lut_lane, 0x7604u));
+                const uint32_t a01 = lds_u32(prmt(cw1[j], lut_lane, 0x7604u));
+                const uint32_t a02 = lds_u32(prmt(cw0[j], lut_lane, 0x7614u));
+                const uint32_t a03 = lds_u32(prmt(cw1[j], lut_lane, 0x7614u));
+                const uint32_t a10 = lds_u32(prmt(cw0[j], lut_lane, 0x7624u));
+                const uint32_t a11 = lds_u32(prmt(cw1[j], lut_lane, 0x7624u));
+                const uint32_t a12 = lds_u32(prmt(cw0[j], lut_lane, 0x7634u));
+                const uint32_t a13 = lds_u32(prmt(cw1[j], lut_lane, 0x7634u));
+                const float d0g = h2f_lo(sw0[j]), d1g = h2f_hi(sw0[j]);
+                const float d0g8 = h2f_lo(sw1[j]), d1g8 = h2f_hi(sw1[j]);
+#pragma unroll
+                for (int a = 0; a < NT; ++a) {
+                    float d[4];
+                    mma_16816_zero(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
+                    acc[a][0] = fmaf(d[0], d0g, acc[a][0]);
+                    acc[a][2] = fmaf(d[2], d0g8, acc[a][2]);
+                    if (!M1) {
+                        acc[a][1] = fmaf(d[1], d0g, acc[a][1]);
+                        acc[a][3] = fmaf(d[3], d0g8, acc[a][3]);
+                    }
+                    mma_16816_zero(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
+                    acc[a][0] = fmaf(d[0], d1g, acc[a][0]);
+                    acc[a][2] = fmaf(d[2], d1g8, acc[a][2]);
+                    if (!M1) {
+                        acc[a][1] = fmaf(d[1], d1g, acc[a][1]);
+                        acc[a][3] = fmaf(d[3], d1g8, acc[a][3]);
+                    }
                 }
             }
         }
 
-        // ---- end of a tile segment: write Y or combine partial sums --------
-        if (sb == nsb - 1 || u + 1 == u1) {
-            const DevProblem &pr = P.prob[q];
-            const int64_t tile_lo = pr.unit_begin + r * nsb, tile_hi = tile_lo + nsb;
-            const int64_t gt = pr.tile_begin + r;
-            const int row_g = (int)(r * 16) + g, row_g8 = row_g + 8;
-            if (u0 <= tile_lo && tile_hi <= u1) {
-#pragma unroll
-                for (int a = 0; a < NT; ++a)
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        if (M1 && (b & 1)) continue;
-                        const int xrow = 8 * a + 2 * t + (b & 1);
-                        const int wrow = (b & 2) ? row_g8 : row_g;
-                        if (xrow < P.m && wrow < pr.n)
-                            store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, acc[a][b]);
-                    }
-            } else {
-                float *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
-#pragma unroll
-                for (int a = 0; a < NT; ++a)
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const int xrow = 8 * a + 2 * t + (b & 1);
-                        const int wrow = g + ((b & 2) ? 8 : 0);
-                        slot[xrow * 16 + wrow] = acc[a][b];
-                    }
-                __threadfence();
-                __syncwarp();
-                const int first = owner_warp(tile_lo, U, P.total_warps);
-                const int last = owner_warp(tile_hi - 1, U, P.total_warps);
-                unsigned arrived = 0;
-                if (lane == 0) arrived = atomicAdd(P.counters + gt, 1u);
-                arrived = __shfl_sync(kFull, arrived, 0);
-                if (arrived == (unsigned)(last - first)) {
-                    __threadfence();
-                    for (int e = lane; e < 16 * P.m; e += 32) {
-                        const int xrow = e >> 4, wl = e & 15;
-                        float sum = 0.f;
-                        for (int c = first; c <= last; ++c)
-                            sum += __ldcg(P.partials + (gt + c) * (int64_t)(16 * kMcap) + xrow * 16 + wl);
-                        const int wrow = (int)(r * 16) + wl;
-                        if (wrow < pr.n)
-                            store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
-                    }
-                    if (lane == 0) P.counters[gt] = 0u;
-                }
-            }
+        // ---- end of the segment: write Y or combine partial sums ------------
+        const int64_t gt = pr.tile_begin + r;
+        const int row_g = (int)(r * 16) + g, row_g8 = row_g + 8;
+        if (u0 <= tile_lo && tile_hi <= u1) {
 #pragma unroll
             for (int a = 0; a < NT; ++a)
 #pragma unroll
-                for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+                for (int b = 0; b < 4; ++b) {
+                    if (M1 && (b & 1)) continue;
+                    const int xrow = 8 * a + 2 * t + (b & 1);
+                    const int wrow = (b & 2) ? row_g8 : row_g;
+                    if (xrow < P.m && wrow < pr.n)
+                        store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, acc[a][b]);
+                }
+        } else {
+            float *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
+#pragma unroll
+            for (int a = 0; a < NT; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int xrow = 8 * a + 2 * t + (b & 1);
+                    const int wrow = g + ((b & 2) ? 8 : 0);
+                    slot[xrow * 16 + wrow] = acc[a][b];
+                }
+            __threadfence();
+            __syncwarp();
+            const int first = owner_warp(tile_lo, U, P.total_warps);
+            const int last = owner_warp(tile_hi - 1, U, P.total_warps);
+            unsigned arrived = 0;
+            if (lane == 0) arrived = atomicAdd(P.counters + gt, 1u);
+            arrived = __shfl_sync(kFull, arrived, 0);
+            if (arrived == (unsigned)(last - first)) {
+                __threadfence();
+                for (int e = lane; e < 16 * P.m; e += 32) {
+                    const int xrow = e >> 4, wl = e & 15;
+                    const float *src = P.partials + (gt + first) * (int64_t)(16 * kMcap) + xrow * 16 + wl;
+                    const int cnt = last - first + 1;
+                    // eight independent loads in flight, added in slot order
+                    float sum = 0.f;
+                    int c = 0;
+                    for (; c + 8 <= cnt; c += 8) {
+                        float v[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + (int64_t)(c + i) * (16 * kMcap));
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) sum += v[i];
+                    }
+                    for (; c < cnt; ++c) sum += __ldcg(src + (int64_t)c * (16 * kMcap));
+                    const int wrow = (int)(r * 16) + wl;
+                    if (wrow < pr.n) store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
+                }
+                if (lane == 0) P.counters[gt] = 0u;
+            }
         }
-
-        // ---- advance (superblock, tile, problem) ---------------------------
-        if (++sb == nsb) {
-            sb = 0;
-            ++r;
-        }
-        if (u + 1 == prob_end && q + 1 < P.count) {
-            ++q;
-            nsb = P.prob[q].nsb;
-            r = 0;
-            sb = 0;
-            prob_end = (q + 1 < P.count) ? P.prob[q + 1].unit_begin : U;
-        }
+        // next segment: same problem, or the next one when this one is done
+        if (u < u1 && u == ((q + 1 < P.count) ? P.prob[q + 1].unit_begin : U)) ++q;
     }
+}
+
+// Base offset of dynamic shared memory in a CTA's shared window (the
+// per-block reserved system area), queried once per device.
+uint32_t dynamic_smem_base() {
+    static uint32_t cached[256];
+    static bool have[256];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return 1024;
+    if (!have[dev]) {
+        int reserved = 0;
+        if (cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+            reserved = 1024;
+        cached[dev] = (uint32_t)reserved;
+        have[dev] = true;
+    }
+    return cached[dev];
 }
 
 template <int NT, bool M1>
 cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programmatic, cudaStream_t stream) {
+    const uint32_t smem = smem_bytes_for_base(dynamic_smem_base());
+    const int kSmemBytes = (int)smem;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
