@@ -73,6 +73,7 @@ tq_status make_layout(const int64_t *n, const int64_t *k, int count, const int64
     if (tq::device_info(&di) != cudaSuccess) return TQ_ERR_CUDA;
     const int64_t ms = m > 32 ? 32 : (m < 1 ? 1 : m);
     lay->plan = tq::plan_group(n, k, count, ms, di.sm_count);
+    if (lay->plan.units >= ((int64_t)1 << 31)) return TQ_ERR_SHAPE;  // > 2^42 weights per call
     lay->counter_off = kStatusBytes;
     lay->partial_off = lay->counter_off + lay->plan.counter_bytes;
     size_t off = lay->partial_off + lay->plan.partial_bytes;

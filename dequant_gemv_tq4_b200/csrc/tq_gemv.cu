@@ -91,8 +91,9 @@ struct GroupParams {
     DevProblem prob[kMaxProblems];
     int count;
     int m;
-    int64_t units;
-    int total_warps;
+    int64_t units;    // < 2^31 (checked on the host)
+    int chunk;        // units per warp: warp w owns [w*chunk, min(units, (w+1)*chunk))
+    int total_warps;  // ceil(units / chunk)
     float *partials;
     unsigned *counters;
     unsigned *status;
@@ -157,13 +158,7 @@ __device__ __forceinline__ void issue_unit_pred(uint32_t pred, const uint8_t *sr
         : "memory");
 }
 
-__device__ __forceinline__ float h2f_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
-__device__ __forceinline__ float h2f_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
-// Warp that owns unit x under the even split of `units` over `warps`.
-__device__ __forceinline__ int owner_warp(int64_t x, int64_t units, int warps) {
-    return (int)(((x + 1) * (int64_t)warps - 1) / units);
-}
 
 // Producer cursor: the next unit this warp will copy, walked incrementally.
 struct Cursor {
@@ -211,15 +206,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     const uint32_t ring = (warp < 8 ? base : kHighRings) + (warp & 7) * kRingWarpBytes;
     const uint32_t bars = kBarAddr + warp * (kStages * 8);
     const bool active = gw < P.total_warps;
-    const int64_t U = P.units;
-    const int64_t u0 = active ? (int64_t)gw * U / P.total_warps : 0;
-    const int64_t u1 = active ? (int64_t)(gw + 1) * U / P.total_warps : 0;
+    const int U = (int)P.units;
+    const int chunk = P.chunk;
+    const int u0 = active ? gw * chunk : 0;
+    const int u1 = active ? min(U, u0 + chunk) : 0;
 
     // ---- prologue: barriers, first bulk copies, lookup table -------------
     // (the packed weights never depend on the preceding grid, so the copies
     // start before the programmatic-dependency wait)
     Cursor cu = {nullptr, nullptr, 0, 0};
-    int64_t pv = u0;  // next unit to copy
+    int pv = u0;  // next unit to copy
     if (active) {
         if (lane == 0) {
             for (int i = 0; i < kStages; ++i) mbar_init(bars + 8 * i, 1);
@@ -234,13 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         }
     }
     {
-        uint32_t *lut = reinterpret_cast<uint32_t *>(smem + (kLutAddr - base));
-        for (int idx = threadIdx.x; idx < 256 * 32; idx += kThreads) {
-            const int v = idx >> 5, l = idx & 31;
-            const uint32_t lo = c_mag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
-            const uint32_t hi = c_mag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
-            lut[v * 64 + l] = lo | (hi << 16);
-        }
+        // entry v holds the same half2 in all 32 lane slots: 8 x 16-byte stores
+        // per entry, two threads per entry
+        uint4 *lut = reinterpret_cast<uint4 *>(smem + (kLutAddr - base));
+        const int v = threadIdx.x >> 1, part = threadIdx.x & 1;
+        const uint32_t lo = c_mag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
+        const uint32_t hi = c_mag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
+        const uint32_t e = lo | (hi << 16);
+        const uint4 e4 = make_uint4(e, e, e, e);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) lut[v * 16 + part * 4 + i] = e4;
     }
     __syncthreads();
     grid_dependency_wait();  // pre-rotated activations and counters are ready
@@ -253,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
 
     int q = 0;
     while (q + 1 < P.count && u0 >= P.prob[q + 1].unit_begin) ++q;
-    int64_t u = u0;
+    int u = u0;
     int stage = 0;
     uint32_t parity = 0;
 
@@ -261,11 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         // ---- one tile segment: units u .. seg_end-1 share the 16 rows --------
         const DevProblem &pr = P.prob[q];
         const int nsb = pr.nsb;
-        const int64_t local = u - pr.unit_begin;
-        const int64_t r = local / nsb;
-        const int sb0 = (int)(local % nsb);
-        const int64_t tile_lo = pr.unit_begin + r * nsb, tile_hi = tile_lo + nsb;
-        const int64_t seg_end = tile_hi < u1 ? tile_hi : u1;
+        const int ub = (int)pr.unit_begin;
+        const int local = u - ub;
+        const int r = local / nsb;
+        const int sb0 = local - r * nsb;
+        const int tile_lo = ub + r * nsb, tile_hi = tile_lo + nsb;
+        const int seg_end = min(tile_hi, u1);
         // activation fragments: rows past m repeat row m-1 (their outputs are
         // never stored), so every lane loads without a predicate
         const uint16_t *xbase[NT];
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                         atomicOr(P.status, kStatusTimeout);
                         int s2 = stage;
                         uint32_t p2 = parity;
-                        for (int64_t v = u + 1; v < pv; ++v) {
+                        for (int v = u + 1; v < pv; ++v) {
                             if (++s2 == kStages) { s2 = 0; p2 ^= 1u; }
                             mbar_wait_slow(bars + 8 * s2, p2, P.timeout_ns);
                         }
@@ -333,8 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                 const uint32_t a11 = lds_u32(prmt(cw1[j], lut_lane, 0x7624u));
                 const uint32_t a12 = lds_u32(prmt(cw0[j], lut_lane, 0x7634u));
                 const uint32_t a13 = lds_u32(prmt(cw1[j], lut_lane, 0x7634u));
-                const float d0g = h2f_lo(sw0[j]), d1g = h2f_hi(sw0[j]);
-                const float d0g8 = h2f_lo(sw1[j]), d1g8 = h2f_hi(sw1[j]);
+                const float2 dg = __half22float2(*reinterpret_cast<const __half2 *>(&sw0[j]));
+                const float2 dg8 = __half22float2(*reinterpret_cast<const __half2 *>(&sw1[j]));
+                const float d0g = dg.x, d1g = dg.y, d0g8 = dg8.x, d1g8 = dg8.y;
 #pragma unroll
                 for (int a = 0; a < NT; ++a) {
                     float d[4];
@@ -358,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
 
         // ---- end of the segment: write Y or combine partial sums ------------
         const int64_t gt = pr.tile_begin + r;
-        const int row_g = (int)(r * 16) + g, row_g8 = row_g + 8;
+        const int row_g = r * 16 + g, row_g8 = row_g + 8;
         if (u0 <= tile_lo && tile_hi <= u1) {
 #pragma unroll
             for (int a = 0; a < NT; ++a)
@@ -382,8 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                 }
             __threadfence();
             __syncwarp();
-            const int first = owner_warp(tile_lo, U, P.total_warps);
-            const int last = owner_warp(tile_hi - 1, U, P.total_warps);
+            const int first = tile_lo / chunk;
+            const int last = (tile_hi - 1) / chunk;
             unsigned arrived = 0;
             if (lane == 0) arrived = atomicAdd(P.counters + gt, 1u);
             arrived = __shfl_sync(kFull, arrived, 0);
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                         for (int i = 0; i < 8; ++i) sum += v[i];
                     }
                     for (; c < cnt; ++c) sum += __ldcg(src + (int64_t)c * (16 * kMcap));
-                    const int wrow = (int)(r * 16) + wl;
+                    const int wrow = r * 16 + wl;
                     if (wrow < pr.n) store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
                 }
                 if (lane == 0) P.counters[gt] = 0u;
@@ -481,9 +482,10 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
     int64_t want = (pl.units + kWarps - 1) / kWarps;  // at least one unit per warp
     if (want > sm_count) want = sm_count;
     if (want < 1) want = 1;
-    pl.grid = (int)want;
-    const int64_t warps = (int64_t)pl.grid * kWarps;
-    pl.total_warps = (int)(pl.units < warps ? pl.units : warps);
+    const int64_t warps = want * kWarps;
+    pl.chunk = (pl.units + warps - 1) / warps;
+    pl.total_warps = (int)((pl.units + pl.chunk - 1) / pl.chunk);
+    pl.grid = (pl.total_warps + kWarps - 1) / kWarps;
     const int64_t mm = m < 1 ? 1 : (m > 32 ? 32 : m);
     pl.mcap = (int)(8 * ((mm + 7) / 8));
     pl.counter_bytes = round_up((size_t)pl.tiles * 4u, 256);
@@ -513,7 +515,9 @@ cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydt
     }
     prm.count = count;
     prm.m = (int)m;
+    if (ub != plan.units || ub >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     prm.units = ub;
+    prm.chunk = (int)plan.chunk;
     prm.total_warps = plan.total_warps;
     prm.partials = partials;
     prm.counters = counters;
