@@ -142,7 +142,7 @@ def make_workload(name: str, rank: int, device):
     mats = []  # (label, W, activation name)
     acts = {}
     if name == "llama3_8b_layer":
-        weights, acts = inputs.llama3_8b_layer(seed=100 * rank, device=device)
+        weights, acts = inputs.llama3_8b_layer(seed=rank_seed(rank), device=device)
         for label, W in weights.items():
             mats.append((label, W, inputs.LLAMA3_8B_INPUTS[label]))
         desc = {"workload": "llama3_8b_layer", "shapes": {k: list(v) for k, v in inputs.LLAMA3_8B_LAYER.items()},
@@ -155,7 +155,7 @@ def make_workload(name: str, rank: int, device):
                 "x": "fp32 ~N(0,1)", "m": 1}
     else:
         for tid, (label, (n, k)) in enumerate(inputs.FFN_70B.items()):
-            mats.append((label, inputs.gaussian_matrix(2 + 100 * rank, tid, n, k, 0.015, torch.bfloat16, device),
+            mats.append((label, inputs.gaussian_matrix(2 + rank_seed(rank), tid, n, k, 0.015, torch.bfloat16, device),
                          "x_" + label))
             acts["x_" + label] = inputs.gaussian_matrix(1, 200 + tid, 1, k, 1.0, torch.bfloat16, device)[0]
         desc = {"workload": "ffn_70b", "shapes": {k: list(v) for k, v in inputs.FFN_70B.items()},
@@ -262,14 +262,27 @@ def time_replays(run, reps: int, flush=None):
     return sum(s.elapsed_time(e) for s, e in zip(starts, ends))
 
 
+def rank_seed(rank: int) -> int:
+    """Layer seed of a rank: every rank quantises and multiplies its own layer
+    (independent problems, weak scaling, no collective on the data path)."""
+    return 100 * rank
+
+
 def max_over_ranks(values, world):
+    """Element-wise max of per-rank timings (NCCL on GPU ranks, gloo on CPU)."""
     if world == 1:
-        return values
+        return list(values)
     import torch.distributed as dist
 
-    t = torch.tensor(values, dtype=torch.float64, device=torch.cuda.current_device())
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.tolist()
+
+
+def job_gbs(bytes_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the bytes all ranks processed / the slowest rank's time."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
 
 
 def barrier(world):
@@ -277,7 +290,8 @@ def barrier(world):
         import torch.distributed as dist
 
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def cpu_oracle_sample(path, rows_per_matrix=None):
@@ -374,8 +388,8 @@ def run_ours(args, world, rank, local):
     packed = path.packed_bytes()
     weights = path.weights()
     hbm, hbm_kind = measured_peaks()
-    value = world * packed / (ms_g * 1e-3) / 1e9
-    quant_gw = world * weights / (ms_q * 1e-3) / 1e9
+    value = job_gbs(packed, world, ms_g)
+    quant_gw = job_gbs(weights, world, ms_q)
 
     # algorithmic bytes per phase (one GPU)
     alg = {

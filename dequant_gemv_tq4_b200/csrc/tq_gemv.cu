@@ -92,8 +92,7 @@ struct GroupParams {
     int count;
     int m;
     int64_t units;    // < 2^31 (checked on the host)
-    int chunk;        // units per warp: warp w owns [w*chunk, min(units, (w+1)*chunk))
-    int total_warps;  // ceil(units / chunk)
+    int total_warps;  // <= units: warp w owns [w*units/W, (w+1)*units/W)
     float *partials;
     unsigned *counters;
     unsigned *status;
@@ -143,13 +142,15 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint6
 }
 
 // One unit (1024 code bytes + 256 scale bytes) into a ring stage, issued by
-// the lanes for which `pred` is set (one lane), without a branch.
+// the lanes for which `pred` is set (one lane), without a branch.  A stage is
+// refilled only after every lane has consumed the values it read from it
+// (data dependence + __syncwarp), so the async-proxy write cannot overtake a
+// generic-proxy read of the same bytes.
 __device__ __forceinline__ void issue_unit_pred(uint32_t pred, const uint8_t *src_c, const uint8_t *src_s,
                                                 uint32_t dst, uint32_t bar) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.u32 p, %0, 0;\n\t"
-        "@p fence.proxy.async.shared::cta;\n\t"
         "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n\t"
         "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%3], [%4], %5, [%1];\n\t"
         "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%6], [%7], %8, [%1];\n\t}" ::"r"(pred),
@@ -207,9 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     const uint32_t bars = kBarAddr + warp * (kStages * 8);
     const bool active = gw < P.total_warps;
     const int U = (int)P.units;
-    const int chunk = P.chunk;
-    const int u0 = active ? gw * chunk : 0;
-    const int u1 = active ? min(U, u0 + chunk) : 0;
+    const int W = P.total_warps;
+    const int u0 = active ? (int)((int64_t)gw * U / W) : 0;
+    const int u1 = active ? (int)((int64_t)(gw + 1) * U / W) : 0;
 
     // ---- prologue: barriers, first bulk copies, lookup table -------------
     // (the packed weights never depend on the preceding grid, so the copies
@@ -306,13 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
             const uint4 c1 = lds128(st + (g + 8) * 64 + t * 16);
             const uint4 s0 = lds128(st + kUnitCodeBytes + g * 16);
             const uint4 s1 = lds128(st + kUnitCodeBytes + (g + 8) * 16);
-            __syncwarp();
-            if (pv < u1) {  // warp-uniform
-                issue_unit_pred(lane == 0, cu.c, cu.s, st, bar);
-                cursor_next(P, cu);
-                ++pv;
-            }
-            if (++stage == kStages) { stage = 0; parity ^= 1u; }
 
             const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
             const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
@@ -355,6 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                     }
                 }
             }
+            // every lane has consumed this stage: refill it with unit pv
+            __syncwarp();
+            if (pv < u1) {  // warp-uniform
+                issue_unit_pred(lane == 0, cu.c, cu.s, st, bar);
+                cursor_next(P, cu);
+                ++pv;
+            }
+            stage = (stage == kStages - 1) ? 0 : stage + 1;
+            parity ^= (stage == 0) ? 1u : 0u;
         }
 
         // ---- end of the segment: write Y or combine partial sums ------------
@@ -383,8 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                 }
             __threadfence();
             __syncwarp();
-            const int first = tile_lo / chunk;
-            const int last = (tile_hi - 1) / chunk;
+            // owner of unit x: the largest w with floor(w*U/W) <= x
+            const int first = (int)(((int64_t)(tile_lo + 1) * W - 1) / U);
+            const int last = (int)(((int64_t)tile_hi * W - 1) / U);
             unsigned arrived = 0;
             if (lane == 0) arrived = atomicAdd(P.counters + gt, 1u);
             arrived = __shfl_sync(kFull, arrived, 0);
@@ -482,10 +486,9 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
     int64_t want = (pl.units + kWarps - 1) / kWarps;  // at least one unit per warp
     if (want > sm_count) want = sm_count;
     if (want < 1) want = 1;
+    pl.grid = (int)want;
     const int64_t warps = want * kWarps;
-    pl.chunk = (pl.units + warps - 1) / warps;
-    pl.total_warps = (int)((pl.units + pl.chunk - 1) / pl.chunk);
-    pl.grid = (pl.total_warps + kWarps - 1) / kWarps;
+    pl.total_warps = (int)(pl.units < warps ? pl.units : warps);
     const int64_t mm = m < 1 ? 1 : (m > 32 ? 32 : m);
     pl.mcap = (int)(8 * ((mm + 7) / 8));
     pl.counter_bytes = round_up((size_t)pl.tiles * 4u, 256);
@@ -517,7 +520,6 @@ cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydt
     prm.m = (int)m;
     if (ub != plan.units || ub >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
     prm.units = ub;
-    prm.chunk = (int)plan.chunk;
     prm.total_warps = plan.total_warps;
     prm.partials = partials;
     prm.counters = counters;

@@ -73,8 +73,7 @@ struct GroupPlan {
     int64_t units;        // sum over problems of tiles * nsb
     int64_t tiles;        // sum over problems of ceil(n / 16)
     int grid;             // CTAs (<= SM count)
-    int64_t chunk;        // units per warp (equal chunks, the last may be short)
-    int total_warps;      // ceil(units / chunk): warps that own work
+    int total_warps;      // min(grid * warps per CTA, units); warp w owns [w*U/W, (w+1)*U/W)
     int mcap;             // 8 * ceil(m / 8)
     size_t counter_bytes; // tiles * 4, rounded up to 256
     size_t partial_bytes; // (tiles + total_warps) * 16 * mcap * 4, rounded up to 256

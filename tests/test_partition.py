@@ -1,7 +1,7 @@
 """Host-side check of the fused product's work split (no GPU).
 
 The fused GEMV splits the (16-row tile, 128-column superblock) units of a
-matrix into equal chunks, one per warp (the last may be shorter); a tile covered by several warps is combined
+matrix evenly over the warps (w owns [w*U/W, (w+1)*U/W), W <= U); a tile covered by several warps is combined
 from per-warp partial slots (slot index tile + warp) by the last warp to
 arrive, which expects exactly owner(first unit) .. owner(last unit) to
 contribute.  This test restates that arithmetic (plan + owner formula) and
@@ -15,31 +15,30 @@ import itertools
 
 def plan(units, sm_count, warps_per_cta=16):
     ctas = min(sm_count, max(1, -(-units // warps_per_cta)))
-    chunk = -(-units // (ctas * warps_per_cta))
-    warps = -(-units // chunk)
-    return chunk, warps
+    return min(units, ctas * warps_per_cta)
 
 
-def owner(x, chunk):
-    return x // chunk
+def owner(x, units, warps):
+    """Largest w with floor(w * units / warps) <= x."""
+    return ((x + 1) * warps - 1) // units
 
 
 def check(n, k, sm_count):
     tiles = -(-n // 16)
     nsb = (k // 32 + 3) // 4
     units = tiles * nsb
-    chunk, warps = plan(units, sm_count)
+    warps = plan(units, sm_count)
     assert warps <= sm_count * 16
-    ranges = [(gw * chunk, min(units, (gw + 1) * chunk)) for gw in range(warps)]
+    ranges = [(gw * units // warps, (gw + 1) * units // warps) for gw in range(warps)]
     assert all(lo < hi for lo, hi in ranges)  # no empty warp
     assert ranges[0][0] == 0 and ranges[-1][1] == units
     assert all(ranges[i][1] == ranges[i + 1][0] for i in range(warps - 1))
     for x in range(units):
-        lo, hi = ranges[owner(x, chunk)]
+        lo, hi = ranges[owner(x, units, warps)]
         assert lo <= x < hi
     slots = set()
     for r in range(tiles):
-        first, last = owner(r * nsb, chunk), owner((r + 1) * nsb - 1, chunk)
+        first, last = owner(r * nsb, units, warps), owner((r + 1) * nsb - 1, units, warps)
         touching = [gw for gw, (lo, hi) in enumerate(ranges) if lo < (r + 1) * nsb and hi > r * nsb]
         assert touching == list(range(first, last + 1))
         whole = [gw for gw in touching if ranges[gw][0] <= r * nsb and (r + 1) * nsb <= ranges[gw][1]]
