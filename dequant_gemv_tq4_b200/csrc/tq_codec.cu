@@ -4,12 +4,14 @@
 // paragraph 格式原理 items 1-3 and the paragraph after them; section
 // 解码速度：分硬件汇总 for the pre-rotated activation.
 //
-// Thread layout used by all three kernels: one warp owns one 128-column
-// superblock (four 32-element blocks) of one row per step; lane = 8*j + p
-// holds elements 4p..4p+3 of block j.  The 32-point transform runs as two
-// butterfly stages in registers (h = 1, 2) and three across lanes (h = 4, 8,
-// 16 via shfl_xor 1, 2, 4), in the codec's stage order, so every fp32 result
-// equals the sequential definition bit for bit.
+// Quantise and dequantise: lane l of a warp owns one 32-element block (32
+// consecutive columns) and the warp walks rows, so the sign pattern of the
+// lane's columns is computed once; the whole 32-point transform runs in
+// registers in the codec's stage order, so every fp32 result equals the
+// sequential definition bit for bit.
+// Pre-rotation: one warp owns one 128-column superblock of one row per step;
+// lane = 8*j + p holds elements 4p..4p+3 of block j; two butterfly stages in
+// registers (h = 1, 2), three across lanes (h = 4, 8, 16 via shfl_xor).
 #include "tq_device.cuh"
 #include "tq_internal.h"
 
@@ -52,118 +54,270 @@ __device__ __forceinline__ uint32_t magnitude_rank(float a, const float (&t)[7])
 }
 
 // -------------------------------------------------------------------------
-// Quantise.  grid.x = superblock column, grid.y * 8 warps stride the rows.
+// Block-per-lane helpers (quantise / dequantise): lane l of a warp owns block
+// 32*seg + l of its rows, i.e. 32 consecutive columns; the whole 32-point
+// transform runs in registers in the codec's stage order.
+// -------------------------------------------------------------------------
+
+// Sign bits of the lane's 32 columns (bit e = 1 where column k0+e flips).
+__device__ __forceinline__ uint32_t block_sign_bits(uint32_t k0) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) m |= (sign_mask(k0 + e) >> 31) << e;
+    return m;
+}
+
+// Packed 16-bit sign masks: word i flips elements 2i (bit 15) and 2i+1 (bit 31).
+__device__ __forceinline__ void packed_sign_words(uint32_t bits, uint32_t (&ps)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ps[i] = (((bits >> (2 * i)) & 1u) << 15) | (((bits >> (2 * i + 1)) & 1u) << 31);
+}
+
+__device__ __forceinline__ void fwht32_regs(float (&v)[32]) {
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = __fadd_rn(a, b);
+                v[i + h] = __fsub_rn(a, b);
+            }
+}
+
+// 32 input elements -> fp32 with the sign flip applied (exact).
+template <int DT>
+__device__ __forceinline__ void load_block(const char *p, uint32_t bits, const uint32_t (&ps)[16], float (&v)[32]);
+
+template <>
+__device__ __forceinline__ void load_block<kF32>(const char *p, uint32_t bits, const uint32_t (&)[16],
+                                                 float (&v)[32]) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 w = __ldg(q + i);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int e = 4 * i + c;
+            v[e] = __uint_as_float(ws[c] ^ ((bits << (31 - e)) & 0x80000000u));
+        }
+    }
+}
+
+template <>
+__device__ __forceinline__ void load_block<kBF16>(const char *p, uint32_t, const uint32_t (&ps)[16],
+                                                  float (&v)[32]) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 w = __ldg(q + i);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t x = ws[c] ^ ps[4 * i + c];
+            v[8 * i + 2 * c] = __uint_as_float(x << 16);
+            v[8 * i + 2 * c + 1] = __uint_as_float(x & 0xffff0000u);
+        }
+    }
+}
+
+template <>
+__device__ __forceinline__ void load_block<kF16>(const char *p, uint32_t, const uint32_t (&ps)[16],
+                                                 float (&v)[32]) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 w = __ldg(q + i);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t x = ws[c] ^ ps[4 * i + c];
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&x));
+            v[8 * i + 2 * c] = f.x;
+            v[8 * i + 2 * c + 1] = f.y;
+        }
+    }
+}
+
+// Logical words W0..W3 (bytes 0-3, 4-7, 8-11, 12-15 of a block) <-> stored
+// words T0..T3 (T_t = logical bytes t, t+4, t+8, t+12): a 4x4 byte transpose.
+__device__ __forceinline__ void transpose_bytes(const uint32_t (&w)[4], uint32_t (&o)[4]) {
+    const uint32_t a = prmt(w[0], w[1], 0x5140u), b = prmt(w[2], w[3], 0x5140u);
+    const uint32_t c = prmt(w[0], w[1], 0x7362u), d = prmt(w[2], w[3], 0x7362u);
+    o[0] = prmt(a, b, 0x5410u);
+    o[1] = prmt(a, b, 0x7632u);
+    o[2] = prmt(c, d, 0x5410u);
+    o[3] = prmt(c, d, 0x7632u);
+}
+
+// -------------------------------------------------------------------------
+// Quantise.  grid.x = 1024-column segment (32 blocks, one per lane),
+// grid.y * 8 warps stride the rows (padded to a multiple of 16).
 // -------------------------------------------------------------------------
 template <int DT>
 __global__ void __launch_bounds__(kCodecThreads) quantize_kernel(const char *__restrict__ w, int64_t ldw, int n,
                                                                    int nb, int nsb, uint32_t *__restrict__ codes,
                                                                    uint32_t *__restrict__ scales) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int j = lane >> 3, p = lane & 7;
-    const int sb = blockIdx.x;
-    const bool valid = sb * kSbBlocks + j < nb;
-    const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
-
-    uint32_t smask[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) smask[i] = sign_mask(col0 + i);
+    const int blk = blockIdx.x * 32 + lane;  // block column of this lane
+    const bool exists = blk < nsb * kSbBlocks;  // padding blocks still get zero codes
+    const bool valid = blk < nb;
+    const int sb = blk >> 2, j = blk & 3;
+    const uint32_t k0 = (uint32_t)blk * kBlock;
+    const uint32_t bits = block_sign_bits(k0);
+    uint32_t ps[16];
+    packed_sign_words(bits, ps);
     float thr[7];
 #pragma unroll
     for (int i = 0; i < 7; ++i) thr[i] = __uint_as_float(c_thr_bits[i]);
 
-    // code gather for the packed store: output word o = 4*tw + jw holds logical
-    // bytes tw, tw+4, tw+8, tw+12 of block jw; logical byte L comes from lane
-    // 8*jw + L/2 (low or high byte of its 16-bit code group).
-    const int o = lane & 15, tw = o >> 2, jw = o & 3;
-    const int byte_shift = 8 * (tw & 1);
-
-    const int rows_padded = (n + 15) & ~15;  // rows past n are written as zeros
+    const int rows_padded = (n + 15) & ~15;
     for (int row = blockIdx.y * kCodecWarps + warp; row < rows_padded; row += gridDim.y * kCodecWarps) {
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid && row < n) load4<DT>(w + ((int64_t)row * ldw + col0) * ElemSize<DT>::value, v);
+        float v[32];
+        if (valid && row < n) {
+            load_block<DT>(w + ((int64_t)row * ldw + k0) * ElemSize<DT>::value, bits, ps, v);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = flip(v[i], smask[i]);
-        fwht32_warp(v, p);
+            for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        }
+        fwht32_regs(v);
 
-        // half-block scale: adjacent pairwise tree of the 16 squares
-        float q0 = __fmul_rn(v[0], v[0]), q1 = __fmul_rn(v[1], v[1]);
-        float q2 = __fmul_rn(v[2], v[2]), q3 = __fmul_rn(v[3], v[3]);
-        float s = __fadd_rn(__fadd_rn(q0, q1), __fadd_rn(q2, q3));
-        s = __fadd_rn(s, __shfl_xor_sync(kFull, s, 1));
-        s = __fadd_rn(s, __shfl_xor_sync(kFull, s, 2));
-        const __half hd = __float2half_rn(__fsqrt_rn(__fmul_rn(s, 0.0625f)));
-        const float D = __half2float(hd);
-        float t[7];
+        // half-block scales: adjacent pairwise tree of the squares
+        uint32_t dbits[2];
+        float D[2];
 #pragma unroll
-        for (int i = 0; i < 7; ++i) t[i] = __fmul_rn(thr[i], D);
-
-        uint32_t c16 = 0;
+        for (int h = 0; h < 2; ++h) {
+            float q[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t code = (v[i] < 0.0f ? 8u : 0u) | magnitude_rank(fabsf(v[i]), t);
-            c16 |= code << (4 * i);
+            for (int e = 0; e < 16; ++e) q[e] = __fmul_rn(v[16 * h + e], v[16 * h + e]);
+#pragma unroll
+            for (int step = 1; step < 16; step <<= 1)
+#pragma unroll
+                for (int i = 0; i < 16; i += 2 * step) q[i] = __fadd_rn(q[i], q[i + step]);
+            const __half hd = __float2half_rn(__fsqrt_rn(__fmul_rn(q[0], 0.0625f)));
+            dbits[h] = __half_as_ushort(hd);
+            D[h] = __half2float(hd);
         }
 
-        uint32_t word = 0;
+        uint32_t lw[4] = {0u, 0u, 0u, 0u};  // logical code words
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t src = __shfl_sync(kFull, c16, 8 * jw + 2 * i + (tw >> 1));
-            word |= ((src >> byte_shift) & 0xffu) << (8 * i);
+        for (int h = 0; h < 2; ++h) {
+            float t[7];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) t[i] = __fmul_rn(thr[i], D[h]);
+#pragma unroll
+            for (int e = 16 * h; e < 16 * h + 16; ++e) {
+                const uint32_t code = (v[e] < 0.0f ? 8u : 0u) | magnitude_rank(fabsf(v[e]), t);
+                lw[e >> 3] |= code << (4 * (e & 7));
+            }
         }
-        const size_t sb_index = unit_row(row, sb, nsb);
-        if (lane < 16) codes[sb_index * 16 + o] = word;
-
-        const uint32_t hbits = __half_as_ushort(hd);
-        const uint32_t hbits_hi = __shfl_xor_sync(kFull, hbits, 4);
-        if (p == 0) scales[sb_index * 4 + j] = hbits | (hbits_hi << 16);
+        if (exists) {
+            uint32_t sw[4];
+            transpose_bytes(lw, sw);
+            const size_t slot = unit_row(row, sb, nsb);
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) codes[slot * 16 + 4 * tt + j] = sw[tt];
+            scales[slot * 4 + j] = dbits[0] | (dbits[1] << 16);
+        }
     }
 }
 
 // -------------------------------------------------------------------------
 // Dequantise: w~ = s .* (H c) / 32, fp32, rounded to the output dtype.
+// The 1/32 is folded into the fp16 scale (exact power-of-two scaling).
 // -------------------------------------------------------------------------
+template <int DT>
+__device__ __forceinline__ void store_block(char *p, uint32_t bits, const uint32_t (&ps)[16], const float (&v)[32]);
+
+template <>
+__device__ __forceinline__ void store_block<kF32>(char *p, uint32_t bits, const uint32_t (&)[16],
+                                                  const float (&v)[32]) {
+    uint4 *q = reinterpret_cast<uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t o[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int e = 4 * i + c;
+            o[c] = __float_as_uint(v[e]) ^ ((bits << (31 - e)) & 0x80000000u);
+        }
+        q[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+template <>
+__device__ __forceinline__ void store_block<kBF16>(char *p, uint32_t, const uint32_t (&ps)[16],
+                                                   const float (&v)[32]) {
+    uint4 *q = reinterpret_cast<uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t o[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * c], v[8 * i + 2 * c + 1]);
+            o[c] = *reinterpret_cast<uint32_t *>(&h) ^ ps[4 * i + c];
+        }
+        q[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+template <>
+__device__ __forceinline__ void store_block<kF16>(char *p, uint32_t, const uint32_t (&ps)[16],
+                                                  const float (&v)[32]) {
+    uint4 *q = reinterpret_cast<uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t o[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            __half2 h = __floats2half2_rn(v[8 * i + 2 * c], v[8 * i + 2 * c + 1]);
+            o[c] = *reinterpret_cast<uint32_t *>(&h) ^ ps[4 * i + c];
+        }
+        q[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_t *__restrict__ codes,
                                                                      const uint32_t *__restrict__ scales, int n,
                                                                      int nb, int nsb, char *__restrict__ out,
                                                                      int64_t ldo) {
-    __shared__ float smag[8];
-    if (threadIdx.x < 8) smag[threadIdx.x] = __uint_as_float(c_mag_bits[threadIdx.x]);
+    __shared__ float cent[16];  // signed centroids c(code)
+    if (threadIdx.x < 16) {
+        const float m = __uint_as_float(c_mag_bits[threadIdx.x & 7]);
+        cent[threadIdx.x] = (threadIdx.x & 8) ? -m : m;
+    }
     __syncthreads();
+    const uint32_t cent_base = (uint32_t)__cvta_generic_to_shared(cent);
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int j = lane >> 3, p = lane & 7;
-    const int sb = blockIdx.x;
-    const bool valid = sb * kSbBlocks + j < nb;
-    const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
-    uint32_t smask[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) smask[i] = sign_mask(col0 + i);
-
-    // logical bytes 2p and 2p+1 of block j live in words 4*((2p)%4)+j and
-    // 4*((2p+1)%4)+j, byte p/2
-    const int src0 = 4 * ((2 * p) & 3) + j, src1 = 4 * ((2 * p + 1) & 3) + j;
-    const int bsh = 8 * (p >> 1);
-    const int half = p >> 2;
+    const int blk = blockIdx.x * 32 + lane;
+    const bool valid = blk < nb;
+    const int sb = blk >> 2, j = blk & 3;
+    const uint32_t k0 = (uint32_t)blk * kBlock;
+    const uint32_t bits = block_sign_bits(k0);
+    uint32_t ps[16];
+    packed_sign_words(bits, ps);
 
     for (int row = blockIdx.y * kCodecWarps + warp; row < n; row += gridDim.y * kCodecWarps) {
-        const size_t sb_index = unit_row(row, sb, nsb);
-        const uint32_t cw = __ldg(codes + sb_index * 16 + (lane & 15));
-        const uint32_t sw = __ldg(scales + sb_index * 4 + j);
-        const uint32_t b0 = (__shfl_sync(kFull, cw, src0) >> bsh) & 0xffu;
-        const uint32_t b1 = (__shfl_sync(kFull, cw, src1) >> bsh) & 0xffu;
-        const uint32_t code[4] = {b0 & 15u, b0 >> 4, b1 & 15u, b1 >> 4};
-        const float D = __half2float(__ushort_as_half((unsigned short)(half ? (sw >> 16) : (sw & 0xffffu))));
-        float v[4];
+        if (!valid) continue;
+        const size_t slot = unit_row(row, sb, nsb);
+        uint32_t sw[4], lw[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float c = __fmul_rn(smag[code[i] & 7u], D);
-            v[i] = (code[i] & 8u) ? -c : c;
+        for (int tt = 0; tt < 4; ++tt) sw[tt] = __ldg(codes + slot * 16 + 4 * tt + j);
+        transpose_bytes(sw, lw);  // the transpose is its own inverse
+        const uint32_t sc = __ldg(scales + slot * 4 + j);
+        const float2 D = __half22float2(*reinterpret_cast<const __half2 *>(&sc));
+        const float Ds[2] = {__fmul_rn(D.x, 0.03125f), __fmul_rn(D.y, 0.03125f)};
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const uint32_t code = (lw[e >> 3] >> (4 * (e & 7))) & 15u;
+            v[e] = __fmul_rn(lds_f32(cent_base + 4 * code), Ds[e >> 4]);
         }
-        fwht32_warp(v, p);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = flip(__fmul_rn(v[i], 0.03125f), smask[i]);
-        if (valid) store4<DT>(out + ((int64_t)row * ldo + col0) * ElemSize<DT>::value, v);
+        fwht32_regs(v);
+        store_block<DT>(out + ((int64_t)row * ldo + k0) * ElemSize<DT>::value, bits, ps, v);
     }
 }
 
@@ -204,10 +358,10 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     in.xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
 }
 
-int rows_grid(int64_t n, int64_t nsb, int sm_count) {
-    // aim for ~8 resident CTAs per SM in total, at least one warp-row per CTA
-    int64_t target = (int64_t)sm_count * 8;
-    int64_t gy = (target + nsb - 1) / nsb;
+int rows_grid(int64_t n, int64_t segs, int sm_count) {
+    // aim for ~4 resident CTAs (32 warps) per SM in total
+    int64_t target = (int64_t)sm_count * 4;
+    int64_t gy = (target + segs - 1) / segs;
     int64_t max_gy = (((n + 15) & ~(int64_t)15) + kCodecWarps - 1) / kCodecWarps;
     if (gy > max_gy) gy = max_gy;
     if (gy > 65535) gy = 65535;
@@ -223,7 +377,8 @@ cudaError_t launch_quantize(const void *w, int dtype, int64_t n, int64_t k, int6
     cudaError_t err = device_info(&di);
     if (err != cudaSuccess) return err;
     const int64_t nb = k / 32, nsb = superblocks(k);
-    dim3 grid((unsigned)nsb, (unsigned)rows_grid(n, nsb, di.sm_count));
+    const int64_t segs = (nsb * kSbBlocks + 31) / 32;
+    dim3 grid((unsigned)segs, (unsigned)rows_grid(n, segs, di.sm_count));
     auto *c = reinterpret_cast<uint32_t *>(codes);
     auto *s = reinterpret_cast<uint32_t *>(scales);
     const char *wp = static_cast<const char *>(w);
@@ -242,7 +397,8 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int6
     cudaError_t err = device_info(&di);
     if (err != cudaSuccess) return err;
     const int64_t nb = k / 32, nsb = superblocks(k);
-    dim3 grid((unsigned)nsb, (unsigned)rows_grid(n, nsb, di.sm_count));
+    const int64_t segs = (nb + 31) / 32;
+    dim3 grid((unsigned)segs, (unsigned)rows_grid(n, segs, di.sm_count));
     auto *c = reinterpret_cast<const uint32_t *>(codes);
     auto *s = reinterpret_cast<const uint32_t *>(scales);
     char *o = static_cast<char *>(w_out);

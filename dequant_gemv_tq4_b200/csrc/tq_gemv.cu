@@ -44,11 +44,15 @@ namespace {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 6;
+constexpr int kStages = 3;    // ring stages per warp
+constexpr int kPerStage = 2;  // consecutive units per stage
 constexpr int kUnitCodeBytes = 1024;
 constexpr int kUnitScaleBytes = 256;
 constexpr int kUnitBytes = kUnitCodeBytes + kUnitScaleBytes;
-constexpr int kRingWarpBytes = kStages * kUnitBytes;  // 7680
+// stage = [codes of unit A | codes of unit B | scales of A | scales of B]
+constexpr int kStageScaleOff = kPerStage * kUnitCodeBytes;
+constexpr int kStageBytes = kPerStage * kUnitBytes;    // 2560
+constexpr int kRingWarpBytes = kStages * kStageBytes;  // 7680
 // Shared-memory map (addresses in the CTA's shared window; the dynamic
 // allocation starts at a small base B <= kMaxSmemBase):
 //   [B, B + 8 rings)            rings of warps 0..7
@@ -141,57 +145,150 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint6
     return false;
 }
 
-// One unit (1024 code bytes + 256 scale bytes) into a ring stage, issued by
-// the lanes for which `pred` is set (one lane), without a branch.  A stage is
-// refilled only after every lane has consumed the values it read from it
-// (data dependence + __syncwarp), so the async-proxy write cannot overtake a
-// generic-proxy read of the same bytes.
-__device__ __forceinline__ void issue_unit_pred(uint32_t pred, const uint8_t *src_c, const uint8_t *src_s,
-                                                uint32_t dst, uint32_t bar) {
+__device__ __forceinline__ void arrive_expect_tx_pred(uint32_t pred, uint32_t bar, uint32_t bytes) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.u32 p, %0, 0;\n\t"
-        "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n\t"
-        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%3], [%4], %5, [%1];\n\t"
-        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%6], [%7], %8, [%1];\n\t}" ::"r"(pred),
-        "r"(bar), "r"(kUnitBytes), "r"(dst), "l"(src_c), "r"(kUnitCodeBytes), "r"(dst + kUnitCodeBytes), "l"(src_s),
-        "r"(kUnitScaleBytes)
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %0, 0;\n\t"
+        "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n\t}" ::"r"(pred),
+        "r"(bar), "r"(bytes)
         : "memory");
 }
 
-
+// Bulk copy global -> shared completing on `bar`, issued by the lanes with
+// `pred` set (one lane), without a branch.
+__device__ __forceinline__ void bulk_copy_pred(uint32_t pred, uint32_t dst, const void *src, uint32_t bytes,
+                                               uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %0, 0;\n\t"
+        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%1], [%2], %3, [%4];\n\t}" ::"r"(pred),
+        "r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
 
 // Producer cursor: the next unit this warp will copy, walked incrementally.
 struct Cursor {
     const uint8_t *c;
     const uint8_t *s;
-    int64_t left;  // units left in the current problem
+    int left;  // units left in the current problem
     int q;
 };
 
-__device__ __forceinline__ Cursor cursor_at(const GroupParams &P, int64_t v) {
+__device__ __forceinline__ int problem_of(const GroupParams &P, int v) {
     int q = 0;
     while (q + 1 < P.count && v >= P.prob[q + 1].unit_begin) ++q;
-    const int64_t local = v - P.prob[q].unit_begin;
-    const int64_t end = (q + 1 < P.count) ? P.prob[q + 1].unit_begin : P.units;
+    return q;
+}
+
+__device__ __forceinline__ int problem_end(const GroupParams &P, int q) {
+    return (int)((q + 1 < P.count) ? P.prob[q + 1].unit_begin : P.units);
+}
+
+__device__ __forceinline__ Cursor cursor_at(const GroupParams &P, int v) {
+    const int q = problem_of(P, v);
+    const int local = v - (int)P.prob[q].unit_begin;
     Cursor cu;
-    cu.c = P.prob[q].codes + local * kUnitCodeBytes;
-    cu.s = P.prob[q].scales + local * kUnitScaleBytes;
-    cu.left = end - v;
+    cu.c = P.prob[q].codes + (int64_t)local * kUnitCodeBytes;
+    cu.s = P.prob[q].scales + (int64_t)local * kUnitScaleBytes;
+    cu.left = problem_end(P, q) - v;
     cu.q = q;
     return cu;
 }
 
-__device__ __forceinline__ void cursor_next(const GroupParams &P, Cursor &cu) {
-    cu.c += kUnitCodeBytes;
-    cu.s += kUnitScaleBytes;
-    if (--cu.left == 0 && cu.q + 1 < P.count) {
+__device__ __forceinline__ void cursor_step(const GroupParams &P, Cursor &cu, int units) {
+    cu.c += units * kUnitCodeBytes;
+    cu.s += units * kUnitScaleBytes;
+    cu.left -= units;
+    if (cu.left == 0 && cu.q + 1 < P.count) {
         ++cu.q;
         cu.c = P.prob[cu.q].codes;
         cu.s = P.prob[cu.q].scales;
-        const int64_t end = (cu.q + 1 < P.count) ? P.prob[cu.q + 1].unit_begin : P.units;
-        cu.left = end - P.prob[cu.q].unit_begin;
+        cu.left = problem_end(P, cu.q) - (int)P.prob[cu.q].unit_begin;
     }
+}
+
+// Copy the next `cnt` (1 or 2) units of the cursor into a stage.  Units of one
+// problem are contiguous, so a pair is one copy per plane; a pair that
+// straddles two problems takes one copy per unit and plane.
+__device__ __forceinline__ void issue_stage(const GroupParams &P, Cursor &cu, int cnt, uint32_t dst, uint32_t bar,
+                                            uint32_t leader) {
+    arrive_expect_tx_pred(leader, bar, (uint32_t)(cnt * kUnitBytes));
+    if (cu.left >= cnt) {
+        bulk_copy_pred(leader, dst, cu.c, (uint32_t)(cnt * kUnitCodeBytes), bar);
+        bulk_copy_pred(leader, dst + kStageScaleOff, cu.s, (uint32_t)(cnt * kUnitScaleBytes), bar);
+        cursor_step(P, cu, cnt);
+    } else {
+        for (int h = 0; h < cnt; ++h) {
+            bulk_copy_pred(leader, dst + h * kUnitCodeBytes, cu.c, kUnitCodeBytes, bar);
+            bulk_copy_pred(leader, dst + kStageScaleOff + h * kUnitScaleBytes, cu.s, kUnitScaleBytes, bar);
+            cursor_step(P, cu, 1);
+        }
+    }
+}
+
+// Write the accumulators of a finished tile segment: straight to Y when this
+// warp covered the whole tile, else through the fixed-order partial sums.
+template <int NT, bool M1, int OT>
+__device__ __noinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
+                                           int u1, int gw, const float (&acc)[NT][4]) {
+    constexpr int kMcap = 8 * NT;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const DevProblem &pr = P.prob[q];
+    const int U = (int)P.units, W = P.total_warps;
+    const int64_t gt = pr.tile_begin + r;
+    const int row_g = r * 16 + g, row_g8 = row_g + 8;
+    if (u0 <= tile_lo && tile_hi <= u1) {
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                if (M1 && (b & 1)) continue;
+                const int xrow = 8 * a + 2 * t + (b & 1);
+                const int wrow = (b & 2) ? row_g8 : row_g;
+                if (xrow < P.m && wrow < pr.n)
+                    store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, acc[a][b]);
+            }
+        return;
+    }
+    float *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int xrow = 8 * a + 2 * t + (b & 1);
+            const int wrow = g + ((b & 2) ? 8 : 0);
+            slot[xrow * 16 + wrow] = acc[a][b];
+        }
+    __syncwarp();
+    // owner of unit x: the largest w with floor(w*U/W) <= x
+    const int first = (int)(((int64_t)(tile_lo + 1) * W - 1) / U);
+    const int last = (int)(((int64_t)tile_hi * W - 1) / U);
+    unsigned arrived = 0;
+    if (lane == 0) {
+        __threadfence();  // release: the warp's slot writes (ordered by the warp barrier)
+        arrived = atomicAdd(P.counters + gt, 1u);
+    }
+    arrived = __shfl_sync(kFull, arrived, 0);
+    if (arrived != (unsigned)(last - first)) return;
+    if (lane == 0) __threadfence();  // acquire: the other contributors' slots
+    __syncwarp();
+    const int cnt = last - first + 1;
+    for (int e = lane; e < 16 * P.m; e += 32) {
+        const int xrow = e >> 4, wl = e & 15;
+        const float *src = P.partials + (gt + first) * (int64_t)(16 * kMcap) + xrow * 16 + wl;
+        // eight independent loads in flight, added in slot order
+        float sum = 0.f;
+        int c = 0;
+        for (; c + 8 <= cnt; c += 8) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + (int64_t)(c + i) * (16 * kMcap));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum += v[i];
+        }
+        for (; c < cnt; ++c) sum += __ldcg(src + (int64_t)c * (16 * kMcap));
+        const int wrow = r * 16 + wl;
+        if (wrow < pr.n) store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
+    }
+    if (lane == 0) P.counters[gt] = 0u;
 }
 
 template <int NT, bool M1, int OT>
@@ -224,10 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         }
         __syncwarp();
         cu = cursor_at(P, u0);
-        for (int i = 0; i < kStages && pv < u1; ++i, ++pv) {
+        for (int i = 0; i < kStages && pv < u1; ++i) {
+            const int cnt = min(kPerStage, u1 - pv);
             const bool skip = P.inject_skip && gw == 0 && i == 1;
-            issue_unit_pred(lane == 0 && !skip, cu.c, cu.s, ring + i * kUnitBytes, bars + 8 * i);
-            cursor_next(P, cu);
+            issue_stage(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0 && !skip);
+            pv += cnt;
         }
     }
     {
@@ -249,65 +347,64 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     const int g = lane >> 2, t = lane & 3;
     // PRMT operand: byte 0 = lane*4, bytes 2..3 = table base >> 16
     const uint32_t lut_lane = kLutAddr | ((uint32_t)lane * 4u);
-    constexpr int kMcap = 8 * NT;
 
-    int q = 0;
-    while (q + 1 < P.count && u0 >= P.prob[q + 1].unit_begin) ++q;
+    // ---- segment state: the tile the current unit belongs to ---------------
+    int q = problem_of(P, u0);
+    int prob_end = problem_end(P, q);
+    int nsb = P.prob[q].nsb;
+    int r, sb, tile_lo;
+    {
+        const int local = u0 - (int)P.prob[q].unit_begin;
+        r = local / nsb;
+        sb = local - r * nsb;
+        tile_lo = (int)P.prob[q].unit_begin + r * nsb;
+    }
+    int seg_end = min(tile_lo + nsb, u1);
+    // activation fragments: rows past m repeat row m-1 (their outputs are never
+    // stored), so every lane loads without a predicate
+    const uint16_t *xbase[NT];
+#pragma unroll
+    for (int a = 0; a < NT; ++a) {
+        const int xrow = min(8 * a + g, P.m - 1);
+        xbase[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
+    }
+
+    float acc[NT][4];
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+
     int u = u0;
     int stage = 0;
     uint32_t parity = 0;
-
     while (u < u1) {
-        // ---- one tile segment: units u .. seg_end-1 share the 16 rows --------
-        const DevProblem &pr = P.prob[q];
-        const int nsb = pr.nsb;
-        const int ub = (int)pr.unit_begin;
-        const int local = u - ub;
-        const int r = local / nsb;
-        const int sb0 = local - r * nsb;
-        const int tile_lo = ub + r * nsb, tile_hi = tile_lo + nsb;
-        const int seg_end = min(tile_hi, u1);
-        // activation fragments: rows past m repeat row m-1 (their outputs are
-        // never stored), so every lane loads without a predicate
-        const uint16_t *xbase[NT];
-#pragma unroll
-        for (int a = 0; a < NT; ++a) {
-            const int xrow = min(8 * a + g, P.m - 1);
-            xbase[a] = pr.xrot + (int64_t)xrow * nsb * 128 + t * 8;
-        }
-
-        float acc[NT][4];
-#pragma unroll
-        for (int a = 0; a < NT; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-
-        int sb = sb0;
-        for (; u < seg_end; ++u, ++sb) {
-            const uint32_t st = ring + stage * kUnitBytes, bar = bars + 8 * stage;
-            bool ok = mbar_try(bar, parity);
+        const uint32_t st = ring + stage * kStageBytes, bar = bars + 8 * stage;
+        bool ok = mbar_try(bar, parity);
+        if (!__all_sync(kFull, ok)) {
+            ok = ok || mbar_wait_slow(bar, parity, P.timeout_ns);
             if (!__all_sync(kFull, ok)) {
-                ok = ok || mbar_wait_slow(bar, parity, P.timeout_ns);
-                if (!__all_sync(kFull, ok)) {
-                    // report, then let the copies still in flight land before leaving
-                    if (lane == 0) {
-                        atomicOr(P.status, kStatusTimeout);
-                        int s2 = stage;
-                        uint32_t p2 = parity;
-                        for (int v = u + 1; v < pv; ++v) {
-                            if (++s2 == kStages) { s2 = 0; p2 ^= 1u; }
-                            mbar_wait_slow(bars + 8 * s2, p2, P.timeout_ns);
-                        }
+                // report, then let the copies still in flight land before leaving
+                if (lane == 0) {
+                    atomicOr(P.status, kStatusTimeout);
+                    int s2 = stage;
+                    uint32_t p2 = parity;
+                    for (int i = 1; i < kStages && u + kPerStage * i < pv; ++i) {
+                        if (++s2 == kStages) { s2 = 0; p2 ^= 1u; }
+                        mbar_wait_slow(bars + 8 * s2, p2, P.timeout_ns);
                     }
-                    __syncwarp();
-                    return;
                 }
+                __syncwarp();
+                return;
             }
-            const uint4 c0 = lds128(st + g * 64 + t * 16);
-            const uint4 c1 = lds128(st + (g + 8) * 64 + t * 16);
-            const uint4 s0 = lds128(st + kUnitCodeBytes + g * 16);
-            const uint4 s1 = lds128(st + kUnitCodeBytes + (g + 8) * 16);
-
+        }
+#pragma unroll 1
+        for (int h = 0; h < kPerStage && u < u1; ++h) {
+            const uint32_t sc = st + h * kUnitCodeBytes, ss = st + kStageScaleOff + h * kUnitScaleBytes;
+            const uint4 c0 = lds128(sc + g * 64 + t * 16);
+            const uint4 c1 = lds128(sc + (g + 8) * 64 + t * 16);
+            const uint4 s0 = lds128(ss + g * 16);
+            const uint4 s1 = lds128(ss + (g + 8) * 16);
             const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
             const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
             const uint32_t sw0[4] = {s0.x, s0.y, s0.z, s0.w};
@@ -329,94 +426,63 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                 const uint32_t a13 = lds_u32(prmt(cw1[j], lut_lane, 0x7634u));
                 const float2 dg = __half22float2(*reinterpret_cast<const __half2 *>(&sw0[j]));
                 const float2 dg8 = __half22float2(*reinterpret_cast<const __half2 *>(&sw1[j]));
-                const float d0g = dg.x, d1g = dg.y, d0g8 = dg8.x, d1g8 = dg8.y;
 #pragma unroll
                 for (int a = 0; a < NT; ++a) {
                     float d[4];
                     mma_16816_zero(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
-                    acc[a][0] = fmaf(d[0], d0g, acc[a][0]);
-                    acc[a][2] = fmaf(d[2], d0g8, acc[a][2]);
+                    acc[a][0] = fmaf(d[0], dg.x, acc[a][0]);
+                    acc[a][2] = fmaf(d[2], dg8.x, acc[a][2]);
                     if (!M1) {
-                        acc[a][1] = fmaf(d[1], d0g, acc[a][1]);
-                        acc[a][3] = fmaf(d[3], d0g8, acc[a][3]);
+                        acc[a][1] = fmaf(d[1], dg.x, acc[a][1]);
+                        acc[a][3] = fmaf(d[3], dg8.x, acc[a][3]);
                     }
                     mma_16816_zero(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
-                    acc[a][0] = fmaf(d[0], d1g, acc[a][0]);
-                    acc[a][2] = fmaf(d[2], d1g8, acc[a][2]);
+                    acc[a][0] = fmaf(d[0], dg.y, acc[a][0]);
+                    acc[a][2] = fmaf(d[2], dg8.y, acc[a][2]);
                     if (!M1) {
-                        acc[a][1] = fmaf(d[1], d1g, acc[a][1]);
-                        acc[a][3] = fmaf(d[3], d1g8, acc[a][3]);
+                        acc[a][1] = fmaf(d[1], dg.y, acc[a][1]);
+                        acc[a][3] = fmaf(d[3], dg8.y, acc[a][3]);
                     }
                 }
             }
-            // every lane has consumed this stage: refill it with unit pv
-            __syncwarp();
-            if (pv < u1) {  // warp-uniform
-                issue_unit_pred(lane == 0, cu.c, cu.s, st, bar);
-                cursor_next(P, cu);
-                ++pv;
-            }
-            stage = (stage == kStages - 1) ? 0 : stage + 1;
-            parity ^= (stage == 0) ? 1u : 0u;
-        }
-
-        // ---- end of the segment: write Y or combine partial sums ------------
-        const int64_t gt = pr.tile_begin + r;
-        const int row_g = r * 16 + g, row_g8 = row_g + 8;
-        if (u0 <= tile_lo && tile_hi <= u1) {
+            ++u;
+            ++sb;
+            if (u == seg_end) {  // warp-uniform
+                flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, acc);
 #pragma unroll
-            for (int a = 0; a < NT; ++a)
+                for (int a = 0; a < NT; ++a)
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    if (M1 && (b & 1)) continue;
-                    const int xrow = 8 * a + 2 * t + (b & 1);
-                    const int wrow = (b & 2) ? row_g8 : row_g;
-                    if (xrow < P.m && wrow < pr.n)
-                        store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, acc[a][b]);
-                }
-        } else {
-            float *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
+                    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+                if (u < u1) {
+                    if (u == prob_end) {  // next problem: new tiles, new activation
+                        ++q;
+                        prob_end = problem_end(P, q);
+                        nsb = P.prob[q].nsb;
+                        r = 0;
+                        tile_lo = u;
 #pragma unroll
-            for (int a = 0; a < NT; ++a)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int xrow = 8 * a + 2 * t + (b & 1);
-                    const int wrow = g + ((b & 2) ? 8 : 0);
-                    slot[xrow * 16 + wrow] = acc[a][b];
-                }
-            __threadfence();
-            __syncwarp();
-            // owner of unit x: the largest w with floor(w*U/W) <= x
-            const int first = (int)(((int64_t)(tile_lo + 1) * W - 1) / U);
-            const int last = (int)(((int64_t)tile_hi * W - 1) / U);
-            unsigned arrived = 0;
-            if (lane == 0) arrived = atomicAdd(P.counters + gt, 1u);
-            arrived = __shfl_sync(kFull, arrived, 0);
-            if (arrived == (unsigned)(last - first)) {
-                __threadfence();
-                for (int e = lane; e < 16 * P.m; e += 32) {
-                    const int xrow = e >> 4, wl = e & 15;
-                    const float *src = P.partials + (gt + first) * (int64_t)(16 * kMcap) + xrow * 16 + wl;
-                    const int cnt = last - first + 1;
-                    // eight independent loads in flight, added in slot order
-                    float sum = 0.f;
-                    int c = 0;
-                    for (; c + 8 <= cnt; c += 8) {
-                        float v[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + (int64_t)(c + i) * (16 * kMcap));
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) sum += v[i];
+                        for (int a = 0; a < NT; ++a) {
+                            const int xrow = min(8 * a + g, P.m - 1);
+                            xbase[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
+                        }
+                    } else {
+                        ++r;
+                        tile_lo += nsb;
                     }
-                    for (; c < cnt; ++c) sum += __ldcg(src + (int64_t)c * (16 * kMcap));
-                    const int wrow = r * 16 + wl;
-                    if (wrow < pr.n) store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
+                    sb = 0;
+                    seg_end = min(tile_lo + nsb, u1);
                 }
-                if (lane == 0) P.counters[gt] = 0u;
             }
         }
-        // next segment: same problem, or the next one when this one is done
-        if (u < u1 && u == ((q + 1 < P.count) ? P.prob[q + 1].unit_begin : U)) ++q;
+        // every lane has consumed this stage: refill it with the next units
+        __syncwarp();
+        if (pv < u1) {  // warp-uniform
+            const int cnt = min(kPerStage, u1 - pv);
+            issue_stage(P, cu, cnt, st, bar, lane == 0);
+            pv += cnt;
+        }
+        stage = (stage == kStages - 1) ? 0 : stage + 1;
+        parity ^= (stage == 0) ? 1u : 0u;
     }
 }
 
