@@ -74,6 +74,7 @@ def load_library() -> ctypes.CDLL:
             "tq_gemm_batch": ([ctypes.POINTER(GemmDesc), I, I64, I, I, P, SZ, P], I),
             "tq_workspace_status": ([P, I, P], I),
             "tq_debug_set_flags": ([ctypes.c_uint32], None),
+            "tq_gemv_static_scratch": ([P, P, I64, I64, P, I, P, I, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -149,6 +150,13 @@ def tq_workspace_status(workspace, clear, stream) -> int:
 
 def tq_debug_set_flags(flags: int) -> None:
     load_library().tq_debug_set_flags(flags)
+
+
+def tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream) -> int:
+    """GEMV without a workspace argument, for callers that cannot allocate
+    device memory: the scratch is a fixed array inside the library (see
+    include/tq.h).  Calls that overlap on the GPU must not share it."""
+    return load_library().tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream)
 
 
 # ---------------------------------------------------------------------------

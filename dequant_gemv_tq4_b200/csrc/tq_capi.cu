@@ -322,3 +322,69 @@ tq_status tq_workspace_status(void *workspace, int clear, void *stream) {
 void tq_debug_set_flags(uint32_t flags) { tq::set_debug_flags(flags); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// GEMV for callers that cannot allocate device memory.
+//
+// Some callers have no way to obtain a workspace: code running inside a
+// custom allocator or a memory-pool callback (where allocating would recurse),
+// plugins handed only the tensors of one operation by a host framework, or
+// processes whose device memory is entirely reserved up front.  For them the
+// scratch of the fused GEMV (status word, split-K counters, partial sums,
+// pre-rotated activation) lives in this fixed device array instead, sized
+// TQ_STATIC_SCRATCH_BYTES, resident on every GPU that loads the library until
+// the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_scratch[TQ_STATIC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[256];
+
+// Device address of g_static_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is asked from the
+// runtime, once per device, with that device current.
+cudaError_t static_scratch_address(void **out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (err != cudaSuccess) return err;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" tq_status tq_gemv_static_scratch(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
+                                            const void *x, tq_dtype xt, void *y, tq_dtype yt, void *stream) {
+    tq_status st = check_gemm_common(codes, scales, n, k, 1, y, yt, n);
+    if (st != TQ_OK || n == 0) return st;
+    if (!valid_dtype(xt)) return TQ_ERR_DTYPE;
+    if ((st = check_matrix_operand(x, k, k)) != TQ_OK) return st;
+    Layout lay;
+    if ((st = make_layout(&n, &k, 1, &k, 1, 1, &lay)) != TQ_OK) return st;
+    if (lay.total > (size_t)TQ_STATIC_SCRATCH_BYTES) return TQ_ERR_SHAPE;  // does not fit the fixed scratch
+    void *scratch = nullptr;
+    if (static_scratch_address(&scratch) != cudaSuccess) return TQ_ERR_CUDA;
+    char *ws = static_cast<char *>(scratch);
+    auto *xrot = reinterpret_cast<uint16_t *>(ws + lay.xrot_off[0]);
+    cudaStream_t s = (cudaStream_t)stream;
+    tq::RotJob job = {x, k, k, xrot};
+    // the pre-rotation launch also zeroes the status word and the counters:
+    // the array keeps whatever the previous call left in it
+    cudaError_t e = tq::launch_prerotate(&job, 1, xt, 1, reinterpret_cast<unsigned *>(ws),
+                                         (int64_t)(lay.partial_off / 4), s);
+    if (e != cudaSuccess) return TQ_ERR_CUDA;
+    tq::GemvProblem pb = {codes, scales, xrot, y, n, n, k};
+    e = tq::launch_group(&pb, 1, 1, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
+                         reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true, s);
+    return from_cuda(e);
+}

@@ -225,6 +225,33 @@ TQ_API tq_status tq_workspace_status(void *workspace, int clear, void *stream);
  */
 TQ_API void tq_debug_set_flags(uint32_t flags);
 
+/*
+ * tq_gemv_static_scratch -- the GEMV of tq_gemv for callers that cannot
+ * allocate device memory (code inside an allocator or memory-pool callback,
+ * plugins that only receive an operation's tensors, processes whose device
+ * memory is all reserved up front).  The pages this library follows have no
+ * counterpart to it: it exists only for such callers.
+ *
+ * Inputs and outputs are as for tq_gemv (x: k elements, y: n elements, both
+ * device memory supplied by the caller); no workspace is passed.  Instead the
+ * scratch lives in one fixed device array of TQ_STATIC_SCRATCH_BYTES inside
+ * the library, present on every GPU that loads it until the process exits.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine) and returns TQ_ERR_SHAPE when the problem's scratch,
+ * tq_gemm_workspace_bytes(1, n, k), exceeds TQ_STATIC_SCRATCH_BYTES.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array, and each starts by
+ * clearing what must start at zero: calls that overlap on the GPU (other
+ * streams, other host threads, without ordering between them) race and give
+ * wrong results.  Run them in order on one stream, or use tq_gemv.
+ */
+#define TQ_STATIC_SCRATCH_BYTES (4u << 20)
+
+TQ_API tq_status tq_gemv_static_scratch(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
+                                        const void *x, tq_dtype xt, void *y, tq_dtype yt, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
