@@ -13,10 +13,12 @@ The step is captured once in a CUDA graph and replayed.
 
 Reported:
   value      GEMV weight GB/s = packed layer bytes (codes + scales) / GEMV
-             phase time (the seven pre-rotate + fused-GEMV launches), L2
-             flushed before every timed replay, CUDA events on the stream;
-  quantize   Gweights/s of the quantise phase (same protocol);
-  ms_per_step  the full step (graph replay), inputs resident in HBM;
+             phase time (one batched pre-rotation + fused-product pass over
+             the seven matrices), steady state: 10 passes per graph replay,
+             alternating with an independent shadow layer so that every pass
+             reads its packed weights from HBM; CUDA events on the stream;
+  quantize   Gweights/s of the quantise phase (10 passes per replay);
+  ms_per_step  the full step (10 steps per graph replay), inputs in HBM;
   e2e        the same GB/s metric through the public API with host buffers:
              every step copies the bf16 weights and activations from pinned
              host memory, runs the path and reads the outputs back;
@@ -198,6 +200,24 @@ class Path:
         inputs, one fused-product launch."""
         self.tq.gemm_batch(self.batch, m=1, ws=self.ws, descs=self.descs)
 
+    def add_shadow(self, mats, acts, device):
+        """A second, independent layer (packed once) so that timed GEMV passes
+        can alternate between two layers whose packed weights together exceed
+        the 126 MB L2: every pass then reads its weights from HBM."""
+        self.shadow = []
+        for label, W, act in mats:
+            n, k = W.shape
+            codes, scales = self.tq.quantize(W)
+            self.shadow.append((codes, scales, n, k, acts[act].view(1, -1),
+                                torch.empty((1, n), dtype=torch.float32, device=device)))
+        self.shadow_descs = self.tq.batch_descs(self.shadow)
+        self.shadow_ws = self.tq.batch_workspace(self.shadow, 1, device)
+
+    def gemv_pair(self):
+        """The layer's batched GEMV, then the shadow layer's."""
+        self.gemv()
+        self.tq.gemm_batch(self.shadow, m=1, ws=self.shadow_ws, descs=self.shadow_descs)
+
     def gemv_one(self, i):
         it = self.items[i]
         return lambda: self.tq.gemv(it["codes"], it["scales"], it["n"], it["k"], it["x"][0], out=it["y"][0],
@@ -231,9 +251,15 @@ class Path:
         return sum(it["y"].numel() * 4 for it in self.items)
 
 
-def capture(fn, use_graph: bool):
+def capture(fn, use_graph: bool, repeat: int = 1):
+    """A callable that runs `fn` `repeat` times: one CUDA graph replay (or
+    eager launches without graphs)."""
+    def body():
+        for _ in range(repeat):
+            fn()
+
     if not use_graph:
-        return fn
+        return body
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
@@ -242,7 +268,7 @@ def capture(fn, use_graph: bool):
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        fn()
+        body()
     return g.replay
 
 
@@ -334,6 +360,9 @@ def run_ours(args, world, rank, local):
     tq.load_library()  # raises: there is no CPU path
     mats, acts, desc = make_workload(args.workload, rank, device)
     path = Path(tq, mats, acts, device)
+    smats, sacts, _ = make_workload(args.workload, rank + 1000, device)
+    path.add_shadow(smats, sacts, device)
+    del smats, sacts
     nmat = len(path.items)
     launches_per_step = 2 * nmat + 2  # quantize + dequantize per matrix; one pre-rotation + one fused product
     warmup = max(3, args.warmup)
@@ -347,15 +376,22 @@ def run_ours(args, world, rank, local):
         path.step()
     torch.cuda.synchronize()
     use_graph = not args.no_graph
+    # Steady-state timing: R passes back to back inside one graph replay, so
+    # the per-replay launch latency of the graph is amortised.  Quantise and
+    # dequantise stream >400 MB per pass (far above L2); the GEMV passes
+    # alternate between the layer and an independent shadow layer (together
+    # 2 x 136 MB of packed weights), so every pass reads its weights from HBM.
+    R = 10
     try:
-        step_run = capture(path.step, use_graph)
-        q_run = capture(path.quantize, use_graph)
-        d_run = capture(path.dequantize, use_graph)
-        g_run = capture(path.gemv, use_graph)
+        step_run = capture(path.step, use_graph, R)
+        q_run = capture(path.quantize, use_graph, R)
+        d_run = capture(path.dequantize, use_graph, R)
+        g_run = capture(path.gemv_pair, use_graph, R // 2)
     except Exception as e:  # graph capture refused: launch eagerly
         print(f"[bench] CUDA graph capture failed ({e}); launching eagerly", file=sys.stderr)
         use_graph = False
-        step_run, q_run, d_run, g_run = path.step, path.quantize, path.dequantize, path.gemv
+        step_run, q_run, d_run, g_run = (capture(path.step, False, R), capture(path.quantize, False, R),
+                                         capture(path.dequantize, False, R), capture(path.gemv_pair, False, R // 2))
     for run in (step_run, q_run, d_run, g_run):
         for _ in range(warmup):
             run()
@@ -383,8 +419,8 @@ def run_ours(args, world, rank, local):
     clocks = sampler.stop()
     t_step, t_q, t_d, t_g = max_over_ranks([t_step, t_q, t_d, t_g], world)
 
-    ms_step = t_step / steps
-    ms_q, ms_d, ms_g = t_q / steps, t_d / steps, t_g / steps
+    ms_step = t_step / (steps * R)
+    ms_q, ms_d, ms_g = t_q / (steps * R), t_d / (steps * R), t_g / (steps * R)
     packed = path.packed_bytes()
     weights = path.weights()
     hbm, hbm_kind = measured_peaks()
@@ -420,7 +456,10 @@ def run_ours(args, world, rank, local):
         "roofline": dict(rooflines[dominant], kernel=dominant, peak_note=f"{hbm_kind} HBM copy bandwidth"),
         "rooflines": rooflines,
         "clocks": clocks,
-        "gpu_launches": launches_per_step * steps,
+        "gpu_launches": launches_per_step * steps * R,
+        "timing": {"passes_per_replay": R, "replays": steps,
+                   "gemv": "passes alternate between the layer and an independent shadow layer (2 x packed bytes > L2)",
+                   "single_matrix": "one tq_gemv per graph replay, L2 flushed before each; includes graph launch latency"},
     }
 
     if not args.skip_e2e:

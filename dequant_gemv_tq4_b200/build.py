@@ -34,15 +34,16 @@ def stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not stale():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str | None = None, defines=()) -> str:
+    target = out or LIB
+    if not force and out is None and not stale():
         return LIB
-    tmp = LIB + f".{os.getpid()}.tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose_ptxas else []), "-o", tmp,
-           *[os.path.join(CSRC, s) for s in SOURCES]]
+    tmp = target + f".{os.getpid()}.tmp"
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose_ptxas else []), *[f"-D{d}" for d in defines],
+           "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
     subprocess.run(cmd, check=True, cwd=CSRC)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

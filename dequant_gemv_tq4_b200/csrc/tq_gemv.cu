@@ -42,9 +42,15 @@ namespace tq {
 
 namespace {
 
-constexpr int kWarps = 16;
+#ifndef TQ_GEMV_WARPS
+#define TQ_GEMV_WARPS 16
+#endif
+#ifndef TQ_GEMV_STAGES
+#define TQ_GEMV_STAGES 3
+#endif
+constexpr int kWarps = TQ_GEMV_WARPS;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 3;    // ring stages per warp
+constexpr int kStages = TQ_GEMV_STAGES;  // ring stages per warp
 constexpr int kPerStage = 2;  // consecutive units per stage
 constexpr int kUnitCodeBytes = 1024;
 constexpr int kUnitScaleBytes = 256;
@@ -55,22 +61,23 @@ constexpr int kStageBytes = kPerStage * kUnitBytes;    // 2560
 constexpr int kRingWarpBytes = kStages * kStageBytes;  // 7680
 // Shared-memory map (addresses in the CTA's shared window; the dynamic
 // allocation starts at a small base B <= kMaxSmemBase):
-//   [B, B + 8 rings)            rings of warps 0..7
+//   [B, B + kWarps/2 rings)     rings of the first half of the warps
 //   [0x10000, 0x20000)          lookup table, 64 KB aligned so that one PRMT
 //                               yields the full address of an entry
-//   [0x20000, + 8 rings)        rings of warps 8..15
+//   [0x20000, + kWarps/2 rings) rings of the second half
 //   then the mbarriers
+constexpr int kLowWarps = kWarps / 2;
 constexpr uint32_t kLutAddr = 0x10000;
-constexpr uint32_t kMaxSmemBase = 0x10000 - 8 * kRingWarpBytes;  // 4096
+constexpr uint32_t kMaxSmemBase = 0x10000 - kLowWarps * kRingWarpBytes;
 constexpr uint32_t kHighRings = 0x20000;
-constexpr uint32_t kBarAddr = kHighRings + 8 * kRingWarpBytes;
+constexpr uint32_t kBarAddr = kHighRings + (kWarps - kLowWarps) * kRingWarpBytes;
 constexpr uint32_t kBarBytes = kWarps * kStages * 8;
+static_assert(kMaxSmemBase >= 1024 && kMaxSmemBase < 0x10000, "ring placement below the table");
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusLayout = 2u;
 constexpr uint64_t kTimeoutNs = 1000000000ull;     // 1 s
 constexpr uint64_t kDebugTimeoutNs = 5000000ull;   // 5 ms under fault injection
 
-static_assert(kWarps == 16, "the shared-memory map places 8 rings below and 8 above the table");
 
 // Dynamic shared memory to request for a dynamic base of `base` bytes.
 inline uint32_t smem_bytes_for_base(uint32_t base) { return kBarAddr + kBarBytes - base; }
@@ -227,7 +234,7 @@ __device__ __forceinline__ void issue_stage(const GroupParams &P, Cursor &cu, in
 // Write the accumulators of a finished tile segment: straight to Y when this
 // warp covered the whole tile, else through the fixed-order partial sums.
 template <int NT, bool M1, int OT>
-__device__ __noinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
+__device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
                                            int u1, int gw, const float (&acc)[NT][4]) {
     constexpr int kMcap = 8 * NT;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
@@ -301,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         if (threadIdx.x == 0) atomicOr(P.status, kStatusLayout);
         return;
     }
-    const uint32_t ring = (warp < 8 ? base : kHighRings) + (warp & 7) * kRingWarpBytes;
+    const uint32_t ring =
+        warp < kLowWarps ? base + warp * kRingWarpBytes : kHighRings + (warp - kLowWarps) * kRingWarpBytes;
     const uint32_t bars = kBarAddr + warp * (kStages * 8);
     const bool active = gw < P.total_warps;
     const int U = (int)P.units;
@@ -329,16 +337,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         }
     }
     {
-        // entry v holds the same half2 in all 32 lane slots: 8 x 16-byte stores
-        // per entry, two threads per entry
+        // entry v holds the same half2 in all 32 lane slots (the first 128 of
+        // its 256 bytes)
         uint4 *lut = reinterpret_cast<uint4 *>(smem + (kLutAddr - base));
-        const int v = threadIdx.x >> 1, part = threadIdx.x & 1;
-        const uint32_t lo = c_mag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
-        const uint32_t hi = c_mag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
-        const uint32_t e = lo | (hi << 16);
-        const uint4 e4 = make_uint4(e, e, e, e);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) lut[v * 16 + part * 4 + i] = e4;
+        for (int idx = threadIdx.x; idx < 256 * 8; idx += kThreads) {  // entry v: 8 x 16 bytes
+            const int v = idx >> 3;
+            const uint32_t lo = c_mag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
+            const uint32_t hi = c_mag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
+            const uint32_t e = lo | (hi << 16);
+            lut[v * 16 + (idx & 7)] = make_uint4(e, e, e, e);
+        }
     }
     __syncthreads();
     grid_dependency_wait();  // pre-rotated activations and counters are ready
@@ -347,6 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     const int g = lane >> 2, t = lane & 3;
     // PRMT operand: byte 0 = lane*4, bytes 2..3 = table base >> 16
     const uint32_t lut_lane = kLutAddr | ((uint32_t)lane * 4u);
+    // this lane's 16 code bytes of rows g and g+8, and its scale words, in a unit
+    const uint32_t off_c = g * 64 + t * 16, off_s = g * 16;
 
     // ---- segment state: the tile the current unit belongs to ---------------
     int q = problem_of(P, u0);
@@ -375,36 +385,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
 #pragma unroll
         for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
 
-    int u = u0;
     int stage = 0;
     uint32_t parity = 0;
-    while (u < u1) {
-        const uint32_t st = ring + stage * kStageBytes, bar = bars + 8 * stage;
-        bool ok = mbar_try(bar, parity);
-        if (!__all_sync(kFull, ok)) {
-            ok = ok || mbar_wait_slow(bar, parity, P.timeout_ns);
+    uint32_t st = ring, bar = bars;
+    for (int u = u0; u < u1; ++u) {
+        const int h = (u - u0) & 1;  // position of the unit in its stage
+        if (h == 0) {                // warp-uniform: a new stage
+            st = ring + stage * kStageBytes;
+            bar = bars + 8 * stage;
+            bool ok = mbar_try(bar, parity);
             if (!__all_sync(kFull, ok)) {
-                // report, then let the copies still in flight land before leaving
-                if (lane == 0) {
-                    atomicOr(P.status, kStatusTimeout);
-                    int s2 = stage;
-                    uint32_t p2 = parity;
-                    for (int i = 1; i < kStages && u + kPerStage * i < pv; ++i) {
-                        if (++s2 == kStages) { s2 = 0; p2 ^= 1u; }
-                        mbar_wait_slow(bars + 8 * s2, p2, P.timeout_ns);
+                ok = ok || mbar_wait_slow(bar, parity, P.timeout_ns);
+                if (!__all_sync(kFull, ok)) {
+                    // report, then let the copies still in flight land before leaving
+                    if (lane == 0) {
+                        atomicOr(P.status, kStatusTimeout);
+                        int s2 = stage;
+                        uint32_t p2 = parity;
+                        for (int i = 1; i < kStages && u + kPerStage * i < pv; ++i) {
+                            if (++s2 == kStages) { s2 = 0; p2 ^= 1u; }
+                            mbar_wait_slow(bars + 8 * s2, p2, P.timeout_ns);
+                        }
                     }
+                    __syncwarp();
+                    return;
                 }
-                __syncwarp();
-                return;
             }
         }
-#pragma unroll 1
-        for (int h = 0; h < kPerStage && u < u1; ++h) {
+        {
             const uint32_t sc = st + h * kUnitCodeBytes, ss = st + kStageScaleOff + h * kUnitScaleBytes;
-            const uint4 c0 = lds128(sc + g * 64 + t * 16);
-            const uint4 c1 = lds128(sc + (g + 8) * 64 + t * 16);
-            const uint4 s0 = lds128(ss + g * 16);
-            const uint4 s1 = lds128(ss + (g + 8) * 16);
+            const uint4 c0 = lds128(sc + off_c);
+            const uint4 c1 = lds128(sc + off_c + 512);
+            const uint4 s0 = lds128(ss + off_s);
+            const uint4 s1 = lds128(ss + off_s + 128);
             const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
             const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
             const uint32_t sw0[4] = {s0.x, s0.y, s0.z, s0.w};
@@ -445,44 +458,44 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                     }
                 }
             }
-            ++u;
-            ++sb;
-            if (u == seg_end) {  // warp-uniform
-                flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, acc);
+        }
+        ++sb;
+        if (u + 1 == seg_end) {  // warp-uniform: the tile segment is complete
+            flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, acc);
 #pragma unroll
-                for (int a = 0; a < NT; ++a)
+            for (int a = 0; a < NT; ++a)
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-                if (u < u1) {
-                    if (u == prob_end) {  // next problem: new tiles, new activation
-                        ++q;
-                        prob_end = problem_end(P, q);
-                        nsb = P.prob[q].nsb;
-                        r = 0;
-                        tile_lo = u;
+                for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+            if (u + 1 < u1) {
+                if (u + 1 == prob_end) {  // next problem: new tiles, new activation
+                    ++q;
+                    prob_end = problem_end(P, q);
+                    nsb = P.prob[q].nsb;
+                    r = 0;
+                    tile_lo = u + 1;
 #pragma unroll
-                        for (int a = 0; a < NT; ++a) {
-                            const int xrow = min(8 * a + g, P.m - 1);
-                            xbase[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
-                        }
-                    } else {
-                        ++r;
-                        tile_lo += nsb;
+                    for (int a = 0; a < NT; ++a) {
+                        const int xrow = min(8 * a + g, P.m - 1);
+                        xbase[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
                     }
-                    sb = 0;
-                    seg_end = min(tile_lo + nsb, u1);
+                } else {
+                    ++r;
+                    tile_lo += nsb;
                 }
+                sb = 0;
+                seg_end = min(tile_lo + nsb, u1);
             }
         }
-        // every lane has consumed this stage: refill it with the next units
-        __syncwarp();
-        if (pv < u1) {  // warp-uniform
-            const int cnt = min(kPerStage, u1 - pv);
-            issue_stage(P, cu, cnt, st, bar, lane == 0);
-            pv += cnt;
+        if (h == kPerStage - 1 || u + 1 == u1) {  // warp-uniform: the stage is consumed
+            __syncwarp();
+            if (pv < u1) {
+                const int cnt = min(kPerStage, u1 - pv);
+                issue_stage(P, cu, cnt, st, bar, lane == 0);
+                pv += cnt;
+            }
+            stage = (stage == kStages - 1) ? 0 : stage + 1;
+            parity ^= (stage == 0) ? 1u : 0u;
         }
-        stage = (stage == kStages - 1) ? 0 : stage + 1;
-        parity ^= (stage == 0) ? 1u : 0u;
     }
 }
 
