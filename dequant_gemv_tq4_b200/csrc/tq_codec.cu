@@ -329,6 +329,11 @@ __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_
 // -------------------------------------------------------------------------
 template <int DT>
 __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_constant__ RotParams prm) {
+    // Launched as a programmatic dependent of the previous kernel in the
+    // stream: wait until every earlier kernel has completed (and its memory is
+    // visible), then let the fused product that follows start its prologue,
+    // which reads packed weights that earlier kernels may have written.
+    grid_dependency_wait();
     grid_dependents_launch();
     const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     for (int64_t i = gtid; i < prm.counters_count; i += (int64_t)gridDim.x * blockDim.x) prm.counters[i] = 0u;
@@ -432,13 +437,21 @@ cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m
     prm.counters_count = counters ? counters_count : 0;
     int64_t grid = (units + kCodecWarps - 1) / kCodecWarps;
     if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kCodecThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     switch (dtype) {
-        case kF32: prerotate_kernel<kF32><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
-        case kBF16: prerotate_kernel<kBF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
-        case kF16: prerotate_kernel<kF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
+        case kF32: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32>, prm);
+        case kBF16: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16>, prm);
+        case kF16: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16>, prm);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace tq

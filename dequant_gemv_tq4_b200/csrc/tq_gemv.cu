@@ -350,6 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     }
     __syncthreads();
     grid_dependency_wait();  // pre-rotated activations and counters are ready
+    // every CTA of this grid is resident: the next pre-rotation may launch and
+    // wait (it waits for this grid's completion before writing anything)
+    grid_dependents_launch();
     if (!active) return;
 
     const int g = lane >> 2, t = lane & 3;
@@ -371,12 +374,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     }
     int seg_end = min(tile_lo + nsb, u1);
     // activation fragments: rows past m repeat row m-1 (their outputs are never
-    // stored), so every lane loads without a predicate
-    const uint16_t *xbase[NT];
+    // stored), so every lane loads without a predicate; xcur[a] walks the
+    // superblocks of the current unit (128 halves per superblock)
+    const uint16_t *xcur[NT];
 #pragma unroll
     for (int a = 0; a < NT; ++a) {
         const int xrow = min(8 * a + g, P.m - 1);
-        xbase[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
+        xcur[a] = P.prob[q].xrot + ((int64_t)xrow * nsb + sb) * 128 + t * 8;
     }
 
     float acc[NT][4];
@@ -422,12 +426,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
             const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
             const uint32_t sw0[4] = {s0.x, s0.y, s0.z, s0.w};
             const uint32_t sw1[4] = {s1.x, s1.y, s1.z, s1.w};
-            const int xoff = sb * 128;
 #pragma unroll
             for (int j = 0; j < kSbBlocks; ++j) {
                 uint4 xb[NT];
 #pragma unroll
-                for (int a = 0; a < NT; ++a) xb[a] = ldg_keep(xbase[a] + xoff + j * 32);
+                for (int a = 0; a < NT; ++a) xb[a] = ldg_keep(xcur[a] + j * 32);
                 // code byte b of word cw: logical byte t + 4b of the block
                 const uint32_t a00 = lds_u32(prmt(cw0[j], lut_lane, 0x7604u));
                 const uint32_t a01 = lds_u32(prmt(cw1[j], lut_lane, 0x7604u));
@@ -460,6 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
             }
         }
         ++sb;
+#pragma unroll
+        for (int a = 0; a < NT; ++a) xcur[a] += 128;
         if (u + 1 == seg_end) {  // warp-uniform: the tile segment is complete
             flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, acc);
 #pragma unroll
@@ -473,17 +478,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                     nsb = P.prob[q].nsb;
                     r = 0;
                     tile_lo = u + 1;
-#pragma unroll
-                    for (int a = 0; a < NT; ++a) {
-                        const int xrow = min(8 * a + g, P.m - 1);
-                        xbase[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
-                    }
                 } else {
                     ++r;
                     tile_lo += nsb;
                 }
                 sb = 0;
                 seg_end = min(tile_lo + nsb, u1);
+#pragma unroll
+                for (int a = 0; a < NT; ++a) {  // back to superblock 0 of the activation
+                    const int xrow = min(8 * a + g, P.m - 1);
+                    xcur[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
+                }
             }
         }
         if (h == kPerStage - 1 || u + 1 == u1) {  // warp-uniform: the stage is consumed
