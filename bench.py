@@ -89,6 +89,35 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+PROFILE_FILES = {  # phase -> committed ncu summary and the sources its kernel is built from
+    "quantize": ("quantize_kernel_llama3_8b_down.md", ("tq_device.cuh", "tq_codec.cu")),
+    "dequantize": ("dequantize_kernel_llama3_8b_down.md", ("tq_device.cuh", "tq_codec.cu")),
+    "gemv": ("gemv_group_kernel_llama3_8b_layer.md", ("tq_device.cuh", "tq_gemv.cu")),
+}
+
+
+def profile_traffic(phase: str, weights: int):
+    """DRAM bytes (read + write) of one pass of `phase` from the committed ncu
+    capture, scaled by the weights processed (traffic grows in proportion to
+    the units), or None when the kernel source changed since the capture."""
+    import hashlib
+
+    name, sources = PROFILE_FILES[phase]
+    try:
+        text = open(os.path.join(ROOT, "profiles", name)).read()
+        fields = dict(ln.split(": ", 1) for ln in text.splitlines() if ": " in ln and ln.split(": ", 1)[0] in
+                      ("traffic_bytes_per_launch", "weights_per_launch", "source_sha256"))
+        h = hashlib.sha256()
+        for src in sources:
+            with open(os.path.join(ROOT, "dequant_gemv_tq4_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != fields["source_sha256"].strip():
+            return None
+        return int(round(int(fields["traffic_bytes_per_launch"]) * weights / int(fields["weights_per_launch"])))
+    except Exception:
+        return None
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
 
@@ -437,8 +466,8 @@ def run_ours(args, world, rank, local):
     for ph, (nbytes, ms, nl) in alg.items():
         ach = nbytes / (ms * 1e-3) / 1e9
         rooflines[ph] = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(ach / hbm, 4), "traffic": None, "bytes_per_step": nbytes,
-                         "ms": round(ms, 5), "launches": nl}
+                         "frac": round(ach / hbm, 4), "traffic": profile_traffic(ph, weights),
+                         "bytes_per_step": nbytes, "ms": round(ms, 5), "launches": nl}
     dominant = max(("quantize", "dequantize", "gemv"), key=lambda ph: alg[ph][1])
 
     line = {
