@@ -75,6 +75,18 @@ def _load():
             lib.tqo_unpack.argtypes = [P, P, I64, I64, P, P]
             lib.tqo_dequantize.argtypes = [P, P, I64, I64, P, I64]
             lib.tqo_gemm.argtypes = [P, P, I64, I64, P, I64, I64, P, I64]
+            lib.tqo_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+            lib.tqo_e4m3_to_f32.restype = ctypes.c_float
+            lib.tqo_e4m3_from_f32.argtypes = [ctypes.c_float]
+            lib.tqo_e4m3_from_f32.restype = ctypes.c_uint8
+            lib.tqo_e2m1_to_f32.argtypes = [ctypes.c_uint8]
+            lib.tqo_e2m1_to_f32.restype = ctypes.c_float
+            lib.tqo_e2m1_from_f32.argtypes = [ctypes.c_float]
+            lib.tqo_e2m1_from_f32.restype = ctypes.c_uint8
+            lib.tqo_nvfp4_quantize.argtypes = [P, I64, I64, I64, P, P, P]
+            lib.tqo_nvfp4_quantize.restype = ctypes.c_int
+            lib.tqo_nvfp4_dequantize.argtypes = [P, P, ctypes.c_float, I64, I64, P, I64]
+            lib.tqo_nvfp4_gemm.argtypes = [P, P, ctypes.c_float, I64, I64, P, I64, I64, P, I64]
             _lib = lib
     return _lib
 
@@ -235,4 +247,65 @@ def gemm(codes: np.ndarray, scales: np.ndarray, n: int, k: int, X: np.ndarray) -
     m = X.shape[0]
     Y = np.zeros((m, n), np.float64)
     lib.tqo_gemm(_ptr(codes), _ptr(scales), n, k, _ptr(X), m, k, _ptr(Y), n)
+    return Y
+
+
+# --------------------------------------------------------------------------
+# NVFP4 comparison codec
+# --------------------------------------------------------------------------
+def e4m3_to_f32(c) -> np.ndarray:
+    lib = _load()
+    return np.array([lib.tqo_e4m3_to_f32(int(v)) for v in np.asarray(c, np.uint8).ravel()], np.float32)
+
+
+def e4m3_from_f32(x) -> np.ndarray:
+    lib = _load()
+    return np.array([lib.tqo_e4m3_from_f32(float(v)) for v in np.asarray(x, np.float32).ravel()], np.uint8)
+
+
+def e2m1_to_f32(c) -> np.ndarray:
+    lib = _load()
+    return np.array([lib.tqo_e2m1_to_f32(int(v)) for v in np.asarray(c, np.uint8).ravel()], np.float32)
+
+
+def e2m1_from_f32(x) -> np.ndarray:
+    lib = _load()
+    return np.array([lib.tqo_e2m1_from_f32(float(v)) for v in np.asarray(x, np.float32).ravel()], np.uint8)
+
+
+def nvfp4_scales_bytes(n: int, k: int) -> int:
+    return tiles(n) * superblocks(k) * 128
+
+
+def nvfp4_quantize(W: np.ndarray):
+    """W float32 [n, k] (k % 32 == 0) -> (codes uint8 [T*NSB*1024], scales uint8 [T*NSB*128], g float)."""
+    lib = _load()
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    n, k = W.shape
+    if k % 32 != 0:
+        raise ValueError("k must be a multiple of 32")
+    codes = np.zeros(codes_bytes(n, k), np.uint8)
+    scales = np.zeros(nvfp4_scales_bytes(n, k), np.uint8)
+    g = np.zeros(1, np.float32)
+    lib.tqo_nvfp4_quantize(_ptr(W), n, k, k, _ptr(codes), _ptr(scales), _ptr(g))
+    return codes, scales, float(g[0])
+
+
+def nvfp4_dequantize(codes, scales, g: float, n: int, k: int) -> np.ndarray:
+    lib = _load()
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    W = np.zeros((n, k), np.float64)
+    lib.tqo_nvfp4_dequantize(_ptr(codes), _ptr(scales), float(g), n, k, _ptr(W), k)
+    return W
+
+
+def nvfp4_gemm(codes, scales, g: float, n: int, k: int, X: np.ndarray) -> np.ndarray:
+    lib = _load()
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    X = np.ascontiguousarray(np.atleast_2d(X), dtype=np.float64)
+    m = X.shape[0]
+    Y = np.zeros((m, n), np.float64)
+    lib.tqo_nvfp4_gemm(_ptr(codes), _ptr(scales), float(g), n, k, _ptr(X), m, k, _ptr(Y), n)
     return Y

@@ -375,3 +375,147 @@ void tqo_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k
     free(w);
     free(tile);
 }
+
+/* ======================================================================== */
+/* NVFP4 comparison codec (the llm-compressor and llama.cpp-quantizer pages */
+/* name NVFP4 checkpoints and "weight and input tensor scales"; the pages   */
+/* give no bit recipe, so this is the plainest reading of the format):      */
+/*   g   = amax|W| / (6 * 448)                      per-tensor fp32 scale    */
+/*   s_b = e4m3_rne_satfinite(amax_b / (6 * g))      per 16-element block     */
+/*   q   = e2m1_rne_satfinite(w / (s_b * g))         per element (0 if s_b=0) */
+/*   w~  = q * s_b * g                                                       */
+/* Every quotient / product is one IEEE fp32 operation in that order.       */
+/* ======================================================================== */
+
+/* E4M3 (bias 7, no infinities, max 448): value of an 8-bit code. */
+float tqo_e4m3_to_f32(uint8_t c) {
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    float v;
+    if (e == 15 && m == 7) v = NAN;
+    else if (e == 0) v = ldexpf((float)m, -9);
+    else v = ldexpf((float)(8 + m), e - 10);
+    return s ? -v : v;
+}
+
+/* Nearest E4M3 code, ties to the even code, finite values above 448 saturate. */
+uint8_t tqo_e4m3_from_f32(float x) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    float a = fabsf(x);
+    if (a >= 448.0f) return sign | 0x7E;
+    /* scan the 127 finite magnitudes in increasing order */
+    uint8_t best = 0;
+    for (int c = 1; c <= 0x7E; ++c) {
+        float v = tqo_e4m3_to_f32((uint8_t)c);
+        if (v <= a) best = (uint8_t)c;
+    }
+    if (best == 0x7E) return sign | best;
+    float lo = tqo_e4m3_to_f32(best), hi = tqo_e4m3_to_f32((uint8_t)(best + 1));
+    double dl = (double)a - lo, dh = (double)hi - a;
+    uint8_t r = best;
+    if (dh < dl || (dh == dl && (best & 1))) r = (uint8_t)(best + 1);
+    return sign | r;
+}
+
+/* E2M1 magnitudes by 3-bit code: 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+float tqo_e2m1_to_f32(uint8_t c) {
+    static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    float v = mag[c & 7];
+    return (c & 8) ? -v : v;
+}
+
+/* Nearest E2M1 code (bit 3 = sign), ties to the even code, saturating at 6.
+ * -0 and +0 both map to code 0 (a zero carries no sign). */
+uint8_t tqo_e2m1_from_f32(float x) {
+    uint8_t sign = (x < 0.0f) ? 8 : 0;
+    float a = fabsf(x);
+    if (a >= 6.0f) return sign | 7;
+    uint8_t best = 0;
+    for (int c = 1; c <= 7; ++c)
+        if (tqo_e2m1_to_f32((uint8_t)c) <= a) best = (uint8_t)c;
+    uint8_t r = best;
+    if (best < 7) {
+        float lo = tqo_e2m1_to_f32(best), hi = tqo_e2m1_to_f32((uint8_t)(best + 1));
+        float dl = a - lo, dh = hi - a; /* exact: all operands are short binary fractions */
+        if (dh < dl || (dh == dl && (best & 1))) r = (uint8_t)(best + 1);
+    }
+    return r == 0 ? 0 : (uint8_t)(sign | r);
+}
+
+/* Packed NVFP4 layout (this repository's): the same tile-major units as
+ * TQ4_1S -- codes [T][NSB][16 rows][64 B] with the same byte order inside a
+ * row's 64 bytes (a pair of 16-element blocks plays the role of one 32-element
+ * block), scales E4M3 [T][NSB][16 rows][8 blocks], plus one fp32 tensor scale.
+ * k must be a multiple of 32.  4.5 bits per weight. */
+static int64_t tqo_nv_scale_offset(int64_t nsb, int64_t row, int64_t blk16) {
+    int64_t sb = blk16 / 8;
+    return (((row / 16) * nsb + sb) * 16 + row % 16) * 8 + blk16 % 8;
+}
+
+int tqo_nvfp4_quantize(const float *W, int64_t n, int64_t k, int64_t ldw, uint8_t *codes, uint8_t *scales,
+                       float *g_out) {
+    if (k % TQO_BLOCK != 0 || n < 0) return 1;
+    int64_t nsb = tqo_superblocks(k), nb16 = k / 16;
+    memset(codes, 0, (size_t)(tqo_tiles(n) * nsb * 1024));
+    memset(scales, 0, (size_t)(tqo_tiles(n) * nsb * 128));
+    float amax = 0.0f;
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t c = 0; c < k; ++c) {
+            float a = fabsf(W[r * ldw + c]);
+            if (a > amax) amax = a;
+        }
+    float g = amax / (6.0f * 448.0f);
+    *g_out = g;
+    float denom = 6.0f * g;
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t b = 0; b < nb16; ++b) {
+            const float *w = W + r * ldw + b * 16;
+            float am = 0.0f;
+            for (int e = 0; e < 16; ++e)
+                if (fabsf(w[e]) > am) am = fabsf(w[e]);
+            uint8_t s = (denom > 0.0f) ? tqo_e4m3_from_f32(am / denom) : 0;
+            float scale = tqo_e4m3_to_f32(s) * g;
+            scales[tqo_nv_scale_offset(nsb, r, b)] = s;
+            for (int e = 0; e < 16; ++e) {
+                uint8_t q = (scale > 0.0f) ? tqo_e2m1_from_f32(w[e] / scale) : 0;
+                int64_t blk32 = b / 2;
+                int el = (int)(b % 2) * 16 + e; /* element index inside the 32-column pair */
+                int L = el / 2;
+                int64_t off = tqo_code_offset(nsb, r, blk32, L);
+                codes[off] |= (uint8_t)((el & 1) ? (q << 4) : q);
+            }
+        }
+    return 0;
+}
+
+void tqo_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, float g, int64_t n, int64_t k, double *W,
+                          int64_t ldw) {
+    int64_t nsb = tqo_superblocks(k), nb16 = k / 16;
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t b = 0; b < nb16; ++b) {
+            double s = (double)tqo_e4m3_to_f32(scales[tqo_nv_scale_offset(nsb, r, b)]) * (double)g;
+            for (int e = 0; e < 16; ++e) {
+                int el = (int)(b % 2) * 16 + e;
+                uint8_t byte = codes[tqo_code_offset(nsb, r, b / 2, el / 2)];
+                uint8_t q = (el & 1) ? (byte >> 4) : (byte & 15);
+                W[r * ldw + b * 16 + e] = (double)tqo_e2m1_to_f32(q) * s;
+            }
+        }
+}
+
+/* Y[m][r] = sum_k w~[r][k] X[m][k] over the NVFP4 reconstruction, fp64. */
+void tqo_nvfp4_gemm(const uint8_t *codes, const uint8_t *scales, float g, int64_t n, int64_t k, const double *X,
+                    int64_t m, int64_t ldx, double *Y, int64_t ldy) {
+    double *tile = (double *)malloc((size_t)16 * (size_t)(k > 0 ? k : 1) * sizeof(double));
+    int64_t nsb = tqo_superblocks(k);
+    for (int64_t r = 0; r < n; ++r) {
+        if (r % 16 == 0) tqo_nvfp4_dequantize(codes + (r / 16) * nsb * 1024, scales + (r / 16) * nsb * 128, g, 16, k,
+                                              tile, k);
+        for (int64_t i = 0; i < m; ++i) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < k; ++c) acc += tile[(r % 16) * k + c] * X[i * ldx + c];
+            Y[i * ldy + r] = acc;
+        }
+    }
+    free(tile);
+}
