@@ -38,6 +38,16 @@ class GemmDesc(ctypes.Structure):
                 ("k", ctypes.c_int64), ("X", ctypes.c_void_p), ("ldx", ctypes.c_int64), ("Y", ctypes.c_void_p),
                 ("ldy", ctypes.c_int64)]
 
+
+class Nvfp4GemmDesc(ctypes.Structure):
+    """Mirror of ``tq_nvfp4_gemm_desc`` in include/tq.h."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("X", ctypes.c_void_p), ("ldx", ctypes.c_int64),
+                ("Y", ctypes.c_void_p), ("ldy", ctypes.c_int64)]
+
+
+TQ_NVFP4_TENSOR_BYTES = 16
+
 _lock = threading.Lock()
 _lib = None
 
@@ -75,6 +85,12 @@ def load_library() -> ctypes.CDLL:
             "tq_workspace_status": ([P, I, P], I),
             "tq_debug_set_flags": ([ctypes.c_uint32], None),
             "tq_gemv_static_scratch": ([P, P, I64, I64, P, I, P, I, P], I),
+            "tq_nvfp4_scales_bytes": ([I64, I64], SZ),
+            "tq_nvfp4_quantize": ([P, I, I64, I64, I64, P, P, P, P], I),
+            "tq_nvfp4_dequantize": ([P, P, P, I64, I64, P, I, I64, P], I),
+            "tq_nvfp4_gemm": ([P, P, P, I64, I64, P, I, I64, I64, P, I, I64, P, SZ, P], I),
+            "tq_nvfp4_gemm_batch_workspace_bytes": ([ctypes.POINTER(Nvfp4GemmDesc), I, I64], SZ),
+            "tq_nvfp4_gemm_batch": ([ctypes.POINTER(Nvfp4GemmDesc), I, I64, I, I, P, SZ, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -157,6 +173,31 @@ def tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream) -> int:
     device memory: the scratch is a fixed array inside the library (see
     include/tq.h).  Calls that overlap on the GPU must not share it."""
     return load_library().tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream)
+
+
+def tq_nvfp4_scales_bytes(n: int, k: int) -> int:
+    return int(load_library().tq_nvfp4_scales_bytes(n, k))
+
+
+def tq_nvfp4_quantize(w, wt, n, k, ldw, codes, scales, tensor_scale, stream) -> int:
+    return load_library().tq_nvfp4_quantize(w, wt, n, k, ldw, codes, scales, tensor_scale, stream)
+
+
+def tq_nvfp4_dequantize(codes, scales, tensor_scale, n, k, w_out, ot, ldo, stream) -> int:
+    return load_library().tq_nvfp4_dequantize(codes, scales, tensor_scale, n, k, w_out, ot, ldo, stream)
+
+
+def tq_nvfp4_gemm(codes, scales, tensor_scale, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_nvfp4_gemm(codes, scales, tensor_scale, n, k, X, xt, m, ldx, Y, yt, ldy, workspace,
+                                        ws_bytes, stream)
+
+
+def tq_nvfp4_gemm_batch_workspace_bytes(descs, count, m) -> int:
+    return int(load_library().tq_nvfp4_gemm_batch_workspace_bytes(descs, count, m))
+
+
+def tq_nvfp4_gemm_batch(descs, count, m, xt, yt, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_nvfp4_gemm_batch(descs, count, m, xt, yt, workspace, ws_bytes, stream)
 
 
 # ---------------------------------------------------------------------------
@@ -303,3 +344,74 @@ def gemm_batch(items, m: int = 1, ws=None, stream=None, descs=None):
 def workspace_status(ws: torch.Tensor, clear: bool = True, stream=None) -> int:
     """0 (TQ_OK) or 8 (TQ_ERR_TIMEOUT) for the last product that used ``ws``."""
     return tq_workspace_status(ws.data_ptr(), 1 if clear else 0, _stream(stream))
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 comparison codec (tensor helpers)
+# ---------------------------------------------------------------------------
+def nvfp4_quantize(w: torch.Tensor, stream=None):
+    """Encode W (n x k) as NVFP4.  Returns (codes uint8 [tq_codes_bytes],
+    scales uint8 [tq_nvfp4_scales_bytes] of E4M3 bytes, tensor block float32[4]
+    holding g at [0] and amax|W| at [1])."""
+    n, k = w.shape
+    codes = torch.empty(tq_codes_bytes(n, k), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(tq_nvfp4_scales_bytes(n, k), dtype=torch.uint8, device=w.device)
+    tensor = torch.empty(TQ_NVFP4_TENSOR_BYTES // 4, dtype=torch.float32, device=w.device)
+    _check(tq_nvfp4_quantize(w.data_ptr(), _dt(w.dtype), n, k, _ld(w), codes.data_ptr(), scales.data_ptr(),
+                             tensor.data_ptr(), _stream(stream)), "tq_nvfp4_quantize")
+    return codes, scales, tensor
+
+
+def nvfp4_dequantize(codes, scales, tensor, n: int, k: int, dtype=torch.bfloat16, out=None,
+                     stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((n, k), dtype=dtype, device=codes.device)
+    _check(tq_nvfp4_dequantize(codes.data_ptr(), scales.data_ptr(), tensor.data_ptr(), n, k, out.data_ptr(),
+                               _dt(out.dtype), _ld(out), _stream(stream)), "tq_nvfp4_dequantize")
+    return out
+
+
+def nvfp4_gemm(codes, scales, tensor, n: int, k: int, X: torch.Tensor, dtype=torch.float32, out=None, ws=None,
+               stream=None) -> torch.Tensor:
+    """Y[m, n] = X[m, k] @ w~[n, k]^T for NVFP4 weights (m <= 32), fused."""
+    X2 = X.view(1, -1) if X.dim() == 1 else X
+    m = X2.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=dtype, device=X.device)
+    if ws is None:
+        ws = workspace(m, n, k, X.device)
+    _check(tq_nvfp4_gemm(codes.data_ptr(), scales.data_ptr(), tensor.data_ptr(), n, k, X2.data_ptr(),
+                         _dt(X2.dtype), m, _ld(X2), out.data_ptr(), _dt(out.dtype), _ld(out), ws.data_ptr(),
+                         ws.numel(), _stream(stream)), "tq_nvfp4_gemm")
+    return out
+
+
+def nvfp4_batch_descs(items):
+    """items: sequence of (codes, scales, tensor, n, k, X [m, k], Y [m, n])."""
+    arr = (Nvfp4GemmDesc * len(items))()
+    for i, (codes, scales, tensor, n, k, X, Y) in enumerate(items):
+        X2 = X.view(1, -1) if X.dim() == 1 else X
+        Y2 = Y.view(1, -1) if Y.dim() == 1 else Y
+        arr[i] = Nvfp4GemmDesc(codes.data_ptr(), scales.data_ptr(), tensor.data_ptr(), n, k, X2.data_ptr(),
+                               _ld(X2), Y2.data_ptr(), _ld(Y2))
+    return arr
+
+
+def nvfp4_batch_workspace(items, m: int, device=None) -> torch.Tensor:
+    descs = nvfp4_batch_descs(items)
+    nbytes = tq_nvfp4_gemm_batch_workspace_bytes(descs, len(items), m)
+    if nbytes == 0:
+        raise ValueError("invalid batch for workspace query")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or torch.cuda.current_device())
+
+
+def nvfp4_gemm_batch(items, m: int = 1, ws=None, stream=None, descs=None):
+    """NVFP4 products for several matrices in two launches; outputs in place."""
+    if descs is None:
+        descs = nvfp4_batch_descs(items)
+    X0, Y0 = items[0][5], items[0][6]
+    if ws is None:
+        ws = nvfp4_batch_workspace(items, m, X0.device)
+    _check(tq_nvfp4_gemm_batch(descs, len(items), m, _dt(X0.dtype), _dt(Y0.dtype), ws.data_ptr(), ws.numel(),
+                               _stream(stream)), "tq_nvfp4_gemm_batch")
+    return [it[6] for it in items]

@@ -307,6 +307,111 @@ tq_status tq_gemm_batch(const tq_gemm_desc *descs, int count, int64_t m, tq_dtyp
     return from_cuda(e);
 }
 
+// ---- NVFP4 comparison codec -------------------------------------------------
+size_t tq_nvfp4_scales_bytes(int64_t n, int64_t k) {
+    if (check_nk(n, k) != TQ_OK) return 0;
+    return (size_t)tq::tiles(n) * (size_t)tq::superblocks(k) * 128u;
+}
+
+static tq_status check_nv_planes(const uint8_t *codes, const uint8_t *scales, const float *tensor_scale) {
+    if (!codes || !scales || !tensor_scale) return TQ_ERR_INVALID_ARG;
+    if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(tensor_scale, 16)) return TQ_ERR_ALIGNMENT;
+    return TQ_OK;
+}
+
+tq_status tq_nvfp4_quantize(const void *w, tq_dtype wt, int64_t n, int64_t k, int64_t ldw, uint8_t *codes,
+                            uint8_t *scales, float *tensor_scale, void *stream) {
+    tq_status st = check_nk(n, k);
+    if (st != TQ_OK) return st;
+    if (!valid_dtype(wt)) return TQ_ERR_DTYPE;
+    if (n == 0) return TQ_OK;
+    if ((st = check_matrix_operand(w, ldw, k)) != TQ_OK) return st;
+    if ((st = check_nv_planes(codes, scales, tensor_scale)) != TQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    // word 1 of the tensor block accumulates amax|W| (as non-negative float bits)
+    unsigned *amax = reinterpret_cast<unsigned *>(tensor_scale) + 1;
+    if (cudaMemsetAsync(amax, 0, sizeof(unsigned), s) != cudaSuccess) return TQ_ERR_CUDA;
+    if (tq::launch_nvfp4_amax(w, wt, n, k, ldw, amax, s) != cudaSuccess) return TQ_ERR_CUDA;
+    return from_cuda(tq::launch_nvfp4_quantize(w, wt, n, k, ldw, amax, codes, scales, tensor_scale, s));
+}
+
+tq_status tq_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *tensor_scale, int64_t n,
+                              int64_t k, void *w_out, tq_dtype ot, int64_t ldo, void *stream) {
+    tq_status st = check_nk(n, k);
+    if (st != TQ_OK) return st;
+    if (!valid_dtype(ot)) return TQ_ERR_DTYPE;
+    if (n == 0) return TQ_OK;
+    if ((st = check_nv_planes(codes, scales, tensor_scale)) != TQ_OK) return st;
+    if ((st = check_matrix_operand(w_out, ldo, k)) != TQ_OK) return st;
+    return from_cuda(
+        tq::launch_nvfp4_dequantize(codes, scales, tensor_scale, n, k, w_out, ot, ldo, (cudaStream_t)stream));
+}
+
+size_t tq_nvfp4_gemm_batch_workspace_bytes(const tq_nvfp4_gemm_desc *descs, int count, int64_t m) {
+    if (!descs || count < 1 || count > TQ_MAX_BATCH) return 0;
+    tq_gemm_desc plain[TQ_MAX_BATCH];
+    for (int i = 0; i < count; ++i)
+        plain[i] = {descs[i].codes, nullptr, descs[i].n, descs[i].k, descs[i].X, descs[i].ldx, descs[i].Y,
+                    descs[i].ldy};
+    return tq_gemm_batch_workspace_bytes(plain, count, m);
+}
+
+tq_status tq_nvfp4_gemm_batch(const tq_nvfp4_gemm_desc *descs, int count, int64_t m, tq_dtype xt, tq_dtype yt,
+                              void *workspace, size_t ws_bytes, void *stream) {
+    if (!descs) return TQ_ERR_INVALID_ARG;
+    if (count < 1 || count > TQ_MAX_BATCH) return TQ_ERR_SHAPE;
+    if (m < 0) return TQ_ERR_INVALID_ARG;
+    if (m > 32) return TQ_ERR_SHAPE;
+    if (!valid_dtype(xt) || !valid_dtype(yt)) return TQ_ERR_DTYPE;
+    tq_status st;
+    tq_gemm_desc plain[TQ_MAX_BATCH];
+    for (int i = 0; i < count; ++i) {
+        const tq_nvfp4_gemm_desc &d = descs[i];
+        // the scale plane of an NVFP4 matrix is bytes; the shared checks only look at pointers
+        if ((st = check_gemm_common(d.codes, reinterpret_cast<const uint16_t *>(d.scales), d.n, d.k, m, d.Y, yt,
+                                    d.ldy)) != TQ_OK)
+            return st;
+        if (d.n == 0) return TQ_ERR_SHAPE;
+        if (!d.tensor_scale) return TQ_ERR_INVALID_ARG;
+        if (!aligned(d.tensor_scale, 16)) return TQ_ERR_ALIGNMENT;
+        if (m > 0 && (st = check_matrix_operand(d.X, d.ldx, d.k)) != TQ_OK) return st;
+        plain[i] = {d.codes, nullptr, d.n, d.k, d.X, d.ldx, d.Y, d.ldy};
+    }
+    if (m == 0) return TQ_OK;
+    Layout lay;
+    int input_of[tq::kMaxProblems];
+    if ((st = batch_layout(plain, count, m, &lay, input_of)) != TQ_OK) return st;
+    if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
+    char *ws = static_cast<char *>(workspace);
+    tq::RotJob jobs[tq::kMaxInputs];
+    tq::GemvProblem pbs[tq::kMaxProblems];
+    for (int i = 0; i < count; ++i) {
+        const int q = input_of[i];
+        auto *xf = reinterpret_cast<uint16_t *>(ws + lay.xrot_off[q]);
+        jobs[q] = {descs[i].X, descs[i].ldx, descs[i].k, xf};
+        pbs[i] = {descs[i].codes, reinterpret_cast<const uint16_t *>(descs[i].scales), xf, descs[i].Y,
+                  descs[i].ldy, descs[i].n, descs[i].k, descs[i].tensor_scale};
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    // no rotation: the activation is only converted to fp16 in fragment order
+    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws),
+                                         (int64_t)(lay.partial_off / 4), s, false);
+    if (e != cudaSuccess) return TQ_ERR_CUDA;
+    e = tq::launch_group_nvfp4(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
+                               reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true,
+                               s);
+    return from_cuda(e);
+}
+
+tq_status tq_nvfp4_gemm(const uint8_t *codes, const uint8_t *scales, const float *tensor_scale, int64_t n, int64_t k,
+                        const void *X, tq_dtype xt, int64_t m, int64_t ldx, void *Y, tq_dtype yt, int64_t ldy,
+                        void *workspace, size_t ws_bytes, void *stream) {
+    if (m > 32) return TQ_ERR_SHAPE;
+    if (n == 0 && check_nk(n, k) == TQ_OK && m >= 0) return TQ_OK;
+    tq_nvfp4_gemm_desc d = {codes, scales, tensor_scale, n, k, X, ldx, Y, ldy};
+    return tq_nvfp4_gemm_batch(&d, 1, m, xt, yt, workspace, ws_bytes, stream);
+}
+
 tq_status tq_workspace_status(void *workspace, int clear, void *stream) {
     if (!workspace) return TQ_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;

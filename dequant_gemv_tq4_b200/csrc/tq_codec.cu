@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_
 // Handles a list of inputs (one warp per (input, row, superblock)) and zeroes
 // the split-K arrival counters of the product that follows.
 // -------------------------------------------------------------------------
-template <int DT>
+template <int DT, bool ROTATE>
 __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_constant__ RotParams prm) {
     // Launched as a programmatic dependent of the previous kernel in the
     // stream: wait until every earlier kernel has completed (and its memory is
@@ -351,11 +351,15 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (valid) load4<DT>(in.x + ((int64_t)row * in.ldx + col0) * ElemSize<DT>::value, v);
+    if (ROTATE) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = flip(v[i], sign_mask(col0 + i));
-    fwht32_warp(v, p);
-    const __half2 lo = __floats2half2_rn(__fmul_rn(v[0], 0.03125f), __fmul_rn(v[1], 0.03125f));
-    const __half2 hi = __floats2half2_rn(__fmul_rn(v[2], 0.03125f), __fmul_rn(v[3], 0.03125f));
+        for (int i = 0; i < 4; ++i) v[i] = flip(v[i], sign_mask(col0 + i));
+        fwht32_warp(v, p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = __fmul_rn(v[i], 0.03125f);
+    }
+    const __half2 lo = __floats2half2_rn(v[0], v[1]);
+    const __half2 hi = __floats2half2_rn(v[2], v[3]);
     // elements 4p, 4p+1 -> t = 2(p&1), q = 2(p>>1) + {0,1}; 4p+2, 4p+3 -> t + 1
     const size_t blk_words = ((size_t)local * kSbBlocks + j) * 16;  // 32 halves per block
     const int t0 = 2 * (p & 1), q0 = 2 * (p >> 1);
@@ -417,7 +421,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int6
 }
 
 cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *counters,
-                             int64_t counters_count, cudaStream_t stream) {
+                             int64_t counters_count, cudaStream_t stream, bool rotate) {
     if (count < 1 || count > kMaxInputs) return cudaErrorInvalidValue;
     RotParams prm = {};
     int64_t units = 0;
@@ -446,10 +450,13 @@ cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    switch (dtype) {
-        case kF32: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32>, prm);
-        case kBF16: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16>, prm);
-        case kF16: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16>, prm);
+    switch (dtype * 2 + (rotate ? 1 : 0)) {
+        case kF32 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, true>, prm);
+        case kBF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, true>, prm);
+        case kF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, true>, prm);
+        case kF32 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, false>, prm);
+        case kBF16 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, false>, prm);
+        case kF16 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, false>, prm);
         default: return cudaErrorInvalidValue;
     }
 }

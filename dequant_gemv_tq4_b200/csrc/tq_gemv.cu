@@ -53,11 +53,11 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kStages = TQ_GEMV_STAGES;  // ring stages per warp
 constexpr int kPerStage = 2;  // consecutive units per stage
 constexpr int kUnitCodeBytes = 1024;
-constexpr int kUnitScaleBytes = 256;
+constexpr int kUnitScaleBytes = 256;  // TQ4_1S: 16 rows x 4 blocks x 2 fp16; NVFP4 uses 128 (16 x 8 E4M3)
 constexpr int kUnitBytes = kUnitCodeBytes + kUnitScaleBytes;
 // stage = [codes of unit A | codes of unit B | scales of A | scales of B]
 constexpr int kStageScaleOff = kPerStage * kUnitCodeBytes;
-constexpr int kStageBytes = kPerStage * kUnitBytes;    // 2560
+constexpr int kStageBytes = kPerStage * kUnitBytes;    // 2560 (room for either codec)
 constexpr int kRingWarpBytes = kStages * kStageBytes;  // 7680
 // Shared-memory map (addresses in the CTA's shared window; the dynamic
 // allocation starts at a small base B <= kMaxSmemBase):
@@ -89,7 +89,8 @@ uint32_t g_debug_flags = 0;
 struct DevProblem {
     const uint8_t *codes;
     const uint8_t *scales;
-    const uint16_t *xrot;
+    const uint16_t *xrot;  // TQ4_1S: pre-rotated activation; NVFP4: activation in fragment order
+    const float *tscale;   // NVFP4 tensor scale (device), nullptr for TQ4_1S
     char *y;
     int64_t ldy;
     int64_t unit_begin;
@@ -189,20 +190,22 @@ __device__ __forceinline__ int problem_end(const GroupParams &P, int q) {
     return (int)((q + 1 < P.count) ? P.prob[q + 1].unit_begin : P.units);
 }
 
+template <int SB>
 __device__ __forceinline__ Cursor cursor_at(const GroupParams &P, int v) {
     const int q = problem_of(P, v);
     const int local = v - (int)P.prob[q].unit_begin;
     Cursor cu;
     cu.c = P.prob[q].codes + (int64_t)local * kUnitCodeBytes;
-    cu.s = P.prob[q].scales + (int64_t)local * kUnitScaleBytes;
+    cu.s = P.prob[q].scales + (int64_t)local * SB;
     cu.left = problem_end(P, q) - v;
     cu.q = q;
     return cu;
 }
 
+template <int SB>
 __device__ __forceinline__ void cursor_step(const GroupParams &P, Cursor &cu, int units) {
     cu.c += units * kUnitCodeBytes;
-    cu.s += units * kUnitScaleBytes;
+    cu.s += units * SB;
     cu.left -= units;
     if (cu.left == 0 && cu.q + 1 < P.count) {
         ++cu.q;
@@ -215,30 +218,82 @@ __device__ __forceinline__ void cursor_step(const GroupParams &P, Cursor &cu, in
 // Copy the next `cnt` (1 or 2) units of the cursor into a stage.  Units of one
 // problem are contiguous, so a pair is one copy per plane; a pair that
 // straddles two problems takes one copy per unit and plane.
+template <int SB>  // scale bytes per unit
 __device__ __forceinline__ void issue_stage(const GroupParams &P, Cursor &cu, int cnt, uint32_t dst, uint32_t bar,
                                             uint32_t leader) {
-    arrive_expect_tx_pred(leader, bar, (uint32_t)(cnt * kUnitBytes));
+    arrive_expect_tx_pred(leader, bar, (uint32_t)(cnt * (kUnitCodeBytes + SB)));
     if (cu.left >= cnt) {
         bulk_copy_pred(leader, dst, cu.c, (uint32_t)(cnt * kUnitCodeBytes), bar);
-        bulk_copy_pred(leader, dst + kStageScaleOff, cu.s, (uint32_t)(cnt * kUnitScaleBytes), bar);
-        cursor_step(P, cu, cnt);
+        bulk_copy_pred(leader, dst + kStageScaleOff, cu.s, (uint32_t)(cnt * SB), bar);
+        cursor_step<SB>(P, cu, cnt);
     } else {
         for (int h = 0; h < cnt; ++h) {
             bulk_copy_pred(leader, dst + h * kUnitCodeBytes, cu.c, kUnitCodeBytes, bar);
-            bulk_copy_pred(leader, dst + kStageScaleOff + h * kUnitScaleBytes, cu.s, kUnitScaleBytes, bar);
-            cursor_step(P, cu, 1);
+            bulk_copy_pred(leader, dst + kStageScaleOff + h * SB, cu.s, SB, bar);
+            cursor_step<SB>(P, cu, 1);
         }
     }
 }
+
+// ---- codec traits -----------------------------------------------------------
+// TQ4_1S: codes are sign-magnitude ranks into the Lloyd-Max magnitudes, scales
+// are fp16 (d0, d1) per 32-block.  NVFP4: codes are E2M1 values, scales are
+// E4M3 bytes per 16-block, plus a per-tensor fp32 scale applied to y.
+enum Codec : int { kCodecTQ4 = 0, kCodecNVFP4 = 1 };
+
+__constant__ uint16_t c_e2m1_f16[8] = {0x0000u, 0x3800u, 0x3c00u, 0x3e00u, 0x4000u, 0x4200u, 0x4400u, 0x4600u};
+
+template <int CODEC>
+struct CodecTraits;
+
+template <>
+struct CodecTraits<kCodecTQ4> {
+    static constexpr int kScaleBytes = 256;
+    // fp16 value of a 4-bit code
+    __device__ static uint32_t code_f16(int c) { return c_mag_f16[c & 7] | ((c & 8) ? 0x8000u : 0u); }
+    // this lane's scale words for row `row` of the unit (4 blocks x (d0, d1))
+    __device__ static uint4 load(uint32_t ss, int row) { return lds128(ss + row * 16); }
+    // (scale of half 0, scale of half 1) of 32-column block j
+    __device__ static float2 pair(const uint4 &w, int j) {
+        const uint32_t v = j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w;
+        return __half22float2(*reinterpret_cast<const __half2 *>(&v));
+    }
+};
+
+template <>
+struct CodecTraits<kCodecNVFP4> {
+    static constexpr int kScaleBytes = 128;
+    __device__ static uint32_t code_f16(int c) { return c_e2m1_f16[c & 7] | ((c & 8) ? 0x8000u : 0u); }
+    // 8 E4M3 bytes of row `row` (16-element blocks 0..7 of the superblock)
+    __device__ static uint4 load(uint32_t ss, int row) {
+        uint32_t a, b;
+        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(a), "=r"(b) : "r"(ss + row * 8));
+        return make_uint4(a, b, 0u, 0u);
+    }
+    // 32-column block j covers 16-element blocks 2j (half 0) and 2j+1 (half 1)
+    __device__ static float2 pair(const uint4 &w, int j) {
+        const uint32_t word = (j < 2) ? w.x : w.y;
+        const uint16_t two = (uint16_t)(word >> (16 * (j & 1)));
+        uint32_t h;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
+        return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+    }
+};
 
 // Write the accumulators of a finished tile segment: straight to Y when this
 // warp covered the whole tile, else through the fixed-order partial sums.
 template <int NT, bool M1, int OT>
 __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
-                                           int u1, int gw, const float (&acc)[NT][4]) {
+                                           int u1, int gw, const float (&acc_in)[NT][4]) {
     constexpr int kMcap = 8 * NT;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const DevProblem &pr = P.prob[q];
+    float acc[NT][4];
+    const float ts = pr.tscale ? __ldg(pr.tscale) : 1.0f;  // NVFP4 tensor scale
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = acc_in[a][b] * ts;
     const int U = (int)P.units, W = P.total_warps;
     const int64_t gt = pr.tile_begin + r;
     const int row_g = r * 16 + g, row_g8 = row_g + 8;
@@ -298,8 +353,10 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
     if (lane == 0) P.counters[gt] = 0u;
 }
 
-template <int NT, bool M1, int OT>
+template <int NT, bool M1, int OT, int CODEC>
 __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
+    using CT = CodecTraits<CODEC>;
+    constexpr int SB = CT::kScaleBytes;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gw = blockIdx.x * kWarps + warp;
@@ -328,11 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
             fence_mbar_init();
         }
         __syncwarp();
-        cu = cursor_at(P, u0);
+        cu = cursor_at<SB>(P, u0);
         for (int i = 0; i < kStages && pv < u1; ++i) {
             const int cnt = min(kPerStage, u1 - pv);
             const bool skip = P.inject_skip && gw == 0 && i == 1;
-            issue_stage(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0 && !skip);
+            issue_stage<SB>(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0 && !skip);
             pv += cnt;
         }
     }
@@ -342,9 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         uint4 *lut = reinterpret_cast<uint4 *>(smem + (kLutAddr - base));
         for (int idx = threadIdx.x; idx < 256 * 8; idx += kThreads) {  // entry v: 8 x 16 bytes
             const int v = idx >> 3;
-            const uint32_t lo = c_mag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
-            const uint32_t hi = c_mag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
-            const uint32_t e = lo | (hi << 16);
+            const uint32_t e = CT::code_f16(v & 15) | (CT::code_f16(v >> 4) << 16);
             lut[v * 16 + (idx & 7)] = make_uint4(e, e, e, e);
         }
     }
@@ -358,8 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     const int g = lane >> 2, t = lane & 3;
     // PRMT operand: byte 0 = lane*4, bytes 2..3 = table base >> 16
     const uint32_t lut_lane = kLutAddr | ((uint32_t)lane * 4u);
-    // this lane's 16 code bytes of rows g and g+8, and its scale words, in a unit
-    const uint32_t off_c = g * 64 + t * 16, off_s = g * 16;
+    // this lane's 16 code bytes of rows g and g+8 in a unit
+    const uint32_t off_c = g * 64 + t * 16;
 
     // ---- segment state: the tile the current unit belongs to ---------------
     int q = problem_of(P, u0);
@@ -417,15 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
             }
         }
         {
-            const uint32_t sc = st + h * kUnitCodeBytes, ss = st + kStageScaleOff + h * kUnitScaleBytes;
+            const uint32_t sc = st + h * kUnitCodeBytes, ss = st + kStageScaleOff + h * SB;
             const uint4 c0 = lds128(sc + off_c);
             const uint4 c1 = lds128(sc + off_c + 512);
-            const uint4 s0 = lds128(ss + off_s);
-            const uint4 s1 = lds128(ss + off_s + 128);
+            const uint4 s0 = CT::load(ss, g);
+            const uint4 s1 = CT::load(ss, g + 8);
             const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
             const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
-            const uint32_t sw0[4] = {s0.x, s0.y, s0.z, s0.w};
-            const uint32_t sw1[4] = {s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
             for (int j = 0; j < kSbBlocks; ++j) {
                 uint4 xb[NT];
@@ -440,8 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                 const uint32_t a11 = lds_u32(prmt(cw1[j], lut_lane, 0x7624u));
                 const uint32_t a12 = lds_u32(prmt(cw0[j], lut_lane, 0x7634u));
                 const uint32_t a13 = lds_u32(prmt(cw1[j], lut_lane, 0x7634u));
-                const float2 dg = __half22float2(*reinterpret_cast<const __half2 *>(&sw0[j]));
-                const float2 dg8 = __half22float2(*reinterpret_cast<const __half2 *>(&sw1[j]));
+                const float2 dg = CT::pair(s0, j);
+                const float2 dg8 = CT::pair(s1, j);
 #pragma unroll
                 for (int a = 0; a < NT; ++a) {
                     float d[4];
@@ -495,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
             __syncwarp();
             if (pv < u1) {
                 const int cnt = min(kPerStage, u1 - pv);
-                issue_stage(P, cu, cnt, st, bar, lane == 0);
+                issue_stage<SB>(P, cu, cnt, st, bar, lane == 0);
                 pv += cnt;
             }
             stage = (stage == kStages - 1) ? 0 : stage + 1;
@@ -521,7 +574,7 @@ uint32_t dynamic_smem_base() {
     return cached[dev];
 }
 
-template <int NT, bool M1>
+template <int NT, bool M1, int CODEC>
 cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programmatic, cudaStream_t stream) {
     const uint32_t smem = smem_bytes_for_base(dynamic_smem_base());
     const int kSmemBytes = (int)smem;
@@ -538,20 +591,20 @@ cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programm
     cudaError_t err;
     switch (dtype) {
         case kF32:
-            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kF32, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
             if (err != cudaSuccess) return err;
-            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kF32>, prm);
+            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kF32, CODEC>, prm);
         case kBF16:
-            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kBF16, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
             if (err != cudaSuccess) return err;
-            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kBF16>, prm);
+            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kBF16, CODEC>, prm);
         case kF16:
-            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kF16, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
             if (err != cudaSuccess) return err;
-            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kF16>, prm);
+            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kF16, CODEC>, prm);
         default:
             return cudaErrorInvalidValue;
     }
@@ -580,9 +633,10 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
     return pl;
 }
 
-cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
-                         unsigned *counters, float *partials, unsigned *status, bool programmatic,
-                         cudaStream_t stream) {
+template <int CODEC>
+cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
+                               unsigned *counters, float *partials, unsigned *status, bool programmatic,
+                               cudaStream_t stream) {
     if (count < 1 || count > kMaxProblems) return cudaErrorInvalidValue;
     GroupParams prm = {};
     int64_t ub = 0, tb = 0;
@@ -591,6 +645,7 @@ cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydt
         d.codes = probs[i].codes;
         d.scales = reinterpret_cast<const uint8_t *>(probs[i].scales);
         d.xrot = probs[i].xrot;
+        d.tscale = probs[i].tensor_scale;
         d.y = static_cast<char *>(probs[i].y);
         d.ldy = probs[i].ldy;
         d.unit_begin = ub;
@@ -612,14 +667,28 @@ cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydt
     prm.timeout_ns = prm.inject_skip ? kDebugTimeoutNs : kTimeoutNs;
     // the partial-slot stride is 16 * 8 * NT floats: NT must match plan.mcap
     const int nt = plan.mcap / 8;
-    if (m == 1 && nt == 1) return launch_nt<1, true>(prm, ydtype, plan.grid, programmatic, stream);
+    if (m == 1 && nt == 1) return launch_nt<1, true, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
     switch (nt) {
-        case 1: return launch_nt<1, false>(prm, ydtype, plan.grid, programmatic, stream);
-        case 2: return launch_nt<2, false>(prm, ydtype, plan.grid, programmatic, stream);
-        case 3: return launch_nt<3, false>(prm, ydtype, plan.grid, programmatic, stream);
-        case 4: return launch_nt<4, false>(prm, ydtype, plan.grid, programmatic, stream);
+        case 1: return launch_nt<1, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+        case 2: return launch_nt<2, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+        case 3: return launch_nt<3, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+        case 4: return launch_nt<4, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
+                         unsigned *counters, float *partials, unsigned *status, bool programmatic,
+                         cudaStream_t stream) {
+    return launch_group_codec<kCodecTQ4>(probs, count, m, ydtype, plan, counters, partials, status, programmatic,
+                                         stream);
+}
+
+cudaError_t launch_group_nvfp4(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
+                               unsigned *counters, float *partials, unsigned *status, bool programmatic,
+                               cudaStream_t stream) {
+    return launch_group_codec<kCodecNVFP4>(probs, count, m, ydtype, plan, counters, partials, status, programmatic,
+                                           stream);
 }
 
 }  // namespace tq

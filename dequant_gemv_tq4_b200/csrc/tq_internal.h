@@ -54,9 +54,10 @@ struct RotJob {  // host-side request
     uint16_t *xrot;
 };
 
-// xrot for m rows of every job (same dtype); also zeroes `counters`.
+// xrot for m rows of every job (same dtype); also zeroes `counters`.  With
+// rotate = false the activation is only converted to fp16 fragment order.
 cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *counters,
-                             int64_t counters_count, cudaStream_t stream);
+                             int64_t counters_count, cudaStream_t stream, bool rotate = true);
 
 // ---- fused product ---------------------------------------------------------
 struct GemvProblem {  // host-side request, m <= 32 rows of pre-rotated activations
@@ -67,6 +68,7 @@ struct GemvProblem {  // host-side request, m <= 32 rows of pre-rotated activati
     int64_t ldy;
     int64_t n;
     int64_t k;
+    const float *tensor_scale = nullptr;  // NVFP4 only (device pointer)
 };
 
 struct GroupPlan {
@@ -88,5 +90,21 @@ void set_debug_flags(uint32_t flags);
 cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
                          unsigned *counters, float *partials, unsigned *status, bool programmatic,
                          cudaStream_t stream);
+
+// ---- NVFP4 comparison codec ---------------------------------------------------
+// Same fused product over NVFP4 planes (E2M1 codes in the TQ4_1S unit layout,
+// E4M3 block scales, a device fp32 tensor scale per problem); xrot holds the
+// activation in fragment order without rotation (launch_prerotate, rotate=false).
+cudaError_t launch_group_nvfp4(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
+                               unsigned *counters, float *partials, unsigned *status, bool programmatic,
+                               cudaStream_t stream);
+
+cudaError_t launch_nvfp4_amax(const void *w, int dtype, int64_t n, int64_t k, int64_t ldw, unsigned *amax_bits,
+                              cudaStream_t stream);
+cudaError_t launch_nvfp4_quantize(const void *w, int dtype, int64_t n, int64_t k, int64_t ldw,
+                                  const unsigned *amax_bits, uint8_t *codes, uint8_t *scales, float *tensor_scale,
+                                  cudaStream_t stream);
+cudaError_t launch_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *tensor_scale,
+                                    int64_t n, int64_t k, void *w_out, int dtype, int64_t ldo, cudaStream_t stream);
 
 }  // namespace tq

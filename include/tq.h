@@ -252,6 +252,83 @@ TQ_API void tq_debug_set_flags(uint32_t flags);
 TQ_API tq_status tq_gemv_static_scratch(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
                                         const void *x, tq_dtype xt, void *y, tq_dtype yt, void *stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * NVFP4 comparison codec
+ * ---------------------------------------------------------------------------
+ * NVFP4 is named, without a bit recipe, by the llm-compressor page
+ * (ai-insight.org/news/11771: NVFP4 checkpoints) and the llama.cpp quantizer
+ * page (bittide.aicompass.dev: "NVFP4 weight and input tensor scales").  This
+ * library implements the plainest reading of the format, for comparison with
+ * TQ4_1S on the same shapes:
+ *   g   = amax|W| / (6 * 448)                       fp32, one per tensor
+ *   s_b = E4M3(amax_b / (6 * g))                    one per 16 elements
+ *   q   = E2M1(w / (value(s_b) * g))                4 bits per element, 0 when
+ *                                                   the scale is 0
+ *   w~  = value(q) * value(s_b) * g
+ * Each quotient and product is one IEEE fp32 operation; both conversions
+ * round to nearest-even and saturate (E4M3 at 448, E2M1 at 6); a zero code
+ * carries no sign.  No rotation.  4.5 bits per weight.
+ *
+ * Layout: the codes plane is the TQ4_1S one (tq_codes_bytes; the two
+ * 16-element blocks of a 32-column pair take the place of one 32-element
+ * block, byte order unchanged: element 2L in the low nibble of logical byte
+ * L).  E2M1 code: bit 3 = sign, bits 0-2 = magnitude index into
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6}.  The scales plane is E4M3 bytes
+ * [T][NSB][16 rows][8 blocks of 16] (tq_nvfp4_scales_bytes).  The tensor
+ * block is TQ_NVFP4_TENSOR_BYTES of device memory: float g at offset 0, the
+ * fp32 amax|W| at offset 4, the rest reserved.
+ */
+#define TQ_NVFP4_TENSOR_BYTES 16
+
+/* ceil(n/16) * ceil(k/128) * 128 bytes; 0 for invalid sizes. */
+TQ_API size_t tq_nvfp4_scales_bytes(int64_t n, int64_t k);
+
+/*
+ * tq_nvfp4_quantize -- encode W (n x k, dtype wt, row stride ldw; the operand
+ * rules of tq_quantize) into codes (tq_codes_bytes), scales
+ * (tq_nvfp4_scales_bytes) and the tensor block (TQ_NVFP4_TENSOR_BYTES); all
+ * device, 16-byte aligned, written.  Three operations on `stream`: a memset of
+ * the amax word, a reduction of amax|W|, the encode.  NaN/Inf inputs are
+ * outside the contract.
+ */
+TQ_API tq_status tq_nvfp4_quantize(const void *w, tq_dtype wt, int64_t n, int64_t k, int64_t ldw, uint8_t *codes,
+                                   uint8_t *scales, float *tensor_scale, void *stream);
+
+/* tq_nvfp4_dequantize -- w~ in fp32, rounded to ot; the operand rules of
+ * tq_dequantize plus the tensor block written by tq_nvfp4_quantize. */
+TQ_API tq_status tq_nvfp4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *tensor_scale,
+                                     int64_t n, int64_t k, void *w_out, tq_dtype ot, int64_t ldo, void *stream);
+
+/*
+ * tq_nvfp4_gemm -- Y[i][r] = sum_k w~[r][k] X[i][k] for i < m <= 32 with the
+ * fused kernel of tq_gemm: codes enter the tensor cores as fp16 E2M1 values,
+ * the activation as fp16 (converted once per call, no rotation), each
+ * 16-column partial sum is scaled by its E4M3 block scale in fp32 and the
+ * row total by g.  Workspace: tq_gemm_workspace_bytes(m, n, k), same rules.
+ * m > 32 returns TQ_ERR_SHAPE.
+ */
+TQ_API tq_status tq_nvfp4_gemm(const uint8_t *codes, const uint8_t *scales, const float *tensor_scale, int64_t n,
+                               int64_t k, const void *X, tq_dtype xt, int64_t m, int64_t ldx, void *Y, tq_dtype yt,
+                               int64_t ldy, void *workspace, size_t ws_bytes, void *stream);
+
+/* Several NVFP4 products in one launch pair, as tq_gemm_batch. */
+typedef struct {
+    const uint8_t *codes;
+    const uint8_t *scales;
+    const float *tensor_scale; /* device tensor block of this matrix */
+    int64_t n;
+    int64_t k;
+    const void *X;
+    int64_t ldx;
+    void *Y;
+    int64_t ldy;
+} tq_nvfp4_gemm_desc;
+
+TQ_API size_t tq_nvfp4_gemm_batch_workspace_bytes(const tq_nvfp4_gemm_desc *descs, int count, int64_t m);
+TQ_API tq_status tq_nvfp4_gemm_batch(const tq_nvfp4_gemm_desc *descs, int count, int64_t m, tq_dtype xt, tq_dtype yt,
+                                     void *workspace, size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
