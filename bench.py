@@ -66,6 +66,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", choices=("llama3_8b_layer", "single_matrix", "ffn_70b"), default="llama3_8b_layer")
     p.add_argument("--skip-cpu-baseline", action="store_true")
     p.add_argument("--skip-e2e", action="store_true")
+    p.add_argument("--skip-codec-comparison", action="store_true",
+                   help="skip the NVFP4 vs TQ4_1S comparison on the Llama-3-8B layer shapes")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     p.add_argument("--cpu-sample-rows", type=int, default=None,
                    help="rows per matrix for the CPU oracle sample (default: 1/8 of each matrix)")
@@ -493,6 +495,9 @@ def run_ours(args, world, rank, local):
 
     if not args.skip_e2e:
         line["e2e"] = run_e2e(tq, path, steps=min(steps, 5), world=world)
+    if args.workload == "llama3_8b_layer" and not args.skip_codec_comparison:
+        line["codec_comparison"] = codec_comparison(tq, path, rank, device, min(steps, 10), warmup, flush, use_graph,
+                                                    world)
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         cb = cpu_oracle_sample(path, args.cpu_sample_rows)
         line["cpu_baseline"] = {"value": round(cb["gemv_gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -501,6 +506,114 @@ def run_ours(args, world, rank, local):
                                 "seconds": round(cb["seconds"], 1)}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, world):
+    """NVFP4 next to TQ4_1S on the same layer: reconstruction rel-L2 over the
+    layer, quantise Gweights/s and fused-product GB/s at M = 1 and M = 16
+    (steady state, passes alternating with a shadow layer as for the main
+    metric).  GB/s counts each codec's own packed bytes."""
+    from dequant_gemv_tq4_b200 import inputs
+
+    R = 10
+    smats, _, _ = make_workload("llama3_8b_layer", rank + 1000, device)
+    x16 = {}
+    for aid, act in enumerate(("attn", "attn_out", "ffn", "ffn_mid")):
+        k = 14336 if act == "ffn_mid" else 4096
+        x16[act] = inputs.gaussian_matrix(1, 300 + aid, 16, k, 1.0, torch.bfloat16, device)
+    act_of = inputs.LLAMA3_8B_INPUTS
+
+    def nv_pack(mats):
+        return [tq.nvfp4_quantize(W) for _, W, _ in mats]
+
+    layer_mats = [(it["label"], it["W"], None) for it in path.items]
+    nv_layer, nv_shadow = nv_pack(layer_mats), nv_pack(smats)
+    tq_shadow = [(c, s) for c, s, *_ in path.shadow]
+    tq_layer = [(it["codes"], it["scales"]) for it in path.items]
+
+    def items_tq(packs, mats, m):
+        out = []
+        for (c, s), (label, W, _) in zip(packs, mats):
+            n, k = W.shape
+            X = x16[act_of[label]][:m]
+            out.append((c, s, n, k, X, torch.empty((m, n), dtype=torch.float32, device=device)))
+        return out
+
+    def items_nv(packs, mats, m):
+        out = []
+        for (c, s, t), (label, W, _) in zip(packs, mats):
+            n, k = W.shape
+            X = x16[act_of[label]][:m]
+            out.append((c, s, t, n, k, X, torch.empty((m, n), dtype=torch.float32, device=device)))
+        return out
+
+    def timed(fn, passes):
+        run = capture(fn, use_graph, passes)
+        for _ in range(warmup):
+            run()
+        torch.cuda.synchronize()
+        return time_replays(run, steps, flush) / (steps * passes)
+
+    result = {}
+    for codec in ("tq4_1s", "nvfp4"):
+        entry = {}
+        if codec == "tq4_1s":
+            packed = path.packed_bytes()
+            entry["bits_per_weight"] = 5.0
+        else:
+            packed = sum(c.numel() + s.numel() + t.numel() * 4 for c, s, t in nv_layer)
+            entry["bits_per_weight"] = 4.5
+        for m in (1, 16):
+            if codec == "tq4_1s":
+                a, b = items_tq(tq_layer, layer_mats, m), items_tq(tq_shadow, smats, m)
+                da, db = tq.batch_descs(a), tq.batch_descs(b)
+                wa, wb = tq.batch_workspace(a, m, device), tq.batch_workspace(b, m, device)
+
+                def pair(a=a, b=b, da=da, db=db, wa=wa, wb=wb, m=m):
+                    tq.gemm_batch(a, m=m, ws=wa, descs=da)
+                    tq.gemm_batch(b, m=m, ws=wb, descs=db)
+            else:
+                a, b = items_nv(nv_layer, layer_mats, m), items_nv(nv_shadow, smats, m)
+                da, db = tq.nvfp4_batch_descs(a), tq.nvfp4_batch_descs(b)
+                wa, wb = tq.nvfp4_batch_workspace(a, m, device), tq.nvfp4_batch_workspace(b, m, device)
+
+                def pair(a=a, b=b, da=da, db=db, wa=wa, wb=wb, m=m):
+                    tq.nvfp4_gemm_batch(a, m=m, ws=wa, descs=da)
+                    tq.nvfp4_gemm_batch(b, m=m, ws=wb, descs=db)
+            ms = timed(pair, R // 2) / 2
+            (ms,) = max_over_ranks([ms], world)
+            entry[f"gemm_m{m}_us"] = round(1e3 * ms, 2)
+            entry[f"gemm_m{m}_gbs"] = round(job_gbs(packed, world, ms), 1)
+        if codec == "tq4_1s":
+            qfn = path.quantize
+        else:
+            def qfn():
+                for (c, s, t), it in zip(nv_layer, path.items):
+                    n, k = it["W"].shape
+                    st = tq.tq_nvfp4_quantize(it["W"].data_ptr(), tq.TQ_BF16, n, k, k, c.data_ptr(), s.data_ptr(),
+                                              t.data_ptr(), torch.cuda.current_stream().cuda_stream)
+                    if st != 0:
+                        raise tq.TQError(st, "tq_nvfp4_quantize")
+        ms_q = timed(qfn, R)
+        (ms_q,) = max_over_ranks([ms_q], world)
+        entry["quantize_gweights_per_s"] = round(job_gbs(path.weights(), world, ms_q), 2)
+        # reconstruction error over the layer: ||W~ - W|| / ||W||
+        num = den = 0.0
+        for i, it in enumerate(path.items):
+            n, k = it["W"].shape
+            if codec == "tq4_1s":
+                Wd = tq.dequantize(it["codes"], it["scales"], n, k, dtype=torch.float32)
+            else:
+                c, s, t = nv_layer[i]
+                Wd = tq.nvfp4_dequantize(c, s, t, n, k, dtype=torch.float32)
+            Wf = it["W"].float()
+            num += float(((Wd - Wf).double() ** 2).sum())
+            den += float((Wf.double() ** 2).sum())
+            del Wd, Wf
+        entry["rel_l2_reconstruction"] = round((num / den) ** 0.5, 5)
+        entry["packed_bytes"] = packed
+        result[codec] = entry
+    return result
 
 
 def run_e2e(tq, path, steps, world):
