@@ -17,10 +17,10 @@
 //    The units of all matrices in the group form one index space, split evenly
 //    over every warp of a one-CTA-per-SM grid (stream-K style), so each warp
 //    streams one contiguous stretch of memory.
-//  * Each warp keeps a ring of kStages units in shared memory filled by
-//    cp.async.bulk (TMA bulk copies, one lane issues, an mbarrier per stage
-//    counts the bytes).  No registers are spent on loads in flight; waits are
-//    bounded in time and report a timeout through a status word.
+//  * Each warp keeps a ring of two stages of two units each in shared memory,
+//    filled by cp.async.bulk (TMA bulk copies, one lane issues, an mbarrier
+//    per stage counts the bytes).  No registers are spent on loads in flight;
+//    waits are bounded in time and report a timeout through a status word.
 //  * The per-weight work is a 4-bit -> fp16 lookup.  A byte holds two codes, so
 //    a 256-entry table of half2 pairs turns one byte into a ready tensor-core
 //    operand.  The table lives in shared memory replicated per lane (entry v,
@@ -32,6 +32,13 @@
 //    NT n-tiles for m <= 8*NT).  One k16 step is exactly one half-block, so the
 //    fp16 half-block scale multiplies the fp32 mma result before it joins the
 //    accumulator.
+//  * One activation row (the decode case) would leave seven of the eight mma
+//    columns idle.  Instead column c carries half-block c of the superblock
+//    (four blocks x two halves): the B fragment is the activation in the four
+//    lanes of column c and zero elsewhere, so the eight mmas of a unit chain
+//    into one accumulator whose columns stay separate half-block sums.  Each
+//    lane then applies two scales per row pair per unit (not sixteen), and the
+//    four lanes of a row add their blocks once per tile.
 //  * Tiles split across warps combine fixed-order partial sums: each
 //    contributor writes its slot, the last to arrive (atomic counter, no
 //    waiting) adds the slots in warp order.  Deterministic for a given GPU.
@@ -42,15 +49,11 @@ namespace tq {
 
 namespace {
 
-#ifndef TQ_GEMV_WARPS
-#define TQ_GEMV_WARPS 16
-#endif
-#ifndef TQ_GEMV_STAGES
-#define TQ_GEMV_STAGES 3
-#endif
-constexpr int kWarps = TQ_GEMV_WARPS;
-constexpr int kThreads = kWarps * 32;
-constexpr int kStages = TQ_GEMV_STAGES;  // ring stages per warp
+// Warps per CTA: one-row products keep few registers live and take 20 warps;
+// the multi-row kernels (more accumulators) take 16 so that they fit 128
+// registers per thread without spilling.
+__host__ __device__ constexpr int warps_for(bool one_row) { return one_row ? 20 : 16; }
+constexpr int kStages = 2;  // ring stages per warp
 constexpr int kPerStage = 2;  // consecutive units per stage
 constexpr int kUnitCodeBytes = 1024;
 constexpr int kUnitScaleBytes = 256;  // TQ4_1S: 16 rows x 4 blocks x 2 fp16; NVFP4 uses 128 (16 x 8 E4M3)
@@ -58,21 +61,29 @@ constexpr int kUnitBytes = kUnitCodeBytes + kUnitScaleBytes;
 // stage = [codes of unit A | codes of unit B | scales of A | scales of B]
 constexpr int kStageScaleOff = kPerStage * kUnitCodeBytes;
 constexpr int kStageBytes = kPerStage * kUnitBytes;    // 2560 (room for either codec)
-constexpr int kRingWarpBytes = kStages * kStageBytes;  // 7680
+constexpr int kRingWarpBytes = kStages * kStageBytes;  // 5120
 // Shared-memory map (addresses in the CTA's shared window; the dynamic
 // allocation starts at a small base B <= kMaxSmemBase):
-//   [B, B + kWarps/2 rings)     rings of the first half of the warps
+//   [B, B + W/2 rings)          rings of the first half of the W warps
 //   [0x10000, 0x20000)          lookup table, 64 KB aligned so that one PRMT
 //                               yields the full address of an entry
-//   [0x20000, + kWarps/2 rings) rings of the second half
+//   [0x20000, + W/2 rings)      rings of the second half
 //   then the mbarriers
-constexpr int kLowWarps = kWarps / 2;
 constexpr uint32_t kLutAddr = 0x10000;
-constexpr uint32_t kMaxSmemBase = 0x10000 - kLowWarps * kRingWarpBytes;
 constexpr uint32_t kHighRings = 0x20000;
-constexpr uint32_t kBarAddr = kHighRings + (kWarps - kLowWarps) * kRingWarpBytes;
-constexpr uint32_t kBarBytes = kWarps * kStages * 8;
-static_assert(kMaxSmemBase >= 1024 && kMaxSmemBase < 0x10000, "ring placement below the table");
+template <int W>
+struct Geometry {
+    static constexpr int kWarps = W;
+    static constexpr int kThreads = W * 32;
+    static constexpr int kLowWarps = W / 2;
+    static constexpr uint32_t kMaxSmemBase = 0x10000 - kLowWarps * kRingWarpBytes;
+    static constexpr uint32_t kBarAddr = kHighRings + (W - kLowWarps) * kRingWarpBytes;
+    static constexpr uint32_t kBarBytes = W * kStages * 8;
+    static_assert(kMaxSmemBase >= 1024 && kMaxSmemBase < 0x10000, "ring placement below the table");
+    static_assert(kBarAddr + kBarBytes - 1024 <= 227 * 1024, "dynamic shared memory per CTA");
+    // dynamic shared memory to request for a dynamic base of `base` bytes
+    static uint32_t smem_bytes_for_base(uint32_t base) { return kBarAddr + kBarBytes - base; }
+};
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusLayout = 2u;
 constexpr uint64_t kTimeoutNs = 1000000000ull;     // 1 s
@@ -80,7 +91,6 @@ constexpr uint64_t kDebugTimeoutNs = 5000000ull;   // 5 ms under fault injection
 
 
 // Dynamic shared memory to request for a dynamic base of `base` bytes.
-inline uint32_t smem_bytes_for_base(uint32_t base) { return kBarAddr + kBarBytes - base; }
 
 __constant__ uint16_t c_mag_f16[8] = TQ_MAG_F16_INIT;
 
@@ -113,6 +123,37 @@ struct GroupParams {
 };
 
 // ---- PTX helpers ------------------------------------------------------------
+// LUT read: the table is written once before the CTA barrier and never again,
+// so its loads may be scheduled freely (no volatile)
+__device__ __forceinline__ uint32_t lds_lut(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void mma_nv(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+__device__ __forceinline__ void mma_acc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 ldg64(const void *p) {
+    uint2 r;
+    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
@@ -176,7 +217,8 @@ __device__ __forceinline__ void bulk_copy_pred(uint32_t pred, uint32_t dst, cons
 struct Cursor {
     const uint8_t *c;
     const uint8_t *s;
-    int left;  // units left in the current problem
+    int left;           // units left in the current problem
+    int sb_left;        // units left in the current tile
     int q;
 };
 
@@ -194,35 +236,42 @@ template <int SB>
 __device__ __forceinline__ Cursor cursor_at(const GroupParams &P, int v) {
     const int q = problem_of(P, v);
     const int local = v - (int)P.prob[q].unit_begin;
+    const int nsb = P.prob[q].nsb;
     Cursor cu;
     cu.c = P.prob[q].codes + (int64_t)local * kUnitCodeBytes;
     cu.s = P.prob[q].scales + (int64_t)local * SB;
     cu.left = problem_end(P, q) - v;
+    cu.sb_left = nsb - local % nsb;
     cu.q = q;
     return cu;
 }
 
+// Advance by `units` (at most cu.sb_left: never past the end of a tile).
 template <int SB>
 __device__ __forceinline__ void cursor_step(const GroupParams &P, Cursor &cu, int units) {
     cu.c += units * kUnitCodeBytes;
     cu.s += units * SB;
     cu.left -= units;
-    if (cu.left == 0 && cu.q + 1 < P.count) {
-        ++cu.q;
-        cu.c = P.prob[cu.q].codes;
-        cu.s = P.prob[cu.q].scales;
-        cu.left = problem_end(P, cu.q) - (int)P.prob[cu.q].unit_begin;
+    cu.sb_left -= units;
+    if (cu.sb_left == 0) {  // next tile
+        if (cu.left == 0 && cu.q + 1 < P.count) {  // of the next problem
+            ++cu.q;
+            cu.c = P.prob[cu.q].codes;
+            cu.s = P.prob[cu.q].scales;
+            cu.left = problem_end(P, cu.q) - (int)P.prob[cu.q].unit_begin;
+        }
+        cu.sb_left = P.prob[cu.q].nsb;
     }
 }
 
 // Copy the next `cnt` (1 or 2) units of the cursor into a stage.  Units of one
-// problem are contiguous, so a pair is one copy per plane; a pair that
-// straddles two problems takes one copy per unit and plane.
+// tile are contiguous in both planes, so a pair is one copy per plane; a pair
+// that straddles two tiles takes one copy per unit and plane.
 template <int SB>  // scale bytes per unit
 __device__ __forceinline__ void issue_stage(const GroupParams &P, Cursor &cu, int cnt, uint32_t dst, uint32_t bar,
                                             uint32_t leader) {
     arrive_expect_tx_pred(leader, bar, (uint32_t)(cnt * (kUnitCodeBytes + SB)));
-    if (cu.left >= cnt) {
+    if (cu.sb_left >= cnt) {
         bulk_copy_pred(leader, dst, cu.c, (uint32_t)(cnt * kUnitCodeBytes), bar);
         bulk_copy_pred(leader, dst + kStageScaleOff, cu.s, (uint32_t)(cnt * SB), bar);
         cursor_step<SB>(P, cu, cnt);
@@ -258,6 +307,11 @@ struct CodecTraits<kCodecTQ4> {
         const uint32_t v = j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w;
         return __half22float2(*reinterpret_cast<const __half2 *>(&v));
     }
+    // (d0, d1) of block j of row `row`
+    __device__ static float2 block(uint32_t ss, int row, int j) {
+        const uint32_t v = lds32(ss + row * 16 + j * 4);
+        return __half22float2(*reinterpret_cast<const __half2 *>(&v));
+    }
 };
 
 template <>
@@ -274,6 +328,14 @@ struct CodecTraits<kCodecNVFP4> {
     __device__ static float2 pair(const uint4 &w, int j) {
         const uint32_t word = (j < 2) ? w.x : w.y;
         const uint16_t two = (uint16_t)(word >> (16 * (j & 1)));
+        uint32_t h;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
+        return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+    }
+    // block scales of the two halves of 32-column block j of row `row`
+    __device__ static float2 block(uint32_t ss, int row, int j) {
+        uint16_t two;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(two) : "r"(ss + row * 8 + j * 2));
         uint32_t h;
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
         return __half22float2(*reinterpret_cast<const __half2 *>(&h));
@@ -353,21 +415,169 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
     if (lane == 0) P.counters[gt] = 0u;
 }
 
+// Products of one unit (16 rows x 128 columns) accumulated into acc: the
+// unit's codes at shared address sc, its scales at ss, the activation
+// fragments at xcur[a] + xoff.
+template <int NT, bool M1, typename CT>
+__device__ __forceinline__ void unit_product(uint32_t sc, uint32_t ss, const uint16_t *const (&xcur)[NT], int xoff,
+                                             uint32_t lut_lane, uint32_t off_c, int g, float (&acc)[NT][4]) {
+    const uint4 c0 = lds128(sc + off_c);
+    const uint4 c1 = lds128(sc + off_c + 512);
+    const uint4 s0 = CT::load(ss, g);
+    const uint4 s1 = CT::load(ss, g + 8);
+    const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
+    const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int j = 0; j < kSbBlocks; ++j) {
+        uint4 xb[NT];
+#pragma unroll
+        for (int a = 0; a < NT; ++a) xb[a] = ldg_keep(xcur[a] + xoff + j * 32);
+        // code byte b of word cw: logical byte t + 4b of the block
+        const uint32_t a00 = lds_lut(prmt(cw0[j], lut_lane, 0x7604u));
+        const uint32_t a01 = lds_lut(prmt(cw1[j], lut_lane, 0x7604u));
+        const uint32_t a02 = lds_lut(prmt(cw0[j], lut_lane, 0x7614u));
+        const uint32_t a03 = lds_lut(prmt(cw1[j], lut_lane, 0x7614u));
+        const uint32_t a10 = lds_lut(prmt(cw0[j], lut_lane, 0x7624u));
+        const uint32_t a11 = lds_lut(prmt(cw1[j], lut_lane, 0x7624u));
+        const uint32_t a12 = lds_lut(prmt(cw0[j], lut_lane, 0x7634u));
+        const uint32_t a13 = lds_lut(prmt(cw1[j], lut_lane, 0x7634u));
+        const float2 dg = CT::pair(s0, j);
+        const float2 dg8 = CT::pair(s1, j);
+#pragma unroll
+        for (int a = 0; a < NT; ++a) {
+            float d[4];
+            mma_nv(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
+            acc[a][0] = fmaf(d[0], dg.x, acc[a][0]);
+            acc[a][2] = fmaf(d[2], dg8.x, acc[a][2]);
+            if (!M1) {
+                acc[a][1] = fmaf(d[1], dg.x, acc[a][1]);
+                acc[a][3] = fmaf(d[3], dg8.x, acc[a][3]);
+            }
+            mma_nv(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
+            acc[a][0] = fmaf(d[0], dg.y, acc[a][0]);
+            acc[a][2] = fmaf(d[2], dg8.y, acc[a][2]);
+            if (!M1) {
+                acc[a][1] = fmaf(d[1], dg.y, acc[a][1]);
+                acc[a][3] = fmaf(d[3], dg8.y, acc[a][3]);
+            }
+        }
+    }
+}
+
+// One activation row: the eight columns of B carry the eight half-blocks
+// (c = 2j + h) of the unit, column c non-zero only in the products of
+// half-block c (its four lanes g == c hold the activation, the others zero),
+// so one accumulator chain keeps the eight partial sums apart.  Lane (g, t)
+// ends with the half-block sums of block t for rows g and g + 8 and scales
+// them with that block's two scales; the lanes' block sums are added when the
+// tile segment is flushed.  xv: this lane's four activation values of
+// half-block g (from the stage).
+template <typename CT>
+__device__ __forceinline__ void unit_product_m1(uint32_t sc, uint32_t ss, uint2 xv, uint32_t lut_lane,
+                                                uint32_t off_c, int g, int t, float (&acc)[1][4]) {
+    const uint4 c0 = lds128(sc + off_c);
+    const uint4 c1 = lds128(sc + off_c + 512);
+    const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
+    const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+    float d[4];
+#pragma unroll
+    for (int j = 0; j < kSbBlocks; ++j) {
+        // code byte b of word cw: logical byte t + 4b of the block
+        const uint32_t a00 = lds_lut(prmt(cw0[j], lut_lane, 0x7604u));
+        const uint32_t a01 = lds_lut(prmt(cw1[j], lut_lane, 0x7604u));
+        const uint32_t a02 = lds_lut(prmt(cw0[j], lut_lane, 0x7614u));
+        const uint32_t a03 = lds_lut(prmt(cw1[j], lut_lane, 0x7614u));
+        const uint32_t a10 = lds_lut(prmt(cw0[j], lut_lane, 0x7624u));
+        const uint32_t a11 = lds_lut(prmt(cw1[j], lut_lane, 0x7624u));
+        const uint32_t a12 = lds_lut(prmt(cw0[j], lut_lane, 0x7634u));
+        const uint32_t a13 = lds_lut(prmt(cw1[j], lut_lane, 0x7634u));
+        const bool p0 = g == 2 * j, p1 = g == 2 * j + 1;
+        if (j == 0)
+            mma_nv(d, a00, a01, a02, a03, p0 ? xv.x : 0u, p0 ? xv.y : 0u);
+        else
+            mma_acc(d, a00, a01, a02, a03, p0 ? xv.x : 0u, p0 ? xv.y : 0u);
+        mma_acc(d, a10, a11, a12, a13, p1 ? xv.x : 0u, p1 ? xv.y : 0u);
+    }
+    const float2 sg = CT::block(ss, g, t), sg8 = CT::block(ss, g + 8, t);
+    acc[0][0] = fmaf(d[0], sg.x, acc[0][0]);
+    acc[0][1] = fmaf(d[1], sg.y, acc[0][1]);
+    acc[0][2] = fmaf(d[2], sg8.x, acc[0][2]);
+    acc[0][3] = fmaf(d[3], sg8.y, acc[0][3]);
+}
+
+// One unit's products; the activation fragments of its superblock start at
+// xcur[a] + xoff.
+template <int NT, bool M1, typename CT>
+__device__ __forceinline__ void unit_any(uint32_t sc, uint32_t ss, const uint16_t *const (&xcur)[NT], int xoff,
+                                         uint32_t lut_lane, uint32_t off_c, uint32_t off_x, int g, int t,
+                                         float (&acc)[NT][4]) {
+    if constexpr (M1) {
+        static_assert(NT == 1, "one activation row uses one n-tile");
+        // this lane's four activation values of half-block g
+        const uint2 xv = ldg64(reinterpret_cast<const char *>(xcur[0] + xoff) + off_x);
+        unit_product_m1<CT>(sc, ss, xv, lut_lane, off_c, g, t, acc);
+    } else {
+        unit_product<NT, M1, CT>(sc, ss, xcur, xoff, lut_lane, off_c, g, acc);
+    }
+}
+
+// The tile segment ending at unit u is complete: write it out, reset the
+// accumulators and move the segment state to the tile of unit u.
 template <int NT, bool M1, int OT, int CODEC>
-__global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
+__device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0, int u1, int gw, int g, int t, int &q,
+                                         int &prob_end, int &nsb, int &r, int &tile_lo, int &seg_end,
+                                         const uint16_t *(&xcur)[NT], float (&acc)[NT][4]) {
+    if constexpr (M1) {
+        // rows g, g + 8: add the two halves, then the four blocks (lanes t)
+        float vg = acc[0][0] + acc[0][1], vg8 = acc[0][2] + acc[0][3];
+        vg += __shfl_xor_sync(kFull, vg, 1);
+        vg8 += __shfl_xor_sync(kFull, vg8, 1);
+        vg += __shfl_xor_sync(kFull, vg, 2);
+        vg8 += __shfl_xor_sync(kFull, vg8, 2);
+        acc[0][0] = vg;
+        acc[0][2] = vg8;
+    }
+    flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, acc);
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    if (u < u1) {
+        if (u == prob_end) {  // next problem: new tiles, new activation
+            ++q;
+            prob_end = problem_end(P, q);
+            nsb = P.prob[q].nsb;
+            r = 0;
+            tile_lo = u;
+        } else {
+            ++r;
+            tile_lo += nsb;
+        }
+        seg_end = min(tile_lo + nsb, u1);
+#pragma unroll
+        for (int a = 0; a < NT; ++a) {  // back to superblock 0 of the activation
+            const int xrow = min(8 * a + g, P.m - 1);
+            xcur[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
+        }
+    }
+}
+
+template <int NT, bool M1, int OT, int CODEC>
+__global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
+    using G = Geometry<warps_for(M1)>;
     using CT = CodecTraits<CODEC>;
     constexpr int SB = CT::kScaleBytes;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gw = blockIdx.x * kWarps + warp;
+    const int gw = blockIdx.x * G::kWarps + warp;
     const uint32_t base = (uint32_t)__cvta_generic_to_shared(smem);
-    if (base > kMaxSmemBase) {  // layout precondition (checked, never expected)
+    if (base > G::kMaxSmemBase) {  // layout precondition (checked, never expected)
         if (threadIdx.x == 0) atomicOr(P.status, kStatusLayout);
         return;
     }
     const uint32_t ring =
-        warp < kLowWarps ? base + warp * kRingWarpBytes : kHighRings + (warp - kLowWarps) * kRingWarpBytes;
-    const uint32_t bars = kBarAddr + warp * (kStages * 8);
+        warp < G::kLowWarps ? base + warp * kRingWarpBytes : kHighRings + (warp - G::kLowWarps) * kRingWarpBytes;
+    const uint32_t bars = G::kBarAddr + warp * (kStages * 8);
     const bool active = gw < P.total_warps;
     const int U = (int)P.units;
     const int W = P.total_warps;
@@ -377,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     // ---- prologue: barriers, first bulk copies, lookup table -------------
     // (the packed weights never depend on the preceding grid, so the copies
     // start before the programmatic-dependency wait)
-    Cursor cu = {nullptr, nullptr, 0, 0};
+    Cursor cu = {nullptr, nullptr, 0, 0, 0};
     int pv = u0;  // next unit to copy
     if (active) {
         if (lane == 0) {
@@ -388,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         cu = cursor_at<SB>(P, u0);
         for (int i = 0; i < kStages && pv < u1; ++i) {
             const int cnt = min(kPerStage, u1 - pv);
-            const bool skip = P.inject_skip && gw == 0 && i == 1;
+            const bool skip = P.inject_skip && gw == 0 && i == 0;
             issue_stage<SB>(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0 && !skip);
             pv += cnt;
         }
@@ -397,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
         // entry v holds the same half2 in all 32 lane slots (the first 128 of
         // its 256 bytes)
         uint4 *lut = reinterpret_cast<uint4 *>(smem + (kLutAddr - base));
-        for (int idx = threadIdx.x; idx < 256 * 8; idx += kThreads) {  // entry v: 8 x 16 bytes
+        for (int idx = threadIdx.x; idx < 256 * 8; idx += G::kThreads) {  // entry v: 8 x 16 bytes
             const int v = idx >> 3;
             const uint32_t e = CT::code_f16(v & 15) | (CT::code_f16(v >> 4) << 16);
             lut[v * 16 + (idx & 7)] = make_uint4(e, e, e, e);
@@ -415,6 +625,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
     const uint32_t lut_lane = kLutAddr | ((uint32_t)lane * 4u);
     // this lane's 16 code bytes of rows g and g+8 in a unit
     const uint32_t off_c = g * 64 + t * 16;
+    // one activation row: byte offset of this lane's 8 bytes of half-block g
+    // (block g/2, half g%2) in a superblock's fragments [4 blocks][4 t][8
+    // halves], relative to xcur (which already holds t)
+    const uint32_t off_x = (g >> 1) * 64 + (g & 1) * 8;
 
     // ---- segment state: the tile the current unit belongs to ---------------
     int q = problem_of(P, u0);
@@ -446,12 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
 
     int stage = 0;
     uint32_t parity = 0;
-    uint32_t st = ring, bar = bars;
-    for (int u = u0; u < u1; ++u) {
-        const int h = (u - u0) & 1;  // position of the unit in its stage
-        if (h == 0) {                // warp-uniform: a new stage
-            st = ring + stage * kStageBytes;
-            bar = bars + 8 * stage;
+    int u = u0;
+    while (u < u1) {
+        const uint32_t st = ring + stage * kStageBytes, bar = bars + 8 * stage;
+        {
             bool ok = mbar_try(bar, parity);
             if (!__all_sync(kFull, ok)) {
                 ok = ok || mbar_wait_slow(bar, parity, P.timeout_ns);
@@ -471,89 +683,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_group_kernel(const __grid_co
                 }
             }
         }
-        {
-            const uint32_t sc = st + h * kUnitCodeBytes, ss = st + kStageScaleOff + h * SB;
-            const uint4 c0 = lds128(sc + off_c);
-            const uint4 c1 = lds128(sc + off_c + 512);
-            const uint4 s0 = CT::load(ss, g);
-            const uint4 s1 = CT::load(ss, g + 8);
-            const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
-            const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+        const int cnt = min(kPerStage, u1 - u);  // units held by this stage
+        if (M1 && cnt == kPerStage && u + kPerStage <= seg_end) {
+            // common one-row case: both units belong to the current tile
+            // segment (the multi-row kernels take the loop below, which keeps
+            // one unit's operands live at a time)
+            unit_any<NT, M1, CT>(st, st + kStageScaleOff, xcur, 0, lut_lane, off_c, off_x, g, t, acc);
+            unit_any<NT, M1, CT>(st + kUnitCodeBytes, st + kStageScaleOff + SB, xcur, 128, lut_lane, off_c, off_x, g,
+                                 t, acc);
 #pragma unroll
-            for (int j = 0; j < kSbBlocks; ++j) {
-                uint4 xb[NT];
+            for (int a = 0; a < NT; ++a) xcur[a] += 256;
+            u += 2;
+            if (u == seg_end)
+                end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
+        } else {
+            for (int h = 0; h < cnt; ++h) {
+                unit_any<NT, M1, CT>(st + h * kUnitCodeBytes, st + kStageScaleOff + h * SB, xcur, 0, lut_lane, off_c,
+                                     off_x, g, t, acc);
 #pragma unroll
-                for (int a = 0; a < NT; ++a) xb[a] = ldg_keep(xcur[a] + j * 32);
-                // code byte b of word cw: logical byte t + 4b of the block
-                const uint32_t a00 = lds_u32(prmt(cw0[j], lut_lane, 0x7604u));
-                const uint32_t a01 = lds_u32(prmt(cw1[j], lut_lane, 0x7604u));
-                const uint32_t a02 = lds_u32(prmt(cw0[j], lut_lane, 0x7614u));
-                const uint32_t a03 = lds_u32(prmt(cw1[j], lut_lane, 0x7614u));
-                const uint32_t a10 = lds_u32(prmt(cw0[j], lut_lane, 0x7624u));
-                const uint32_t a11 = lds_u32(prmt(cw1[j], lut_lane, 0x7624u));
-                const uint32_t a12 = lds_u32(prmt(cw0[j], lut_lane, 0x7634u));
-                const uint32_t a13 = lds_u32(prmt(cw1[j], lut_lane, 0x7634u));
-                const float2 dg = CT::pair(s0, j);
-                const float2 dg8 = CT::pair(s1, j);
-#pragma unroll
-                for (int a = 0; a < NT; ++a) {
-                    float d[4];
-                    mma_16816_zero(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
-                    acc[a][0] = fmaf(d[0], dg.x, acc[a][0]);
-                    acc[a][2] = fmaf(d[2], dg8.x, acc[a][2]);
-                    if (!M1) {
-                        acc[a][1] = fmaf(d[1], dg.x, acc[a][1]);
-                        acc[a][3] = fmaf(d[3], dg8.x, acc[a][3]);
-                    }
-                    mma_16816_zero(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
-                    acc[a][0] = fmaf(d[0], dg.y, acc[a][0]);
-                    acc[a][2] = fmaf(d[2], dg8.y, acc[a][2]);
-                    if (!M1) {
-                        acc[a][1] = fmaf(d[1], dg.y, acc[a][1]);
-                        acc[a][3] = fmaf(d[3], dg8.y, acc[a][3]);
-                    }
-                }
+                for (int a = 0; a < NT; ++a) xcur[a] += 128;
+                ++u;
+                if (u == seg_end)
+                    end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
             }
         }
-        ++sb;
-#pragma unroll
-        for (int a = 0; a < NT; ++a) xcur[a] += 128;
-        if (u + 1 == seg_end) {  // warp-uniform: the tile segment is complete
-            flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, acc);
-#pragma unroll
-            for (int a = 0; a < NT; ++a)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-            if (u + 1 < u1) {
-                if (u + 1 == prob_end) {  // next problem: new tiles, new activation
-                    ++q;
-                    prob_end = problem_end(P, q);
-                    nsb = P.prob[q].nsb;
-                    r = 0;
-                    tile_lo = u + 1;
-                } else {
-                    ++r;
-                    tile_lo += nsb;
-                }
-                sb = 0;
-                seg_end = min(tile_lo + nsb, u1);
-#pragma unroll
-                for (int a = 0; a < NT; ++a) {  // back to superblock 0 of the activation
-                    const int xrow = min(8 * a + g, P.m - 1);
-                    xcur[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
-                }
-            }
+        __syncwarp();  // every lane has read the stage: it may be refilled
+        if (pv < u1) {
+            const int c2 = min(kPerStage, u1 - pv);
+            issue_stage<SB>(P, cu, c2, st, bar, lane == 0);
+            pv += c2;
         }
-        if (h == kPerStage - 1 || u + 1 == u1) {  // warp-uniform: the stage is consumed
-            __syncwarp();
-            if (pv < u1) {
-                const int cnt = min(kPerStage, u1 - pv);
-                issue_stage<SB>(P, cu, cnt, st, bar, lane == 0);
-                pv += cnt;
-            }
-            stage = (stage == kStages - 1) ? 0 : stage + 1;
-            parity ^= (stage == 0) ? 1u : 0u;
-        }
+        stage = (stage == kStages - 1) ? 0 : stage + 1;
+        parity ^= (stage == 0) ? 1u : 0u;
     }
 }
 
@@ -576,11 +737,12 @@ uint32_t dynamic_smem_base() {
 
 template <int NT, bool M1, int CODEC>
 cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programmatic, cudaStream_t stream) {
-    const uint32_t smem = smem_bytes_for_base(dynamic_smem_base());
+    using G = Geometry<warps_for(M1)>;
+    const uint32_t smem = G::smem_bytes_for_base(dynamic_smem_base());
     const int kSmemBytes = (int)smem;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(G::kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -620,6 +782,8 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
         pl.tiles += tiles(n[i]);
         pl.units += tiles(n[i]) * superblocks(k[i]);
     }
+    // one activation row runs the one-row kernel (see launch_group_codec)
+    const int kWarps = warps_for(m == 1);
     int64_t want = (pl.units + kWarps - 1) / kWarps;  // at least one unit per warp
     if (want > sm_count) want = sm_count;
     if (want < 1) want = 1;
@@ -667,7 +831,10 @@ cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, i
     prm.timeout_ns = prm.inject_skip ? kDebugTimeoutNs : kTimeoutNs;
     // the partial-slot stride is 16 * 8 * NT floats: NT must match plan.mcap
     const int nt = plan.mcap / 8;
-    if (m == 1 && nt == 1) return launch_nt<1, true, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+    const bool one_row = m == 1 && nt == 1;
+    // the plan's warps must all exist in the launched grid
+    if (plan.total_warps > (int64_t)plan.grid * warps_for(one_row)) return cudaErrorInvalidValue;
+    if (one_row) return launch_nt<1, true, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
     switch (nt) {
         case 1: return launch_nt<1, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
         case 2: return launch_nt<2, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
