@@ -120,7 +120,22 @@ struct GroupParams {
     unsigned *status;
     uint64_t timeout_ns;
     int inject_skip;
+    double inv_units;  // 1.0 / units and 1.0 / total_warps (host-computed):
+    double inv_warps;  // the split arithmetic divides without 64-bit integer division
 };
+
+// floor(n / d) for 0 <= n < 2^52, 0 < d < 2^31, given inv_d = 1.0 / d.  The
+// double estimate is within one of the quotient (n is exact in a double and
+// the product's relative error is ~2^-52), and one integer step corrects it.
+// A 64-bit integer division is a long instruction sequence; this is a few.
+__device__ __forceinline__ int64_t div_floor(int64_t n, int64_t d, double inv_d) {
+    int64_t q = __double2ll_rz((double)n * inv_d);
+    if ((q + 1) * d <= n)
+        ++q;
+    else if (q * d > n)
+        --q;
+    return q;
+}
 
 // ---- PTX helpers ------------------------------------------------------------
 // LUT read: the table is written once before the CTA barrier and never again,
@@ -223,8 +238,11 @@ struct Cursor {
 };
 
 __device__ __forceinline__ int problem_of(const GroupParams &P, int v) {
+    // the largest q with unit_begin <= v (independent loads, not a dependent walk)
     int q = 0;
-    while (q + 1 < P.count && v >= P.prob[q + 1].unit_begin) ++q;
+#pragma unroll
+    for (int i = 1; i < kMaxProblems; ++i)
+        if (i < P.count && v >= P.prob[i].unit_begin) q = i;
     return q;
 }
 
@@ -383,16 +401,13 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
         }
     __syncwarp();
     // owner of unit x: the largest w with floor(w*U/W) <= x
-    const int first = (int)(((int64_t)(tile_lo + 1) * W - 1) / U);
-    const int last = (int)(((int64_t)tile_hi * W - 1) / U);
+    const int first = (int)div_floor((int64_t)(tile_lo + 1) * W - 1, U, P.inv_units);
+    const int last = (int)div_floor((int64_t)tile_hi * W - 1, U, P.inv_units);
     unsigned arrived = 0;
-    if (lane == 0) {
-        __threadfence();  // release: the warp's slot writes (ordered by the warp barrier)
-        arrived = atomicAdd(P.counters + gt, 1u);
-    }
+    if (lane == 0)  // release the warp's slot writes (ordered by the warp barrier); acquire the others'
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(P.counters + gt) : "memory");
     arrived = __shfl_sync(kFull, arrived, 0);
     if (arrived != (unsigned)(last - first)) return;
-    if (lane == 0) __threadfence();  // acquire: the other contributors' slots
     __syncwarp();
     const int cnt = last - first + 1;
     for (int e = lane; e < 16 * P.m; e += 32) {
@@ -581,8 +596,8 @@ __global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const
     const bool active = gw < P.total_warps;
     const int U = (int)P.units;
     const int W = P.total_warps;
-    const int u0 = active ? (int)((int64_t)gw * U / W) : 0;
-    const int u1 = active ? (int)((int64_t)(gw + 1) * U / W) : 0;
+    const int u0 = active ? (int)div_floor((int64_t)gw * U, W, P.inv_warps) : 0;
+    const int u1 = active ? (int)div_floor((int64_t)(gw + 1) * U, W, P.inv_warps) : 0;
 
     // ---- prologue: barriers, first bulk copies, lookup table -------------
     // (the packed weights never depend on the preceding grid, so the copies
@@ -828,6 +843,8 @@ cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, i
     prm.counters = counters;
     prm.status = status;
     prm.inject_skip = (g_debug_flags & 1u) ? 1 : 0;
+    prm.inv_units = 1.0 / (double)prm.units;
+    prm.inv_warps = 1.0 / (double)prm.total_warps;
     prm.timeout_ns = prm.inject_skip ? kDebugTimeoutNs : kTimeoutNs;
     // the partial-slot stride is 16 * 8 * NT floats: NT must match plan.mcap
     const int nt = plan.mcap / 8;
