@@ -55,12 +55,12 @@ tq_status check_planes(const uint8_t *codes, const uint16_t *scales) {
 tq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 
 // Workspace of a fused-product call:
-//   [0, 256)           status word (timeout flag of the last call)
-//   [256, ...)         split-K arrival counters, one per 16-row tile
-//   partial slots      (tiles + warps) * 16 * mcap floats
+//   [0, 256)           header: status word (timeout flag of the last call),
+//                      call tag (advanced by every call)
+//   partial slots      (tiles + warps) * 16 * mcap tagged sums (8 bytes each)
 //   pre-rotated inputs one area per distinct activation (calls that rotate)
 struct Layout {
-    size_t counter_off, partial_off, xrot_off[tq::kMaxInputs], total;
+    size_t partial_off, xrot_off[tq::kMaxInputs], total;
     int inputs;
     tq::GroupPlan plan;
 };
@@ -74,8 +74,7 @@ tq_status make_layout(const int64_t *n, const int64_t *k, int count, const int64
     const int64_t ms = m > 32 ? 32 : (m < 1 ? 1 : m);
     lay->plan = tq::plan_group(n, k, count, ms, di.sm_count);
     if (lay->plan.units >= ((int64_t)1 << 31)) return TQ_ERR_SHAPE;  // > 2^42 weights per call
-    lay->counter_off = kStatusBytes;
-    lay->partial_off = lay->counter_off + lay->plan.counter_bytes;
+    lay->partial_off = kStatusBytes;
     size_t off = lay->partial_off + lay->plan.partial_bytes;
     lay->inputs = inputs;
     for (int i = 0; i < inputs; ++i) {
@@ -152,7 +151,7 @@ tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t
     if (!xrot) return TQ_ERR_INVALID_ARG;
     if (!aligned(xrot, 16)) return TQ_ERR_ALIGNMENT;
     tq::RotJob job = {X, ldx, k, xrot};
-    return from_cuda(tq::launch_prerotate(&job, 1, xt, m, nullptr, 0, (cudaStream_t)stream));
+    return from_cuda(tq::launch_prerotate(&job, 1, xt, m, nullptr, (cudaStream_t)stream));
 }
 
 size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
@@ -195,13 +194,12 @@ tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, 
     if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
     char *ws = static_cast<char *>(workspace);
     cudaStream_t s = (cudaStream_t)stream;
-    // status word and arrival counters must start at zero; the workspace may
-    // have held anything (another call's partial sums or activations)
-    if (cudaMemsetAsync(ws, 0, lay.partial_off, s) != cudaSuccess) return TQ_ERR_CUDA;
+    // clear the status word and advance the call tag (the pre-rotation does
+    // this in the calls that rotate)
+    if (tq::launch_prepare_header(reinterpret_cast<unsigned *>(ws), s) != cudaSuccess) return TQ_ERR_CUDA;
     tq::GemvProblem pb = {codes, scales, xrot, Y, ldy, n, k};
-    return from_cuda(tq::launch_group(&pb, 1, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
-                                      reinterpret_cast<float *>(ws + lay.partial_off),
-                                      reinterpret_cast<unsigned *>(ws), true, s));
+    return from_cuda(tq::launch_group(&pb, 1, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
+                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s));
 }
 
 tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X, tq_dtype xt,
@@ -221,13 +219,12 @@ tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64
     for (int64_t i0 = 0; i0 < m; i0 += 32) {
         const int64_t ms = (m - i0) < 32 ? (m - i0) : 32;
         tq::RotJob job = {static_cast<const char *>(X) + (size_t)i0 * (size_t)ldx * xsize, ldx, k, xrot};
-        // zeroes the status word and the counters that follow it
-        cudaError_t e = tq::launch_prerotate(&job, 1, xt, ms, reinterpret_cast<unsigned *>(ws),
-                                             (int64_t)(lay.partial_off / 4), s);
+        // also clears the status word and advances the call tag
+        cudaError_t e = tq::launch_prerotate(&job, 1, xt, ms, reinterpret_cast<unsigned *>(ws), s);
         if (e != cudaSuccess) return TQ_ERR_CUDA;
         tq::GemvProblem pb = {codes, scales, xrot, static_cast<char *>(Y) + (size_t)i0 * (size_t)ldy * ysize, ldy, n, k};
-        e = tq::launch_group(&pb, 1, ms, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
-                             reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true, s);
+        e = tq::launch_group(&pb, 1, ms, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
+                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
         if (e != cudaSuccess) return TQ_ERR_CUDA;
     }
     return TQ_OK;
@@ -299,11 +296,10 @@ tq_status tq_gemm_batch(const tq_gemm_desc *descs, int count, int64_t m, tq_dtyp
         pbs[i] = {descs[i].codes, descs[i].scales, xrot, descs[i].Y, descs[i].ldy, descs[i].n, descs[i].k};
     }
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws),
-                                         (int64_t)(lay.partial_off / 4), s);
+    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws), s);
     if (e != cudaSuccess) return TQ_ERR_CUDA;
-    e = tq::launch_group(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
-                         reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true, s);
+    e = tq::launch_group(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
+                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
     return from_cuda(e);
 }
 
@@ -394,11 +390,10 @@ tq_status tq_nvfp4_gemm_batch(const tq_nvfp4_gemm_desc *descs, int count, int64_
     }
     cudaStream_t s = (cudaStream_t)stream;
     // no rotation: the activation is only converted to fp16 in fragment order
-    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws),
-                                         (int64_t)(lay.partial_off / 4), s, false);
+    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws), s, false);
     if (e != cudaSuccess) return TQ_ERR_CUDA;
-    e = tq::launch_group_nvfp4(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
-                               reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true,
+    e = tq::launch_group_nvfp4(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
+                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true,
                                s);
     return from_cuda(e);
 }
@@ -435,7 +430,7 @@ void tq_debug_set_flags(uint32_t flags) { tq::set_debug_flags(flags); }
 // custom allocator or a memory-pool callback (where allocating would recurse),
 // plugins handed only the tensors of one operation by a host framework, or
 // processes whose device memory is entirely reserved up front.  For them the
-// scratch of the fused GEMV (status word, split-K counters, partial sums,
+// scratch of the fused GEMV (header: status word and call tag, partial sums,
 // pre-rotated activation) lives in this fixed device array instead, sized
 // TQ_STATIC_SCRATCH_BYTES, resident on every GPU that loads the library until
 // the process exits.
@@ -483,13 +478,12 @@ extern "C" tq_status tq_gemv_static_scratch(const uint8_t *codes, const uint16_t
     auto *xrot = reinterpret_cast<uint16_t *>(ws + lay.xrot_off[0]);
     cudaStream_t s = (cudaStream_t)stream;
     tq::RotJob job = {x, k, k, xrot};
-    // the pre-rotation launch also zeroes the status word and the counters:
-    // the array keeps whatever the previous call left in it
-    cudaError_t e = tq::launch_prerotate(&job, 1, xt, 1, reinterpret_cast<unsigned *>(ws),
-                                         (int64_t)(lay.partial_off / 4), s);
+    // the pre-rotation launch also clears the status word and advances the
+    // call tag: the array keeps whatever the previous call left in it
+    cudaError_t e = tq::launch_prerotate(&job, 1, xt, 1, reinterpret_cast<unsigned *>(ws), s);
     if (e != cudaSuccess) return TQ_ERR_CUDA;
     tq::GemvProblem pb = {codes, scales, xrot, y, n, n, k};
-    e = tq::launch_group(&pb, 1, 1, yt, lay.plan, reinterpret_cast<unsigned *>(ws + lay.counter_off),
-                         reinterpret_cast<float *>(ws + lay.partial_off), reinterpret_cast<unsigned *>(ws), true, s);
+    e = tq::launch_group(&pb, 1, 1, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
+                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
     return from_cuda(e);
 }

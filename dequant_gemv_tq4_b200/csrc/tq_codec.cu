@@ -324,8 +324,9 @@ __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_
 // -------------------------------------------------------------------------
 // Pre-rotation of activations into the fused kernel's fragment order:
 // element e of a block goes to slot t*8 + q with t = (e%8)/2, q = 2*(e/8) + e%2.
-// Handles a list of inputs (one warp per (input, row, superblock)) and zeroes
-// the split-K arrival counters of the product that follows.
+// Handles a list of inputs (one warp per (input, row, superblock)) and
+// prepares the header of the product that follows (status cleared, tag
+// advanced).
 // -------------------------------------------------------------------------
 template <int DT, bool ROTATE>
 __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_constant__ RotParams prm) {
@@ -335,8 +336,10 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     // which reads packed weights that earlier kernels may have written.
     grid_dependency_wait();
     grid_dependents_launch();
-    const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (int64_t i = gtid; i < prm.counters_count; i += (int64_t)gridDim.x * blockDim.x) prm.counters[i] = 0u;
+    if (prm.header && blockIdx.x == 0 && threadIdx.x == 0) {
+        prm.header[kHeaderStatus] = 0u;
+        prm.header[kHeaderTag] += 1u;  // the previous call (and its product) has completed
+    }
 
     const int lane = threadIdx.x & 31;
     const int j = lane >> 3, p = lane & 7;
@@ -420,8 +423,34 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int6
     return cudaGetLastError();
 }
 
-cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *counters,
-                             int64_t counters_count, cudaStream_t stream, bool rotate) {
+namespace {
+
+__global__ void __launch_bounds__(32) prepare_header_kernel(unsigned *header) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    if (threadIdx.x == 0) {
+        header[kHeaderStatus] = 0u;
+        header[kHeaderTag] += 1u;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prepare_header(unsigned *header, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(32);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prepare_header_kernel, header);
+}
+
+cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *header,
+                             cudaStream_t stream, bool rotate) {
     if (count < 1 || count > kMaxInputs) return cudaErrorInvalidValue;
     RotParams prm = {};
     int64_t units = 0;
@@ -437,8 +466,7 @@ cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m
     }
     prm.count = count;
     prm.units = units;
-    prm.counters = counters;
-    prm.counters_count = counters ? counters_count : 0;
+    prm.header = header;
     int64_t grid = (units + kCodecWarps - 1) / kCodecWarps;
     if (grid < 1) grid = 1;
     cudaLaunchConfig_t cfg = {};

@@ -39,9 +39,11 @@
 //    into one accumulator whose columns stay separate half-block sums.  Each
 //    lane then applies two scales per row pair per unit (not sixteen), and the
 //    four lanes of a row add their blocks once per tile.
-//  * Tiles split across warps combine fixed-order partial sums: each
-//    contributor writes its slot, the last to arrive (atomic counter, no
-//    waiting) adds the slots in warp order.  Deterministic for a given GPU.
+//  * Tiles split across warps combine fixed-order partial sums: the later
+//    contributors store (value, call tag) words without fences or atomics,
+//    and the tile's first warp, which reaches its part of the tile last, adds
+//    them in warp order once each carries this call's tag (a bounded poll).
+//    Deterministic for a given GPU.
 #include "tq_device.cuh"
 #include "tq_internal.h"
 
@@ -115,9 +117,8 @@ struct GroupParams {
     int m;
     int64_t units;    // < 2^31 (checked on the host)
     int total_warps;  // <= units: warp w owns [w*units/W, (w+1)*units/W)
-    float *partials;
-    unsigned *counters;
-    unsigned *status;
+    uint64_t *partials;  // tagged partial sums (value bits | call tag << 32)
+    unsigned *header;    // workspace header: status word, call tag
     uint64_t timeout_ns;
     int inject_skip;
     double inv_units;  // 1.0 / units and 1.0 / total_warps (host-computed):
@@ -360,11 +361,84 @@ struct CodecTraits<kCodecNVFP4> {
     }
 };
 
+// Relaxed 64-bit global store / load (single-copy atomic: a value and its
+// call tag are seen together or not at all).
+__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+template <int NT>
+struct AccTile {
+    float v[NT][4];
+};
+
+// The first contributor of a split tile: its own sums plus those of warps
+// gw+1 .. last, the owner of the tile's last unit (the largest w with
+// floor(w*U/W) <= x), added in warp order once each word carries the tag.
+template <int NT, bool M1, int OT>
+__device__ __noinline__ void reduce_first(const GroupParams &P, int q, int r, int tile_hi, int gw, uint32_t tag,
+                                          AccTile<NT> acc) {
+    constexpr int kMcap = 8 * NT;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const DevProblem &pr = P.prob[q];
+    const int64_t gt = pr.tile_begin + r;
+    const int U = (int)P.units, W = P.total_warps;
+    const int last = (int)div_floor((int64_t)tile_hi * W - 1, U, P.inv_units);
+    const uint64_t *base = P.partials + (gt + gw + 1) * (int64_t)(16 * kMcap);
+    uint64_t t0 = 0;
+    bool timed_out = false;
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (M1 && (b & 1)) continue;
+            const int xrow = 8 * a + 2 * t + (b & 1);
+            const int wl = g + ((b & 2) ? 8 : 0);
+            if (xrow >= P.m) continue;
+            const uint64_t *src = base + xrow * 16 + wl;
+            float sum = acc.v[a][b];
+            for (int w0 = gw + 1; w0 <= last; w0 += 8) {
+                const int cnt = min(8, last - w0 + 1);
+                uint64_t v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)  // up to eight loads in flight
+                    if (i < cnt) v[i] = ld_relaxed_u64(src + (int64_t)(w0 - gw - 1 + i) * (16 * kMcap));
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (i >= cnt) break;
+                    for (uint32_t it = 0; (uint32_t)(v[i] >> 32) != tag && !timed_out; ++it) {
+                        if (t0 == 0) t0 = global_ns();
+                        if ((it & 63u) == 63u && (global_ns() - t0 > P.timeout_ns || it >= (1u << 30)))
+                            timed_out = true;
+                        v[i] = ld_relaxed_u64(src + (int64_t)(w0 - gw - 1 + i) * (16 * kMcap));
+                    }
+                    sum += __uint_as_float((uint32_t)v[i]);
+                }
+            }
+            const int wrow = r * 16 + wl;
+            if (!timed_out && wrow < pr.n) store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
+        }
+    if (timed_out) atomicOr(P.header + kHeaderStatus, kStatusTimeout);
+}
+
 // Write the accumulators of a finished tile segment: straight to Y when this
-// warp covered the whole tile, else through the fixed-order partial sums.
+// warp covered the whole tile, else through the tagged partial sums.
+//
+// A tile split over warps gw0 < ... < gwk: the tile starts in gw0's range and
+// is that warp's last segment, reached at the end of its work; for every
+// later contributor it is the first segment, reached at the start.  So the
+// later contributors store their sums, each as one 64-bit word (fp32 value,
+// call tag), with no fence and no atomic, and gw0 adds them (own part first,
+// then warp order: deterministic), polling until each word carries this
+// call's tag.  The wait is bounded in time and reports a timeout.
 template <int NT, bool M1, int OT>
 __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
-                                           int u1, int gw, const float (&acc_in)[NT][4]) {
+                                           int u1, int gw, uint32_t tag, const float (&acc_in)[NT][4]) {
     constexpr int kMcap = 8 * NT;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const DevProblem &pr = P.prob[q];
@@ -374,7 +448,6 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
     for (int a = 0; a < NT; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) acc[a][b] = acc_in[a][b] * ts;
-    const int U = (int)P.units, W = P.total_warps;
     const int64_t gt = pr.tile_begin + r;
     const int row_g = r * 16 + g, row_g8 = row_g + 8;
     if (u0 <= tile_lo && tile_hi <= u1) {
@@ -390,44 +463,26 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
             }
         return;
     }
-    float *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
+    const uint64_t tag_hi = (uint64_t)tag << 32;
+    if (tile_lo < u0) {  // a later contributor: store the tagged sums and go on
+        uint64_t *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int xrow = 8 * a + 2 * t + (b & 1);
+                const int wrow = g + ((b & 2) ? 8 : 0);
+                if (xrow < P.m) st_relaxed_u64(slot + xrow * 16 + wrow, tag_hi | __float_as_uint(acc[a][b]));
+            }
+        return;
+    }
+    // the first contributor (kept out of line: rare, and register hungry)
+    AccTile<NT> own;
 #pragma unroll
     for (int a = 0; a < NT; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int xrow = 8 * a + 2 * t + (b & 1);
-            const int wrow = g + ((b & 2) ? 8 : 0);
-            slot[xrow * 16 + wrow] = acc[a][b];
-        }
-    __syncwarp();
-    // owner of unit x: the largest w with floor(w*U/W) <= x
-    const int first = (int)div_floor((int64_t)(tile_lo + 1) * W - 1, U, P.inv_units);
-    const int last = (int)div_floor((int64_t)tile_hi * W - 1, U, P.inv_units);
-    unsigned arrived = 0;
-    if (lane == 0)  // release the warp's slot writes (ordered by the warp barrier); acquire the others'
-        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(P.counters + gt) : "memory");
-    arrived = __shfl_sync(kFull, arrived, 0);
-    if (arrived != (unsigned)(last - first)) return;
-    __syncwarp();
-    const int cnt = last - first + 1;
-    for (int e = lane; e < 16 * P.m; e += 32) {
-        const int xrow = e >> 4, wl = e & 15;
-        const float *src = P.partials + (gt + first) * (int64_t)(16 * kMcap) + xrow * 16 + wl;
-        // eight independent loads in flight, added in slot order
-        float sum = 0.f;
-        int c = 0;
-        for (; c + 8 <= cnt; c += 8) {
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + (int64_t)(c + i) * (16 * kMcap));
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sum += v[i];
-        }
-        for (; c < cnt; ++c) sum += __ldcg(src + (int64_t)c * (16 * kMcap));
-        const int wrow = r * 16 + wl;
-        if (wrow < pr.n) store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
-    }
-    if (lane == 0) P.counters[gt] = 0u;
+        for (int b = 0; b < 4; ++b) own.v[a][b] = acc[a][b];
+    reduce_first<NT, M1, OT>(P, q, r, tile_hi, gw, tag, own);
 }
 
 // Products of one unit (16 rows x 128 columns) accumulated into acc: the
@@ -539,7 +594,8 @@ __device__ __forceinline__ void unit_any(uint32_t sc, uint32_t ss, const uint16_
 // The tile segment ending at unit u is complete: write it out, reset the
 // accumulators and move the segment state to the tile of unit u.
 template <int NT, bool M1, int OT, int CODEC>
-__device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0, int u1, int gw, int g, int t, int &q,
+__device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0, int u1, int gw, int g, int t,
+                                         uint32_t tag, int &q,
                                          int &prob_end, int &nsb, int &r, int &tile_lo, int &seg_end,
                                          const uint16_t *(&xcur)[NT], float (&acc)[NT][4]) {
     if constexpr (M1) {
@@ -552,7 +608,7 @@ __device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0,
         acc[0][0] = vg;
         acc[0][2] = vg8;
     }
-    flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, acc);
+    flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, tag, acc);
 #pragma unroll
     for (int a = 0; a < NT; ++a)
 #pragma unroll
@@ -587,7 +643,7 @@ __global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const
     const int gw = blockIdx.x * G::kWarps + warp;
     const uint32_t base = (uint32_t)__cvta_generic_to_shared(smem);
     if (base > G::kMaxSmemBase) {  // layout precondition (checked, never expected)
-        if (threadIdx.x == 0) atomicOr(P.status, kStatusLayout);
+        if (threadIdx.x == 0) atomicOr(P.header + kHeaderStatus, kStatusLayout);
         return;
     }
     const uint32_t ring =
@@ -629,11 +685,13 @@ __global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const
         }
     }
     __syncthreads();
-    grid_dependency_wait();  // pre-rotated activations and counters are ready
+    grid_dependency_wait();  // pre-rotated activations and the header are ready
     // every CTA of this grid is resident: the next pre-rotation may launch and
     // wait (it waits for this grid's completion before writing anything)
     grid_dependents_launch();
     if (!active) return;
+    // this call's tag (advanced by the launch that prepared the header)
+    const uint32_t tag = *reinterpret_cast<volatile const unsigned *>(P.header + kHeaderTag);
 
     const int g = lane >> 2, t = lane & 3;
     // PRMT operand: byte 0 = lane*4, bytes 2..3 = table base >> 16
@@ -685,7 +743,7 @@ __global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const
                 if (!__all_sync(kFull, ok)) {
                     // report, then let the copies still in flight land before leaving
                     if (lane == 0) {
-                        atomicOr(P.status, kStatusTimeout);
+                        atomicOr(P.header + kHeaderStatus, kStatusTimeout);
                         int s2 = stage;
                         uint32_t p2 = parity;
                         for (int i = 1; i < kStages && u + kPerStage * i < pv; ++i) {
@@ -710,7 +768,7 @@ __global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const
             for (int a = 0; a < NT; ++a) xcur[a] += 256;
             u += 2;
             if (u == seg_end)
-                end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
+                end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, tag, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
         } else {
             for (int h = 0; h < cnt; ++h) {
                 unit_any<NT, M1, CT>(st + h * kUnitCodeBytes, st + kStageScaleOff + h * SB, xcur, 0, lut_lane, off_c,
@@ -719,7 +777,7 @@ __global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const
                 for (int a = 0; a < NT; ++a) xcur[a] += 128;
                 ++u;
                 if (u == seg_end)
-                    end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
+                    end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, tag, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
             }
         }
         __syncwarp();  // every lane has read the stage: it may be refilled
@@ -807,15 +865,13 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
     pl.total_warps = (int)(pl.units < warps ? pl.units : warps);
     const int64_t mm = m < 1 ? 1 : (m > 32 ? 32 : m);
     pl.mcap = (int)(8 * ((mm + 7) / 8));
-    pl.counter_bytes = round_up((size_t)pl.tiles * 4u, 256);
-    pl.partial_bytes = round_up((size_t)(pl.tiles + pl.total_warps) * 16u * (size_t)pl.mcap * 4u, 256);
+    pl.partial_bytes = round_up((size_t)(pl.tiles + pl.total_warps) * 16u * (size_t)pl.mcap * 8u, 256);
     return pl;
 }
 
 template <int CODEC>
 cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
-                               unsigned *counters, float *partials, unsigned *status, bool programmatic,
-                               cudaStream_t stream) {
+                               unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream) {
     if (count < 1 || count > kMaxProblems) return cudaErrorInvalidValue;
     GroupParams prm = {};
     int64_t ub = 0, tb = 0;
@@ -840,8 +896,7 @@ cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, i
     prm.units = ub;
     prm.total_warps = plan.total_warps;
     prm.partials = partials;
-    prm.counters = counters;
-    prm.status = status;
+    prm.header = header;
     prm.inject_skip = (g_debug_flags & 1u) ? 1 : 0;
     prm.inv_units = 1.0 / (double)prm.units;
     prm.inv_warps = 1.0 / (double)prm.total_warps;
@@ -862,17 +917,13 @@ cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, i
 }
 
 cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
-                         unsigned *counters, float *partials, unsigned *status, bool programmatic,
-                         cudaStream_t stream) {
-    return launch_group_codec<kCodecTQ4>(probs, count, m, ydtype, plan, counters, partials, status, programmatic,
-                                         stream);
+                         unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream) {
+    return launch_group_codec<kCodecTQ4>(probs, count, m, ydtype, plan, header, partials, programmatic, stream);
 }
 
 cudaError_t launch_group_nvfp4(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
-                               unsigned *counters, float *partials, unsigned *status, bool programmatic,
-                               cudaStream_t stream) {
-    return launch_group_codec<kCodecNVFP4>(probs, count, m, ydtype, plan, counters, partials, status, programmatic,
-                                           stream);
+                               unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream) {
+    return launch_group_codec<kCodecNVFP4>(probs, count, m, ydtype, plan, header, partials, programmatic, stream);
 }
 
 }  // namespace tq

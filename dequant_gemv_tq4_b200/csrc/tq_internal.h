@@ -43,8 +43,7 @@ struct RotParams {
     RotInput in[kMaxInputs];
     int count;
     int64_t units;
-    unsigned *counters;
-    int64_t counters_count;
+    unsigned *header;  // product workspace header (see below), or nullptr
 };
 
 struct RotJob {  // host-side request
@@ -54,10 +53,22 @@ struct RotJob {  // host-side request
     uint16_t *xrot;
 };
 
-// xrot for m rows of every job (same dtype); also zeroes `counters`.  With
-// rotate = false the activation is only converted to fp16 fragment order.
-cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *counters,
-                             int64_t counters_count, cudaStream_t stream, bool rotate = true);
+// Header of a fused-product workspace (its first 256 bytes): word 0 is the
+// status word (timeout flag), word 1 the call tag.  Every call first clears
+// the status and advances the tag; the product's split-K partial sums are
+// stored with the tag of their call, so entries of earlier calls never match.
+constexpr int kHeaderStatus = 0;
+constexpr int kHeaderTag = 1;
+
+// xrot for m rows of every job (same dtype); also prepares `header` (status
+// cleared, tag advanced) when it is not null.  With rotate = false the
+// activation is only converted to fp16 fragment order.
+cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *header,
+                             cudaStream_t stream, bool rotate = true);
+
+// Only the header preparation (for products whose activation is already
+// pre-rotated).  Launched as a programmatic dependent like the pre-rotation.
+cudaError_t launch_prepare_header(unsigned *header, cudaStream_t stream);
 
 // ---- fused product ---------------------------------------------------------
 struct GemvProblem {  // host-side request, m <= 32 rows of pre-rotated activations
@@ -77,8 +88,7 @@ struct GroupPlan {
     int grid;             // CTAs (<= SM count)
     int total_warps;      // min(grid * warps per CTA, units); warp w owns [w*U/W, (w+1)*U/W)
     int mcap;             // 8 * ceil(m / 8)
-    size_t counter_bytes; // tiles * 4, rounded up to 256
-    size_t partial_bytes; // (tiles + total_warps) * 16 * mcap * 4, rounded up to 256
+    size_t partial_bytes; // (tiles + total_warps) * 16 * mcap * 8 (value + tag), rounded up to 256
 };
 
 GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, int sm_count);
@@ -88,16 +98,14 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
 void set_debug_flags(uint32_t flags);
 
 cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
-                         unsigned *counters, float *partials, unsigned *status, bool programmatic,
-                         cudaStream_t stream);
+                         unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream);
 
 // ---- NVFP4 comparison codec ---------------------------------------------------
 // Same fused product over NVFP4 planes (E2M1 codes in the TQ4_1S unit layout,
 // E4M3 block scales, a device fp32 tensor scale per problem); xrot holds the
 // activation in fragment order without rotation (launch_prerotate, rotate=false).
 cudaError_t launch_group_nvfp4(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
-                               unsigned *counters, float *partials, unsigned *status, bool programmatic,
-                               cudaStream_t stream);
+                               unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream);
 
 cudaError_t launch_nvfp4_amax(const void *w, int dtype, int64_t n, int64_t k, int64_t ldw, unsigned *amax_bits,
                               cudaStream_t stream);

@@ -142,8 +142,15 @@ TQ_API tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, 
 
 /* Workspace bytes needed by tq_gemm / tq_gemv / tq_gemm_xrot on the CURRENT
  * device for these sizes (the split-K partition depends on its SM count).
- * Layout: a status word (256 bytes), split-K counters, partial sums and the
- * pre-rotated activation. */
+ * Layout: a 256-byte header (status word, call tag), the split-K partial
+ * sums and the pre-rotated activation.
+ *
+ * Every call clears the status word and advances the 32-bit call tag before
+ * its product; split-K partial sums are stored together with the tag of
+ * their call, so words left by earlier calls never match.  A workspace that
+ * has never been used holds arbitrary bytes and a stale word could match the
+ * first call's tag by chance (probability 2^-32 per word read): zero-fill a
+ * new workspace once (later calls need no clearing). */
 TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -156,8 +163,8 @@ TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *              (ldy >= n)
  *   workspace  device, >= tq_gemm_workspace_bytes(m, n, k) bytes, 256-byte
  *              aligned, exclusively owned by this call until it completes
- *              on `stream` (no zero-fill needed; calls that overlap on the
- *              GPU must use different workspaces)
+ *              on `stream` (zero-filled once when new, see above; calls
+ *              that overlap on the GPU must use different workspaces)
  * m <= 32 runs the skinny kernel in one pass; larger m runs it once per
  * 32-row slice of X (weights re-read per slice).
  */
@@ -172,9 +179,9 @@ TQ_API tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n
 /*
  * tq_gemm_xrot -- the product with an activation already pre-rotated by
  * tq_prerotate (one xrot shared by every matrix that consumes the same
- * input, e.g. q/k/v).  m <= 32.  Same workspace rules as tq_gemm (no
- * zero-fill needed: the call clears its split-K counters with one
- * cudaMemsetAsync on `stream` before the kernel).
+ * input, e.g. q/k/v).  m <= 32.  Same workspace rules as tq_gemm (a
+ * one-thread launch on `stream` clears the status word and advances the call
+ * tag before the product).
  */
 TQ_API tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const uint16_t *xrot,
                        int64_t m, void *Y, tq_dtype yt, int64_t ldy, void *workspace, size_t ws_bytes, void *stream);
