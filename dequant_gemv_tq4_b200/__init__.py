@@ -85,6 +85,8 @@ def load_library() -> ctypes.CDLL:
             "tq_workspace_status": ([P, I, P], I),
             "tq_debug_set_flags": ([ctypes.c_uint32], None),
             "tq_gemv_static_scratch": ([P, P, I64, I64, P, I, P, I, P], I),
+            "tq_gemm_prefill_workspace_bytes": ([I64, I64], SZ),
+            "tq_gemm_prefill": ([P, P, I64, I64, P, I, I64, I64, P, I, I64, P, SZ, P], I),
             "tq_nvfp4_scales_bytes": ([I64, I64], SZ),
             "tq_nvfp4_quantize": ([P, I, I64, I64, I64, P, P, P, P], I),
             "tq_nvfp4_dequantize": ([P, P, P, I64, I64, P, I, I64, P], I),
@@ -173,6 +175,15 @@ def tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream) -> int:
     device memory: the scratch is a fixed array inside the library (see
     include/tq.h).  Calls that overlap on the GPU must not share it."""
     return load_library().tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream)
+
+
+def tq_gemm_prefill_workspace_bytes(m: int, k: int) -> int:
+    return int(load_library().tq_gemm_prefill_workspace_bytes(m, k))
+
+
+def tq_gemm_prefill(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_gemm_prefill(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes,
+                                          stream)
 
 
 def tq_nvfp4_scales_bytes(n: int, k: int) -> int:
@@ -282,6 +293,28 @@ def gemm(codes, scales, n: int, k: int, X: torch.Tensor, dtype=torch.float32, ou
     _check(tq_gemm(codes.data_ptr(), scales.data_ptr(), n, k, X2.data_ptr(), _dt(X2.dtype), m, _ld(X2),
                    out.data_ptr(), _dt(out.dtype), _ld(out), ws.data_ptr(), ws.numel(), _stream(stream)),
            "tq_gemm")
+    return out
+
+
+def prefill_workspace(m: int, k: int, device=None) -> torch.Tensor:
+    nbytes = tq_gemm_prefill_workspace_bytes(m, k)
+    if nbytes == 0:
+        raise ValueError("invalid sizes for workspace query")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or torch.cuda.current_device())
+
+
+def gemm_prefill(codes, scales, n: int, k: int, X: torch.Tensor, dtype=torch.float32, out=None, ws=None,
+                 stream=None) -> torch.Tensor:
+    """Y[m, n] = X[m, k] @ w~[n, k]^T on the tensor-core prefill path (any m)."""
+    X2 = X.view(1, -1) if X.dim() == 1 else X
+    m = X2.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=dtype, device=X.device)
+    if ws is None:
+        ws = prefill_workspace(m, k, X.device)
+    _check(tq_gemm_prefill(codes.data_ptr(), scales.data_ptr(), n, k, X2.data_ptr(), _dt(X2.dtype), m, _ld(X2),
+                           out.data_ptr(), _dt(out.dtype), _ld(out), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "tq_gemm_prefill")
     return out
 
 

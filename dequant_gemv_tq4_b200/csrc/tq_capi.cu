@@ -154,8 +154,17 @@ tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t
     return from_cuda(tq::launch_prerotate(&job, 1, xt, m, nullptr, (cudaStream_t)stream));
 }
 
+// Products with more activation rows than the skinny kernel takes run on
+// the tcgen05 prefill kernel.
+constexpr int64_t kSkinnyMaxM = 32;
+
+static size_t prefill_workspace(int64_t m, int64_t k) {
+    return kStatusBytes + tq::prefill_xrot_bytes(m < 1 ? 1 : m, k);
+}
+
 size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 0 || check_nk(n, k) != TQ_OK) return 0;
+    if (m > kSkinnyMaxM) return prefill_workspace(m, k);
     Layout lay;
     if (make_layout(&n, &k, 1, &k, 1, m, &lay) != TQ_OK) return 0;
     return lay.total;
@@ -180,6 +189,20 @@ static tq_status check_gemm_common(const uint8_t *codes, const uint16_t *scales,
 static tq_status check_workspace(void *workspace, size_t ws_bytes, size_t need) {
     if (!workspace || !aligned(workspace, 256) || ws_bytes < need) return TQ_ERR_WORKSPACE;
     return TQ_OK;
+}
+
+static tq_status run_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
+                             tq_dtype xt, int64_t m, int64_t ldx, void *Y, tq_dtype yt, int64_t ldy, void *workspace,
+                             size_t ws_bytes, void *stream) {
+    tq_status st;
+    if ((st = check_workspace(workspace, ws_bytes, prefill_workspace(m, k))) != TQ_OK) return st;
+    if ((m + 255) / 256 > 65535) return TQ_ERR_SHAPE;
+    char *ws = static_cast<char *>(workspace);
+    const cudaError_t e =
+        tq::launch_prefill(codes, scales, n, k, X, xt, m, ldx, reinterpret_cast<uint16_t *>(ws + kStatusBytes), Y, yt,
+                           ldy, reinterpret_cast<unsigned *>(ws), (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
 }
 
 tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const uint16_t *xrot,
@@ -209,6 +232,7 @@ tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64
     if (st != TQ_OK || n == 0 || m == 0) return st;
     if (!valid_dtype(xt)) return TQ_ERR_DTYPE;
     if ((st = check_matrix_operand(X, ldx, k)) != TQ_OK) return st;
+    if (m > kSkinnyMaxM) return run_prefill(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream);
     Layout lay;
     if ((st = make_layout(&n, &k, 1, &k, 1, m, &lay)) != TQ_OK) return st;
     if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
@@ -233,6 +257,21 @@ tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64
 tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *x, tq_dtype xt,
                   void *y, tq_dtype yt, void *workspace, size_t ws_bytes, void *stream) {
     return tq_gemm(codes, scales, n, k, x, xt, 1, k, y, yt, n, workspace, ws_bytes, stream);
+}
+
+size_t tq_gemm_prefill_workspace_bytes(int64_t m, int64_t k) {
+    if (m < 0 || check_nk(0, k) != TQ_OK) return 0;
+    return prefill_workspace(m, k);
+}
+
+tq_status tq_gemm_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
+                          tq_dtype xt, int64_t m, int64_t ldx, void *Y, tq_dtype yt, int64_t ldy, void *workspace,
+                          size_t ws_bytes, void *stream) {
+    tq_status st = check_gemm_common(codes, scales, n, k, m, Y, yt, ldy);
+    if (st != TQ_OK || n == 0 || m == 0) return st;
+    if (!valid_dtype(xt)) return TQ_ERR_DTYPE;
+    if ((st = check_matrix_operand(X, ldx, k)) != TQ_OK) return st;
+    return run_prefill(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream);
 }
 
 // ---- batch: several matrices, one pre-rotation per distinct input ----------

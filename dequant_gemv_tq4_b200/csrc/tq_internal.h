@@ -100,6 +100,15 @@ void set_debug_flags(uint32_t flags);
 cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
                          unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream);
 
+// ---- large-M product on tcgen05 (tq_prefill.cu) ---------------------------------
+// Y = X w~^T for any m: X is first pre-rotated into plain row-major fp16 xrot
+// (prefill_xrot_bytes), then one CTA per 128 weight rows x 256 activation rows
+// decodes the weight tile into shared memory and multiplies on the tensor cores.
+size_t prefill_xrot_bytes(int64_t m, int64_t k);
+cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
+                           int xdtype, int64_t m, int64_t ldx, uint16_t *xrot, void *y, int ydtype, int64_t ldy,
+                           unsigned *header, cudaStream_t stream);
+
 // ---- NVFP4 comparison codec ---------------------------------------------------
 // Same fused product over NVFP4 planes (E2M1 codes in the TQ4_1S unit layout,
 // E4M3 block scales, a device fp32 tensor scale per problem); xrot holds the

@@ -1,0 +1,596 @@
+// tq_prefill.cu -- the large-M product (prefill) on the fifth-generation
+// tensor cores: Y = X w~^T for TQ4_1S weights, many activation rows.
+//
+// Method: TQ4_1S page ("企业官网建设流程全解析", hotelren.com/news/5458160),
+// section 解码速度：分硬件汇总: the activation is rotated once with the block
+// transform; afterwards every weight contributes centroid(code) * scale.  The
+// same holds for a whole matrix of activations:
+//
+//   Y[m][r] = sum_blocks sum_e c[r][e] * xrot[m][e],   c = +-M[mag] * d_half
+//
+// so the weights enter the tensor cores as decoded centroids times their fp16
+// half-block scale, with no per-weight inverse transform, and X enters as its
+// fp16 pre-rotation H(s .* x)/32.
+//
+// B200 design:
+//  * One CTA per output tile of 128 weight rows x 256 activation rows (one
+//    tcgen05.mma of M = 128, N = 256, K = 16 per 16 columns; fp32 accumulator
+//    of 128 lanes x 256 columns in tensor memory).  Both operands are K-major
+//    in shared memory with the 128-byte swizzle.
+//  * The activation tile (256 rows x 64 columns of fp16 per stage) arrives by
+//    TMA (cp.async.bulk.tensor, no multicast).
+//  * The weight tile (128 rows x 64 columns per stage) is decoded by four
+//    warps, one row per thread: the row's code words come from global memory
+//    (one stage ahead, in registers), a 4x4 byte transpose restores element
+//    order, a lane-replicated shared table turns each code byte into an fp16
+//    pair, one fp16 multiply applies the half-block scale, and 16-byte stores
+//    write the swizzled rows.  A proxy fence then publishes them to the tensor
+//    cores.
+//  * One thread issues the MMAs; tcgen05.commit releases each stage to its
+//    producers and finally signals the epilogue.  The four decode warps then
+//    read the accumulator (tcgen05.ld, one weight row per thread) and store Y
+//    with consecutive threads on consecutive columns.
+//  * Three stages; every mbarrier wait is bounded in time and reports through
+//    the workspace status word.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+
+namespace {
+
+constexpr int kPM = 128;                 // weight rows per tile (MMA M)
+constexpr int kPN = 256;                 // activation rows per tile (MMA N)
+constexpr int kPK = 64;                  // columns per stage: one 128-byte swizzle row of fp16
+constexpr int kPStages = 3;
+constexpr int kATile = kPM * kPK * 2;    // 16 KB
+constexpr int kBTile = kPN * kPK * 2;    // 32 KB
+constexpr int kDecodeWarps = 4;          // warps 2..5
+constexpr int kPThreads = (2 + kDecodeWarps) * 32;
+constexpr int kTmemCols = 256;
+
+// Shared-memory map (addresses in the CTA's shared window; the dynamic
+// allocation starts at a base B <= kPMaxBase):
+//   [align1024(B), + 3 x 16 KB)   weight tiles (A)
+//   [0x10000, 0x20000)            code-pair table (entry v, lane l at 256 v + 4 l)
+//   [0x20000, 0x38000)            activation tiles (B), 3 x 32 KB
+//   [0x38000, ...)                mbarriers, tensor-memory address
+constexpr uint32_t kPLut = 0x10000;
+constexpr uint32_t kPBTiles = 0x20000;
+constexpr uint32_t kPBars = kPBTiles + kPStages * kBTile;  // full_a[3] full_b[3] empty[3] accum
+constexpr uint32_t kPTmemSlot = kPBars + 16 * 8;
+constexpr uint32_t kPEnd = kPTmemSlot + 16;
+constexpr uint32_t kPMaxBase = 0x10000 - kPStages * kATile - 1024;
+static_assert(kPEnd - 1024 <= 227 * 1024, "dynamic shared memory per CTA");
+
+constexpr unsigned kPStatusTimeout = 1u;
+constexpr unsigned kPStatusLayout = 2u;
+
+__constant__ uint16_t c_pmag_f16[8] = TQ_MAG_F16_INIT;
+
+// ---- PTX wrappers -----------------------------------------------------------
+__device__ __forceinline__ uint64_t p_global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void p_mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool p_mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of a barrier; false after timeout_ns (or 2^30 polls).
+__device__ __noinline__ bool p_mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+    if (p_mbar_try(bar, parity)) return true;
+    const uint64_t t0 = p_global_ns();
+    for (uint32_t it = 0; it < (1u << 30); ++it) {
+        if (p_mbar_try(bar, parity)) return true;
+        if (p_global_ns() - t0 > timeout_ns) return false;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void p_mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void p_mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// 2-D TMA load of box {64 columns, 256 rows} at (x = column, y = row).
+__device__ __forceinline__ void p_tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Generic-proxy shared-memory writes become visible to the async proxy
+// (tensor-core operand reads).
+__device__ __forceinline__ void p_fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void p_tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void p_tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory operand descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), descriptor version 1.
+__device__ __forceinline__ uint64_t p_smem_desc(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t kPIdesc = (1u << 4) | ((uint32_t)(kPN >> 3) << 17) | ((uint32_t)(kPM >> 4) << 24);
+
+__device__ __forceinline__ void p_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kPIdesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` once every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void p_mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void p_tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t p_lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
+__device__ __forceinline__ void p_sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+__device__ __forceinline__ uint32_t p_hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+struct PrefillParams {
+    const uint8_t *codes;   // TQ4_1S codes plane
+    const uint8_t *scales;  // TQ4_1S scales plane (fp16 pairs)
+    int n;                  // weight rows
+    int tiles;              // ceil(n / 16)
+    int nsb;                // superblocks per row
+    int m;                  // activation rows
+    int nk;                 // 64-column stages: ceil(k / 64)
+    char *y;
+    int64_t ldy;
+    unsigned *header;       // workspace header (status word)
+    uint64_t timeout_ns;
+};
+
+// One weight row's words for one 64-column stage: for each of the four
+// 16-byte chunks of the row's superblock slot, the two words that belong to
+// the stage's two blocks; and the (d0, d1) fp16 pairs of those blocks.
+struct RowWords {
+    uint2 c[4];
+    uint2 s;
+};
+
+__device__ __forceinline__ uint2 p_ldg64(const void *ptr) {
+    uint2 r;
+    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(ptr));
+    return r;
+}
+
+__device__ __forceinline__ RowWords load_row(const PrefillParams &P, int row, int kt) {
+    RowWords w;
+    if (row >= P.tiles * 16) {  // past the padded rows of the last tile
+#pragma unroll
+        for (int b = 0; b < 4; ++b) w.c[b] = make_uint2(0u, 0u);
+        w.s = make_uint2(0u, 0u);
+        return w;
+    }
+    const int sb = kt >> 1, hb = kt & 1;  // superblock, and which half of it (blocks 2hb, 2hb+1)
+    const size_t slot = ((size_t)(row >> 4) * P.nsb + sb) * 16 + (row & 15);
+    const uint8_t *c = P.codes + slot * 64 + 8 * hb;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) w.c[b] = p_ldg64(c + 16 * b);
+    w.s = p_ldg64(P.scales + slot * 16 + 8 * hb);
+    return w;
+}
+
+// 4x4 byte transpose: out[i] byte b = in[b] byte i.
+__device__ __forceinline__ void p_transpose4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t (&o)[4]) {
+    const uint32_t a = prmt(w0, w1, 0x5140u), b = prmt(w2, w3, 0x5140u);
+    const uint32_t c = prmt(w0, w1, 0x7362u), d = prmt(w2, w3, 0x7362u);
+    o[0] = prmt(a, b, 0x5410u);
+    o[1] = prmt(a, b, 0x7632u);
+    o[2] = prmt(c, d, 0x5410u);
+    o[3] = prmt(c, d, 0x7632u);
+}
+
+// Decode one row's 64 columns into the swizzled weight tile.  In a row's
+// 64-byte superblock slot, logical byte L of block j sits at chunk L % 4,
+// word j, byte L / 4; so for a fixed block the four chunks' words, byte-
+// transposed, give logical words i = 0..3, each holding elements 8i .. 8i+7
+// (element 2L in the low nibble of byte L).  Logical word i of block jj lands
+// in 16-byte chunk 4 jj + i of the tile row, stored at chunk (4 jj + i) xor
+// (row % 8) (the 128-byte swizzle).
+__device__ __forceinline__ void decode_row(const RowWords &w, int row, uint32_t atile, uint32_t lut_lane) {
+    const uint32_t rbase = atile + (uint32_t)row * 128u;
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+        uint32_t L[4];
+        if (jj == 0)
+            p_transpose4(w.c[0].x, w.c[1].x, w.c[2].x, w.c[3].x, L);
+        else
+            p_transpose4(w.c[0].y, w.c[1].y, w.c[2].y, w.c[3].y, L);
+        const uint32_t sw = jj == 0 ? w.s.x : w.s.y;  // (d0, d1) of the block
+        const uint32_t d0 = prmt(sw, sw, 0x1010u), d1 = prmt(sw, sw, 0x3232u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t d = i < 2 ? d0 : d1;  // elements 0..15 take d0, 16..31 d1
+            const uint32_t o0 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7604u)), d);
+            const uint32_t o1 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7614u)), d);
+            const uint32_t o2 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7624u)), d);
+            const uint32_t o3 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7634u)), d);
+            const uint32_t chunk = (uint32_t)(4 * jj + i) ^ (uint32_t)(row & 7);
+            p_sts128(rbase + chunk * 16u, o0, o1, o2, o3);
+        }
+    }
+}
+
+template <int OT>
+__global__ void __launch_bounds__(kPThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PrefillParams P) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(smem);
+    if (base > kPMaxBase) {  // layout precondition (checked, never expected)
+        if (threadIdx.x == 0) atomicOr(P.header, kPStatusLayout);
+        return;
+    }
+    const uint32_t abase = (base + 1023u) & ~1023u;
+    const int n0 = blockIdx.x * kPM, m0 = blockIdx.y * kPN;
+    auto a_tile = [&](int s) { return abase + (uint32_t)s * kATile; };
+    auto b_tile = [&](int s) { return kPBTiles + (uint32_t)s * kBTile; };
+    auto full_a = [&](int s) { return kPBars + 8u * s; };
+    auto full_b = [&](int s) { return kPBars + 24u + 8u * s; };
+    auto empty = [&](int s) { return kPBars + 48u + 8u * s; };
+    const uint32_t accum = kPBars + 72u;
+
+    // ---- set-up: barriers, code-pair table, tensor memory ------------------
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            p_mbar_init(full_a(s), 32 * kDecodeWarps);
+            p_mbar_init(full_b(s), 1);
+            p_mbar_init(empty(s), 1);
+        }
+        p_mbar_init(accum, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    {
+        uint4 *lut = reinterpret_cast<uint4 *>(smem + (kPLut - base));
+        for (int idx = threadIdx.x; idx < 256 * 8; idx += kPThreads) {  // entry v: 8 x 16 bytes
+            const int v = idx >> 3;
+            const uint32_t lo = c_pmag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
+            const uint32_t hi = c_pmag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
+            const uint32_t e = lo | (hi << 16);
+            lut[v * 16 + (idx & 7)] = make_uint4(e, e, e, e);
+        }
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(kPTmemSlot),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    p_tc_fence_before();
+    __syncthreads();
+    p_tc_fence_after();
+    const uint32_t tmem = p_lds_u32(kPTmemSlot);
+    // the activation tiles are the pre-rotation's output
+    grid_dependency_wait();
+    grid_dependents_launch();
+
+    if (warp == 0) {
+        // ---- activation tiles by TMA ----------------------------------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int kt = 0; kt < P.nk; ++kt) {
+                const int s = kt % kPStages;
+                const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
+                if (!p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns)) {
+                    atomicOr(P.header, kPStatusTimeout);
+                    break;
+                }
+                p_mbar_expect_tx(full_b(s), kBTile);
+                p_tma_load_2d(b_tile(s), &xmap, kt * kPK, m0, full_b(s));
+                ++issued;
+            }
+            // no copy may still be in flight when the CTA exits
+            for (int kt = issued > kPStages ? issued - kPStages : 0; kt < issued; ++kt)
+                p_mbar_wait(full_b(kt % kPStages), (uint32_t)(kt / kPStages) & 1u, P.timeout_ns);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---- MMA issue ----------------------------------------------------------
+        if (lane == 0) {
+            for (int kt = 0; kt < P.nk; ++kt) {
+                const int s = kt % kPStages;
+                const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
+                if (!p_mbar_wait(full_a(s), ph, P.timeout_ns) || !p_mbar_wait(full_b(s), ph, P.timeout_ns)) {
+                    atomicOr(P.header, kPStatusTimeout);
+                    break;
+                }
+                p_tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kPK / 16; ++kk)  // 16 columns = 32 bytes along the swizzled row
+                    p_mma(tmem, p_smem_desc(a_tile(s) + 32u * kk), p_smem_desc(b_tile(s) + 32u * kk),
+                          (kt | kk) != 0 ? 1u : 0u);
+                p_mma_commit(empty(s));  // the stage is free once these MMAs have read it
+            }
+            p_mma_commit(accum);  // the accumulator is final once every MMA has completed
+        }
+        __syncwarp();
+    } else {
+        // ---- weight tiles: decode ---------------------------------------------
+        const int row = (warp - 2) * 32 + lane;  // tile row of this thread
+        const uint32_t lut_lane = kPLut | ((uint32_t)lane * 4u);
+        RowWords cur = load_row(P, n0 + row, 0);
+        for (int kt = 0; kt < P.nk; ++kt) {
+            const int s = kt % kPStages;
+            const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
+            RowWords nxt = cur;
+            if (kt + 1 < P.nk) nxt = load_row(P, n0 + row, kt + 1);  // one stage ahead
+            // (warp-uniform decision: the epilogue below runs warp-synchronous loads)
+            if (!__all_sync(kFull, p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns))) {
+                if (lane == 0) atomicOr(P.header, kPStatusTimeout);
+                break;
+            }
+            decode_row(cur, row, a_tile(s), lut_lane);
+            p_fence_proxy_async();
+            p_mbar_arrive(full_a(s));
+            cur = nxt;
+        }
+        // ---- epilogue: tensor memory -> Y ------------------------------------
+        const int q = warp & 3;                 // this warp's quarter of the 128 lanes
+        const int wrow = n0 + q * 32 + lane;    // weight row = accumulator lane
+        if (!__all_sync(kFull, p_mbar_wait(accum, 0u, P.timeout_ns))) {
+            if (lane == 0) atomicOr(P.header, kPStatusTimeout);
+        } else {
+            p_tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < kPN / 32; ++c) {
+                uint32_t v[32];
+                p_tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
+                if (wrow < P.n) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int mrow = m0 + c * 32 + e;
+                        if (mrow < P.m)
+                            store1<OT>(P.y + ((int64_t)mrow * P.ldy + wrow) * ElemSize<OT>::value,
+                                       __uint_as_float(v[e]));
+                    }
+                }
+            }
+        }
+    }
+    // ---- teardown ---------------------------------------------------------------
+    p_tc_fence_before();
+    __syncthreads();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+}
+
+// ---- pre-rotation of X into plain row-major fp16 ---------------------------------
+// xrot[row][col] = fp16(H(s .* x)/32) per 32-block (one warp per row and
+// superblock: lane = block j (lane / 8) and four consecutive elements
+// (lane % 8)); also clears the workspace status word.
+struct PlainRotParams {
+    const char *x;
+    int64_t ldx;
+    uint16_t *xrot;
+    int64_t m;
+    int k;
+    int nsb;
+    unsigned *header;
+};
+
+template <int DT>
+__global__ void __launch_bounds__(256) prerotate_plain_kernel(const __grid_constant__ PlainRotParams R) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    if (R.header && blockIdx.x == 0 && threadIdx.x == 0) {
+        R.header[kHeaderStatus] = 0u;
+        R.header[kHeaderTag] += 1u;
+    }
+    const int lane = threadIdx.x & 31;
+    const int j = lane >> 3, p = lane & 7;
+    const int64_t warps = (int64_t)gridDim.x * 8;
+    for (int64_t wu = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); wu < R.m * R.nsb; wu += warps) {
+        const int64_t row = wu / R.nsb;
+        const int sb = (int)(wu - row * R.nsb);
+        const uint32_t col0 = (uint32_t)sb * 128u + 32u * j + 4u * p;
+        const bool valid = (int)col0 < R.k;  // k is a multiple of 32: whole blocks
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        if (valid) load4<DT>(R.x + (row * R.ldx + col0) * ElemSize<DT>::value, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = flip(v[i], sign_mask(col0 + i));
+        butterfly_local4(v);
+#pragma unroll
+        for (int st = 0; st < 3; ++st) {
+            const int xo = 1 << st;
+            const bool upper = (p & xo) != 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] = butterfly_xlane(v[i], xo, upper);
+        }
+        if (valid) {
+            const __half2 lo = __floats2half2_rn(__fmul_rn(v[0], 0.03125f), __fmul_rn(v[1], 0.03125f));
+            const __half2 hi = __floats2half2_rn(__fmul_rn(v[2], 0.03125f), __fmul_rn(v[3], 0.03125f));
+            uint2 o;
+            o.x = *reinterpret_cast<const uint32_t *>(&lo);
+            o.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(R.xrot + row * R.k + col0) = o;
+        }
+    }
+}
+
+// ---- host side ------------------------------------------------------------------
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to
+// the driver library).
+EncodeTiled encode_tiled() {
+    static std::once_flag once;
+    static EncodeTiled fn = nullptr;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(ptr);
+    });
+    return fn;
+}
+
+// Base offset of dynamic shared memory in a CTA's shared window.
+uint32_t prefill_smem_base() {
+    int dev = 0, reserved = 1024;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+        reserved = 1024;
+    return (uint32_t)reserved;
+}
+
+cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
+
+template <int OT>
+cudaError_t launch_prefill_kernel(const CUtensorMap &map, const PrefillParams &prm, dim3 grid, uint32_t smem,
+                                  cudaStream_t stream) {
+    cudaError_t err =
+        cudaFuncSetAttribute(prefill_kernel<OT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<OT>, map, prm);
+}
+
+template <int DT>
+cudaError_t launch_plain_rotation(const PlainRotParams &r, cudaStream_t stream) {
+    const int64_t warps = r.m * r.nsb;
+    int64_t grid = (warps + 7) / 8;
+    if (grid > 148 * 16) grid = 148 * 16;
+    if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prerotate_plain_kernel<DT>, r);
+}
+
+}  // namespace
+
+size_t prefill_xrot_bytes(int64_t m, int64_t k) { return round_up((size_t)m * (size_t)k * 2u, 256); }
+
+cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
+                           int xdtype, int64_t m, int64_t ldx, uint16_t *xrot, void *y, int ydtype, int64_t ldy,
+                           unsigned *header, cudaStream_t stream) {
+    if (n < 1 || m < 1 || k < 32 || k % 32 != 0) return cudaErrorInvalidValue;
+    const int64_t grid_y = (m + kPN - 1) / kPN, grid_x = (n + kPM - 1) / kPM;
+    if (grid_y > 65535 || grid_x > 0x7fffffff) return cudaErrorInvalidValue;
+    EncodeTiled encode = encode_tiled();
+    if (!encode) return cudaErrorNotSupported;
+    // 1. X -> plain fp16 pre-rotation (clears the status word)
+    PlainRotParams r = {static_cast<const char *>(X), ldx, xrot, m, (int)k, (int)superblocks(k), header};
+    cudaError_t err;
+    switch (xdtype) {
+        case kF32: err = launch_plain_rotation<kF32>(r, stream); break;
+        case kBF16: err = launch_plain_rotation<kBF16>(r, stream); break;
+        case kF16: err = launch_plain_rotation<kF16>(r, stream); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (err != cudaSuccess) return err;
+    // 2. the tensor map of xrot: k x m fp16, rows of k*2 bytes, boxes of
+    //    64 columns x 256 rows, 128-byte swizzle, zero fill outside
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
+    const cuuint64_t strides[1] = {(cuuint64_t)k * 2u};
+    const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)kPN};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xrot, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    // 3. the product
+    PrefillParams prm;
+    prm.codes = codes;
+    prm.scales = reinterpret_cast<const uint8_t *>(scales);
+    prm.n = (int)n;
+    prm.tiles = (int)tiles(n);
+    prm.nsb = (int)superblocks(k);
+    prm.m = (int)m;
+    prm.nk = (int)((k + kPK - 1) / kPK);
+    prm.y = static_cast<char *>(y);
+    prm.ldy = ldy;
+    prm.header = header;
+    prm.timeout_ns = 1000000000ull;
+    const uint32_t base = prefill_smem_base();
+    if (base > kPMaxBase) return cudaErrorInvalidValue;
+    const uint32_t smem = kPEnd - base;
+    const dim3 grid((unsigned)grid_x, (unsigned)grid_y);
+    switch (ydtype) {
+        case kF32: return launch_prefill_kernel<kF32>(map, prm, grid, smem, stream);
+        case kBF16: return launch_prefill_kernel<kBF16>(map, prm, grid, smem, stream);
+        case kF16: return launch_prefill_kernel<kF16>(map, prm, grid, smem, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace tq

@@ -165,8 +165,9 @@ TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *              aligned, exclusively owned by this call until it completes
  *              on `stream` (zero-filled once when new, see above; calls
  *              that overlap on the GPU must use different workspaces)
- * m <= 32 runs the skinny kernel in one pass; larger m runs it once per
- * 32-row slice of X (weights re-read per slice).
+ * m <= 32 runs the skinny kernel in one pass; larger m runs the tensor-core
+ * prefill product of tq_gemm_prefill (its workspace is then the size that
+ * tq_gemm_workspace_bytes(m, n, k) returns for that m).
  */
 TQ_API tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X, tq_dtype xt,
                   int64_t m, int64_t ldx, void *Y, tq_dtype yt, int64_t ldy, void *workspace, size_t ws_bytes,
@@ -175,6 +176,27 @@ TQ_API tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n
 /* tq_gemv -- tq_gemm with m = 1 (x: k elements, y: n elements). */
 TQ_API tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *x, tq_dtype xt,
                   void *y, tq_dtype yt, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * tq_gemm_prefill -- the same product for many activation rows (prefill) on
+ * the fifth-generation tensor cores (TQ page, 解码速度 section: rotate the
+ * activation once, then every weight is centroid times scale).  X is first
+ * pre-rotated into a plain row-major fp16 matrix in the workspace; then each
+ * CTA takes 128 weight rows x 256 activation rows: it decodes its weight rows
+ * 64 columns at a time into shared memory (centroid x half-block scale, fp16),
+ * receives the matching activation columns by TMA, and accumulates
+ * tcgen05.mma products (fp16 operands, fp32 accumulator in tensor memory).
+ * Compared with tq_gemm's skinny path the weight enters as fp16(c * d), one
+ * more rounding per weight (relative 2^-11).  Same operand rules as tq_gemm;
+ * any m >= 1 (m <= 16,776,960).  Returns TQ_ERR_UNSUPPORTED if the driver
+ * offers no tensor-map encoder.
+ *   workspace  >= tq_gemm_prefill_workspace_bytes(m, k) bytes (256-byte
+ *              header + m*k fp16), 256-byte aligned
+ */
+TQ_API size_t tq_gemm_prefill_workspace_bytes(int64_t m, int64_t k);
+TQ_API tq_status tq_gemm_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
+                                 tq_dtype xt, int64_t m, int64_t ldx, void *Y, tq_dtype yt, int64_t ldy,
+                                 void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * tq_gemm_xrot -- the product with an activation already pre-rotated by
