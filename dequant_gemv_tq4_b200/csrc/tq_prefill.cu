@@ -19,17 +19,20 @@
 //    in shared memory with the 128-byte swizzle.
 //  * The activation tile (256 rows x 64 columns of fp16 per stage) arrives by
 //    TMA (cp.async.bulk.tensor, no multicast).
-//  * The weight tile (128 rows x 64 columns per stage) is decoded by four
-//    warps, one row per thread: the row's code words come from global memory
-//    (one stage ahead, in registers), a 4x4 byte transpose restores element
+//  * The weight tile (128 rows x 64 columns per stage) is decoded by eight
+//    warps, one row and one 32-column block per thread: each thread reads its
+//    row's 64-byte superblock slot with 16-byte loads (neighbouring threads,
+//    neighbouring slots), three superblocks ahead in registers; a 4x4 byte
+//    transpose restores element
 //    order, a lane-replicated shared table turns each code byte into an fp16
 //    pair, one fp16 multiply applies the half-block scale, and 16-byte stores
 //    write the swizzled rows.  A proxy fence then publishes them to the tensor
 //    cores.
 //  * One thread issues the MMAs; tcgen05.commit releases each stage to its
-//    producers and finally signals the epilogue.  The four decode warps then
-//    read the accumulator (tcgen05.ld, one weight row per thread) and store Y
-//    with consecutive threads on consecutive columns.
+//    producers and finally signals the epilogue.  The eight decode warps then
+//    read the accumulator (tcgen05.ld, one weight row per thread, two warps per
+//    32-lane quarter) and store Y with consecutive threads on consecutive
+//    columns.
 //  * Three stages; every mbarrier wait is bounded in time and reports through
 //    the workspace status word.
 #include <cuda.h>
@@ -49,9 +52,10 @@ constexpr int kPK = 64;                  // columns per stage: one 128-byte swiz
 constexpr int kPStages = 3;
 constexpr int kATile = kPM * kPK * 2;    // 16 KB
 constexpr int kBTile = kPN * kPK * 2;    // 32 KB
-constexpr int kDecodeWarps = 4;          // warps 2..5
+constexpr int kDecodeWarps = 8;          // warps 2..9: (row, block) per thread
 constexpr int kPThreads = (2 + kDecodeWarps) * 32;
 constexpr int kTmemCols = 256;
+constexpr int kAhead = 3;       // superblocks of row slots held in registers ahead of the decode
 
 // Shared-memory map (addresses in the CTA's shared window; the dynamic
 // allocation starts at a base B <= kPMaxBase):
@@ -198,75 +202,88 @@ struct PrefillParams {
     uint64_t timeout_ns;
 };
 
-// One weight row's words for one 64-column stage: for each of the four
-// 16-byte chunks of the row's superblock slot, the two words that belong to
-// the stage's two blocks; and the (d0, d1) fp16 pairs of those blocks.
-struct RowWords {
-    uint2 c[4];
-    uint2 s;
+// One weight row's superblock slot: its four 16-byte code chunks (chunk b,
+// word j holds byte b of logical words of block j, see decode_block) and its
+// 16 bytes of scales ((d0, d1) of blocks 0..3).
+struct RowSlot {
+    uint4 c[4];
+    uint4 s;
 };
 
-__device__ __forceinline__ uint2 p_ldg64(const void *ptr) {
-    uint2 r;
-    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(ptr));
+__device__ __forceinline__ uint4 p_ldg128(const void *ptr) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(ptr));
     return r;
 }
 
-__device__ __forceinline__ RowWords load_row(const PrefillParams &P, int row, int kt) {
-    RowWords w;
-    if (row >= P.tiles * 16) {  // past the padded rows of the last tile
+// Whole 64-byte slots with 16-byte loads: neighbouring threads read
+// neighbouring slots.
+__device__ __forceinline__ RowSlot load_slot(const PrefillParams &P, int row, int sb) {
+    RowSlot w;
+    if (row >= P.tiles * 16 || sb >= P.nsb) {  // past the padded rows, or past the last superblock
 #pragma unroll
-        for (int b = 0; b < 4; ++b) w.c[b] = make_uint2(0u, 0u);
-        w.s = make_uint2(0u, 0u);
+        for (int b = 0; b < 4; ++b) w.c[b] = make_uint4(0u, 0u, 0u, 0u);
+        w.s = make_uint4(0u, 0u, 0u, 0u);
         return w;
     }
-    const int sb = kt >> 1, hb = kt & 1;  // superblock, and which half of it (blocks 2hb, 2hb+1)
     const size_t slot = ((size_t)(row >> 4) * P.nsb + sb) * 16 + (row & 15);
-    const uint8_t *c = P.codes + slot * 64 + 8 * hb;
+    const uint8_t *c = P.codes + slot * 64;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) w.c[b] = p_ldg64(c + 16 * b);
-    w.s = p_ldg64(P.scales + slot * 16 + 8 * hb);
+    for (int b = 0; b < 4; ++b) w.c[b] = p_ldg128(c + 16 * b);
+    w.s = p_ldg128(P.scales + slot * 16);
+    return w;
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int j) {
+    return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+// One weight row's words of one 32-column block j.
+struct BlockWords {
+    uint32_t c[4];
+    uint32_t s;
+};
+
+__device__ __forceinline__ BlockWords block_of(const RowSlot &r, int j) {
+    BlockWords w;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) w.c[b] = word_of(r.c[b], j);
+    w.s = word_of(r.s, j);
     return w;
 }
 
 // 4x4 byte transpose: out[i] byte b = in[b] byte i.
-__device__ __forceinline__ void p_transpose4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t (&o)[4]) {
-    const uint32_t a = prmt(w0, w1, 0x5140u), b = prmt(w2, w3, 0x5140u);
-    const uint32_t c = prmt(w0, w1, 0x7362u), d = prmt(w2, w3, 0x7362u);
+__device__ __forceinline__ void p_transpose4(const uint32_t (&w)[4], uint32_t (&o)[4]) {
+    const uint32_t a = prmt(w[0], w[1], 0x5140u), b = prmt(w[2], w[3], 0x5140u);
+    const uint32_t c = prmt(w[0], w[1], 0x7362u), d = prmt(w[2], w[3], 0x7362u);
     o[0] = prmt(a, b, 0x5410u);
     o[1] = prmt(a, b, 0x7632u);
     o[2] = prmt(c, d, 0x5410u);
     o[3] = prmt(c, d, 0x7632u);
 }
 
-// Decode one row's 64 columns into the swizzled weight tile.  In a row's
-// 64-byte superblock slot, logical byte L of block j sits at chunk L % 4,
-// word j, byte L / 4; so for a fixed block the four chunks' words, byte-
+// Decode one row's 32-column block jj of the stage into the swizzled weight
+// tile.  In a row's 64-byte superblock slot, logical byte L of block j sits at
+// chunk L % 4, word j, byte L / 4; so the block's four chunk words, byte-
 // transposed, give logical words i = 0..3, each holding elements 8i .. 8i+7
-// (element 2L in the low nibble of byte L).  Logical word i of block jj lands
-// in 16-byte chunk 4 jj + i of the tile row, stored at chunk (4 jj + i) xor
-// (row % 8) (the 128-byte swizzle).
-__device__ __forceinline__ void decode_row(const RowWords &w, int row, uint32_t atile, uint32_t lut_lane) {
+// (element 2L in the low nibble of byte L).  Logical word i lands in 16-byte
+// chunk 4 jj + i of the tile row, stored at chunk (4 jj + i) xor (row % 8)
+// (the 128-byte swizzle).
+__device__ __forceinline__ void decode_block(const BlockWords &w, int row, int jj, uint32_t atile,
+                                             uint32_t lut_lane) {
     const uint32_t rbase = atile + (uint32_t)row * 128u;
+    uint32_t L[4];
+    p_transpose4(w.c, L);
+    const uint32_t d0 = prmt(w.s, w.s, 0x1010u), d1 = prmt(w.s, w.s, 0x3232u);  // (d, d) of each half
 #pragma unroll
-    for (int jj = 0; jj < 2; ++jj) {
-        uint32_t L[4];
-        if (jj == 0)
-            p_transpose4(w.c[0].x, w.c[1].x, w.c[2].x, w.c[3].x, L);
-        else
-            p_transpose4(w.c[0].y, w.c[1].y, w.c[2].y, w.c[3].y, L);
-        const uint32_t sw = jj == 0 ? w.s.x : w.s.y;  // (d0, d1) of the block
-        const uint32_t d0 = prmt(sw, sw, 0x1010u), d1 = prmt(sw, sw, 0x3232u);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t d = i < 2 ? d0 : d1;  // elements 0..15 take d0, 16..31 d1
-            const uint32_t o0 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7604u)), d);
-            const uint32_t o1 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7614u)), d);
-            const uint32_t o2 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7624u)), d);
-            const uint32_t o3 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7634u)), d);
-            const uint32_t chunk = (uint32_t)(4 * jj + i) ^ (uint32_t)(row & 7);
-            p_sts128(rbase + chunk * 16u, o0, o1, o2, o3);
-        }
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t d = i < 2 ? d0 : d1;  // elements 0..15 take d0, 16..31 d1
+        const uint32_t o0 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7604u)), d);
+        const uint32_t o1 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7614u)), d);
+        const uint32_t o2 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7624u)), d);
+        const uint32_t o3 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7634u)), d);
+        const uint32_t chunk = (uint32_t)(4 * jj + i) ^ (uint32_t)(row & 7);
+        p_sts128(rbase + chunk * 16u, o0, o1, o2, o3);
     }
 }
 
@@ -364,34 +381,51 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- weight tiles: decode ---------------------------------------------
-        const int row = (warp - 2) * 32 + lane;  // tile row of this thread
+        // ---- weight tiles: decode (thread = one row, one 32-column block) ---------
+        const int td = (warp - 2) * 32 + lane;
+        const int row = td & (kPM - 1), jj = td / kPM;
         const uint32_t lut_lane = kPLut | ((uint32_t)lane * 4u);
-        RowWords cur = load_row(P, n0 + row, 0);
-        for (int kt = 0; kt < P.nk; ++kt) {
-            const int s = kt % kPStages;
-            const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
-            RowWords nxt = cur;
-            if (kt + 1 < P.nk) nxt = load_row(P, n0 + row, kt + 1);  // one stage ahead
-            // (warp-uniform decision: the epilogue below runs warp-synchronous loads)
-            if (!__all_sync(kFull, p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns))) {
-                if (lane == 0) atomicOr(P.header, kPStatusTimeout);
-                break;
+        // row slots kAhead superblocks ahead, in a register ring (the loop is
+        // unrolled by kAhead so that every ring index is a constant)
+        RowSlot w[kAhead];
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) w[i] = load_slot(P, n0 + row, i);
+        const int nsb_stages = (P.nk + 1) / 2;  // superblocks touched by the stages
+        bool ok = true;
+        for (int sb0 = 0; sb0 < nsb_stages && ok; sb0 += kAhead) {
+#pragma unroll
+            for (int i = 0; i < kAhead; ++i) {
+                const int sb = sb0 + i;
+                if (sb >= nsb_stages || !ok) break;
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {  // the superblock's two stages
+                    const int kt = 2 * sb + hb;
+                    if (kt >= P.nk) break;
+                    const int s = kt % kPStages;
+                    const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
+                    // (warp-uniform decision: the epilogue below runs warp-synchronous loads)
+                    if (!__all_sync(kFull, p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns))) {
+                        if (lane == 0) atomicOr(P.header, kPStatusTimeout);
+                        ok = false;
+                        break;
+                    }
+                    decode_block(block_of(w[i], 2 * hb + jj), row, jj, a_tile(s), lut_lane);
+                    p_fence_proxy_async();
+                    p_mbar_arrive(full_a(s));
+                }
+                w[i] = load_slot(P, n0 + row, sb + kAhead);
             }
-            decode_row(cur, row, a_tile(s), lut_lane);
-            p_fence_proxy_async();
-            p_mbar_arrive(full_a(s));
-            cur = nxt;
         }
         // ---- epilogue: tensor memory -> Y ------------------------------------
         const int q = warp & 3;                 // this warp's quarter of the 128 lanes
         const int wrow = n0 + q * 32 + lane;    // weight row = accumulator lane
+        const int c0 = ((warp - 2) >> 2) * (kPN / 64);  // two warps per quarter: half of the columns each
         if (!__all_sync(kFull, p_mbar_wait(accum, 0u, P.timeout_ns))) {
             if (lane == 0) atomicOr(P.header, kPStatusTimeout);
         } else {
             p_tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < kPN / 32; ++c) {
+            for (int c = c0; c < c0 + kPN / 64; ++c) {
                 uint32_t v[32];
                 p_tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
                 if (wrow < P.n) {
