@@ -24,7 +24,10 @@ Reported:
              host memory, runs the path and reads the outputs back;
   roofline   for the phase with the largest share of the step, against the
              measured HBM copy bandwidth; rooflines for every phase;
-  cpu_baseline  the CPU oracle (single thread) on a bounded row sample.
+  cpu_baseline  the CPU oracle (single thread) on a bounded row sample;
+  prefill    the large-M tensor-core product on an 8192 x 8192 weight times
+             2048 activation rows: whole call and product alone, TFLOP/s
+             against the measured dense bf16 tensor peak.
 
 Multi-GPU (torchrun): every rank runs its own layer (independent problems,
 no collective on the data path, weak scaling); times are the max over ranks.
@@ -68,6 +71,7 @@ def parse_args(argv=None):
     p.add_argument("--skip-e2e", action="store_true")
     p.add_argument("--skip-codec-comparison", action="store_true",
                    help="skip the NVFP4 vs TQ4_1S comparison on the Llama-3-8B layer shapes")
+    p.add_argument("--skip-prefill", action="store_true", help="omit the large-M tensor-core product line")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     p.add_argument("--cpu-sample-rows", type=int, default=None,
                    help="rows per matrix for the CPU oracle sample (default: 1/8 of each matrix)")
@@ -495,6 +499,8 @@ def run_ours(args, world, rank, local):
 
     if not args.skip_e2e:
         line["e2e"] = run_e2e(tq, path, steps=min(steps, 5), world=world)
+    if args.workload == "llama3_8b_layer" and not args.skip_prefill:
+        line["prefill"] = prefill_measure(tq, rank, device, min(steps, 10), warmup, flush)
     if args.workload == "llama3_8b_layer" and not args.skip_codec_comparison:
         line["codec_comparison"] = codec_comparison(tq, path, rank, device, min(steps, 10), warmup, flush, use_graph,
                                                     world)
@@ -614,6 +620,75 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
         entry["packed_bytes"] = packed
         result[codec] = entry
     return result
+
+
+PREFILL_PROFILE = ("prefill_kernel_8192x8192_m2048.md", ("tq_device.cuh", "tq_prefill.cu"))
+
+
+def prefill_measure(tq, rank, device, steps, warmup, flush):
+    """The large-M product on its configured workload: an 8192 x 8192 weight
+    (bf16 ~N(0, 0.02^2)) times 2048 activation rows (bf16 ~N(0, 1)), bf16 out.
+    Times the whole call (plain pre-rotation + tensor-core product) and the
+    product alone over a pre-rotated activation; the product's TFLOP/s is set
+    against the measured dense bf16 tensor peak (fp16 operands run at the bf16
+    rate).  cuBLAS bf16 on the dense weight of the same shape is context.
+    Inputs total 74 MB (< L2), so L2 is flushed before every timed call."""
+    import hashlib
+
+    from dequant_gemv_tq4_b200 import inputs
+
+    n = k = 8192
+    m = 2048
+    W = inputs.gaussian_matrix(rank_seed(rank), 40, n, k, 0.02, torch.bfloat16, device)
+    X = inputs.gaussian_matrix(rank_seed(rank) + 1, 41, m, k, 1.0, torch.bfloat16, device)
+    codes, scales = tq.quantize(W)
+    ws = tq.prefill_workspace(m, k, device)
+    hdr = torch.zeros(256, dtype=torch.uint8, device=device)
+    xr = tq.prerotate_plain(X)
+    Y = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+    full = lambda: tq.gemm_prefill(codes, scales, n, k, X, out=Y, ws=ws)
+    prod = lambda: tq.gemm_prefill_xrot(codes, scales, n, k, xr, out=Y, ws=hdr)
+    dense = lambda: torch.matmul(X, W.t(), out=Y)
+    res = {}
+    for name, fn in (("call", full), ("product", prod), ("cublas_bf16_dense", dense)):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        res[name] = time_replays(fn, steps, flush) / steps
+    st = tq.workspace_status(ws) or tq.workspace_status(hdr)
+    flops = 2.0 * m * n * k
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+        peak, kind = float(peaks["bf16_tflops"]), "measured"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    ach = flops / (res["product"] * 1e-3) / 1e12
+    traffic = None
+    try:
+        text = open(os.path.join(ROOT, "profiles", PREFILL_PROFILE[0])).read()
+        fields = dict(ln.split(": ", 1) for ln in text.splitlines() if ": " in ln)
+        h = hashlib.sha256()
+        for src in PREFILL_PROFILE[1]:
+            with open(os.path.join(ROOT, "dequant_gemv_tq4_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] == fields["source_sha256"].strip():
+            traffic = int(fields["traffic_bytes_per_launch"])
+    except Exception:
+        traffic = None
+    return {
+        "workload": "8192x8192 TQ4_1S weight (bf16 source ~N(0,0.02^2)) x 2048 bf16 activation rows ~N(0,1), bf16 out",
+        "ms_call": round(res["call"], 5), "tflops_call": round(flops / (res["call"] * 1e-3) / 1e12, 1),
+        "ms_product": round(res["product"], 5),
+        "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(ach / peak, 4), "traffic": traffic, "kernel": "prefill_kernel",
+                     "peak_note": f"{kind} dense bf16 burst (fp16 operands, same nominal rate)",
+                     "algorithmic": "2*m*n*k flops per launch"},
+        "cublas_bf16_dense_ms": round(res["cublas_bf16_dense"], 5),
+        "cublas_bf16_dense_tflops": round(flops / (res["cublas_bf16_dense"] * 1e-3) / 1e12, 1),
+        "status": int(st), "l2": "flushed (256 MB write) before every timed call",
+    }
 
 
 def run_e2e(tq, path, steps, world):

@@ -87,6 +87,9 @@ def load_library() -> ctypes.CDLL:
             "tq_gemv_static_scratch": ([P, P, I64, I64, P, I, P, I, P], I),
             "tq_gemm_prefill_workspace_bytes": ([I64, I64], SZ),
             "tq_gemm_prefill": ([P, P, I64, I64, P, I, I64, I64, P, I, I64, P, SZ, P], I),
+            "tq_prefill_xrot_bytes": ([I64, I64], SZ),
+            "tq_prerotate_plain": ([P, I, I64, I64, I64, P, P], I),
+            "tq_gemm_prefill_xrot": ([P, P, I64, I64, P, I64, P, I, I64, P, SZ, P], I),
             "tq_nvfp4_scales_bytes": ([I64, I64], SZ),
             "tq_nvfp4_quantize": ([P, I, I64, I64, I64, P, P, P, P], I),
             "tq_nvfp4_dequantize": ([P, P, P, I64, I64, P, I, I64, P], I),
@@ -179,6 +182,18 @@ def tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream) -> int:
 
 def tq_gemm_prefill_workspace_bytes(m: int, k: int) -> int:
     return int(load_library().tq_gemm_prefill_workspace_bytes(m, k))
+
+
+def tq_prefill_xrot_bytes(m: int, k: int) -> int:
+    return int(load_library().tq_prefill_xrot_bytes(m, k))
+
+
+def tq_prerotate_plain(X, xt, m, k, ldx, xrot, stream) -> int:
+    return load_library().tq_prerotate_plain(X, xt, m, k, ldx, xrot, stream)
+
+
+def tq_gemm_prefill_xrot(codes, scales, n, k, xrot, m, Y, yt, ldy, workspace, ws_bytes, stream) -> int:
+    return load_library().tq_gemm_prefill_xrot(codes, scales, n, k, xrot, m, Y, yt, ldy, workspace, ws_bytes, stream)
 
 
 def tq_gemm_prefill(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream) -> int:
@@ -315,6 +330,31 @@ def gemm_prefill(codes, scales, n: int, k: int, X: torch.Tensor, dtype=torch.flo
     _check(tq_gemm_prefill(codes.data_ptr(), scales.data_ptr(), n, k, X2.data_ptr(), _dt(X2.dtype), m, _ld(X2),
                            out.data_ptr(), _dt(out.dtype), _ld(out), ws.data_ptr(), ws.numel(), _stream(stream)),
            "tq_gemm_prefill")
+    return out
+
+
+def prerotate_plain(X: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """Plain row-major fp16 pre-rotation of X (m x k) for the prefill product."""
+    X2 = X.view(1, -1) if X.dim() == 1 else X
+    m, k = X2.shape
+    if out is None:
+        out = torch.empty((m, k), dtype=torch.float16, device=X.device)
+    _check(tq_prerotate_plain(X2.data_ptr(), _dt(X2.dtype), m, k, _ld(X2), out.data_ptr(), _stream(stream)),
+           "tq_prerotate_plain")
+    return out
+
+
+def gemm_prefill_xrot(codes, scales, n: int, k: int, xrot: torch.Tensor, dtype=torch.float32, out=None, ws=None,
+                      stream=None) -> torch.Tensor:
+    """The tensor-core product over an activation from ``prerotate_plain``."""
+    m = xrot.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=dtype, device=xrot.device)
+    if ws is None:
+        ws = torch.zeros(256, dtype=torch.uint8, device=xrot.device)
+    _check(tq_gemm_prefill_xrot(codes.data_ptr(), scales.data_ptr(), n, k, xrot.data_ptr(), m, out.data_ptr(),
+                                _dt(out.dtype), _ld(out), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "tq_gemm_prefill_xrot")
     return out
 
 

@@ -274,6 +274,41 @@ tq_status tq_gemm_prefill(const uint8_t *codes, const uint16_t *scales, int64_t 
     return run_prefill(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream);
 }
 
+size_t tq_prefill_xrot_bytes(int64_t m, int64_t k) {
+    if (m < 0 || check_nk(0, k) != TQ_OK) return 0;
+    return (size_t)m * (size_t)k * 2u;
+}
+
+tq_status tq_prerotate_plain(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
+                             void *stream) {
+    tq_status st = check_nk(m, k);
+    if (st != TQ_OK) return st;
+    if (!valid_dtype(xt)) return TQ_ERR_DTYPE;
+    if (m == 0) return TQ_OK;
+    if (m > TQ_MAX_N) return TQ_ERR_SHAPE;
+    if ((st = check_matrix_operand(X, ldx, k)) != TQ_OK) return st;
+    if (!xrot) return TQ_ERR_INVALID_ARG;
+    if (!aligned(xrot, 16)) return TQ_ERR_ALIGNMENT;
+    return from_cuda(tq::launch_prerotate_plain(X, xt, m, k, ldx, xrot, nullptr, (cudaStream_t)stream));
+}
+
+tq_status tq_gemm_prefill_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
+                               const uint16_t *xrot, int64_t m, void *Y, tq_dtype yt, int64_t ldy, void *workspace,
+                               size_t ws_bytes, void *stream) {
+    tq_status st = check_gemm_common(codes, scales, n, k, m, Y, yt, ldy);
+    if (st != TQ_OK || n == 0 || m == 0) return st;
+    if (!xrot) return TQ_ERR_INVALID_ARG;
+    if (!aligned(xrot, 16)) return TQ_ERR_ALIGNMENT;
+    if ((m + 255) / 256 > 65535) return TQ_ERR_SHAPE;
+    if ((st = check_workspace(workspace, ws_bytes, kStatusBytes)) != TQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned *header = static_cast<unsigned *>(workspace);
+    if (tq::launch_prepare_header(header, s) != cudaSuccess) return TQ_ERR_CUDA;
+    const cudaError_t e = tq::launch_prefill_product(codes, scales, n, k, xrot, m, Y, yt, ldy, header, s);
+    if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
 // ---- batch: several matrices, one pre-rotation per distinct input ----------
 static tq_status batch_layout(const tq_gemm_desc *descs, int count, int64_t m, Layout *lay, int *input_of) {
     int64_t n[tq::kMaxProblems], k[tq::kMaxProblems], ik[tq::kMaxInputs];

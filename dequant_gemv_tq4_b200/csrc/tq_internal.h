@@ -108,6 +108,14 @@ size_t prefill_xrot_bytes(int64_t m, int64_t k);
 cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
                            int xdtype, int64_t m, int64_t ldx, uint16_t *xrot, void *y, int ydtype, int64_t ldy,
                            unsigned *header, cudaStream_t stream);
+// The two steps of launch_prefill on their own: the plain pre-rotation (header
+// may be null; otherwise it clears the status word and advances the call tag)
+// and the product over an xrot it wrote.
+cudaError_t launch_prerotate_plain(const void *X, int xdtype, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
+                                   unsigned *header, cudaStream_t stream);
+cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
+                                   const uint16_t *xrot, int64_t m, void *y, int ydtype, int64_t ldy,
+                                   unsigned *header, cudaStream_t stream);
 
 // ---- NVFP4 comparison codec ---------------------------------------------------
 // Same fused product over NVFP4 planes (E2M1 codes in the TQ4_1S unit layout,

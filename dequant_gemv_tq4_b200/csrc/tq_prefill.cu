@@ -573,36 +573,37 @@ cudaError_t launch_plain_rotation(const PlainRotParams &r, cudaStream_t stream) 
 
 size_t prefill_xrot_bytes(int64_t m, int64_t k) { return round_up((size_t)m * (size_t)k * 2u, 256); }
 
-cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
-                           int xdtype, int64_t m, int64_t ldx, uint16_t *xrot, void *y, int ydtype, int64_t ldy,
-                           unsigned *header, cudaStream_t stream) {
+cudaError_t launch_prerotate_plain(const void *X, int xdtype, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
+                                   unsigned *header, cudaStream_t stream) {
+    if (m < 1 || k < 32 || k % 32 != 0) return cudaErrorInvalidValue;
+    PlainRotParams r = {static_cast<const char *>(X), ldx, xrot, m, (int)k, (int)superblocks(k), header};
+    switch (xdtype) {
+        case kF32: return launch_plain_rotation<kF32>(r, stream);
+        case kBF16: return launch_plain_rotation<kBF16>(r, stream);
+        case kF16: return launch_plain_rotation<kF16>(r, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
+                                   const uint16_t *xrot, int64_t m, void *y, int ydtype, int64_t ldy,
+                                   unsigned *header, cudaStream_t stream) {
     if (n < 1 || m < 1 || k < 32 || k % 32 != 0) return cudaErrorInvalidValue;
     const int64_t grid_y = (m + kPN - 1) / kPN, grid_x = (n + kPM - 1) / kPM;
     if (grid_y > 65535 || grid_x > 0x7fffffff) return cudaErrorInvalidValue;
     EncodeTiled encode = encode_tiled();
     if (!encode) return cudaErrorNotSupported;
-    // 1. X -> plain fp16 pre-rotation (clears the status word)
-    PlainRotParams r = {static_cast<const char *>(X), ldx, xrot, m, (int)k, (int)superblocks(k), header};
-    cudaError_t err;
-    switch (xdtype) {
-        case kF32: err = launch_plain_rotation<kF32>(r, stream); break;
-        case kBF16: err = launch_plain_rotation<kBF16>(r, stream); break;
-        case kF16: err = launch_plain_rotation<kF16>(r, stream); break;
-        default: return cudaErrorInvalidValue;
-    }
-    if (err != cudaSuccess) return err;
-    // 2. the tensor map of xrot: k x m fp16, rows of k*2 bytes, boxes of
-    //    64 columns x 256 rows, 128-byte swizzle, zero fill outside
+    // the tensor map of xrot: k x m fp16, rows of k*2 bytes, boxes of
+    // 64 columns x 256 rows, 128-byte swizzle, zero fill outside
     CUtensorMap map;
     const cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
     const cuuint64_t strides[1] = {(cuuint64_t)k * 2u};
     const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)kPN};
     const cuuint32_t estr[2] = {1u, 1u};
-    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xrot, dims, strides, box, estr,
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(xrot), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    // 3. the product
     PrefillParams prm;
     prm.codes = codes;
     prm.scales = reinterpret_cast<const uint8_t *>(scales);
@@ -625,6 +626,19 @@ cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t
         case kF16: return launch_prefill_kernel<kF16>(map, prm, grid, smem, stream);
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
+                           int xdtype, int64_t m, int64_t ldx, uint16_t *xrot, void *y, int ydtype, int64_t ldy,
+                           unsigned *header, cudaStream_t stream) {
+    if (n < 1 || m < 1 || k < 32 || k % 32 != 0) return cudaErrorInvalidValue;
+    if ((m + kPN - 1) / kPN > 65535) return cudaErrorInvalidValue;
+    if (!encode_tiled()) return cudaErrorNotSupported;
+    // 1. X -> plain fp16 pre-rotation (clears the status word)
+    cudaError_t err = launch_prerotate_plain(X, xdtype, m, k, ldx, xrot, header, stream);
+    if (err != cudaSuccess) return err;
+    // 2. the product
+    return launch_prefill_product(codes, scales, n, k, xrot, m, y, ydtype, ldy, header, stream);
 }
 
 }  // namespace tq

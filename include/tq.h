@@ -199,6 +199,32 @@ TQ_API tq_status tq_gemm_prefill(const uint8_t *codes, const uint16_t *scales, i
                                  void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * The two steps of tq_gemm_prefill as separate calls, so that one rotated
+ * activation serves every matrix that consumes it (e.g. q/k/v in a prefill;
+ * TQ page, paragraph 适用前提与边界, the attention tensors share one rotation).
+ *
+ * tq_prefill_xrot_bytes -- m * k * 2: the plain pre-rotated activation, a
+ * row-major m x k fp16 matrix, element [i][c] = fp16(H(s .* x_i)/32) at
+ * column c (blocks of 32 along k, in order).
+ *
+ * tq_prerotate_plain -- writes that matrix for the m rows of X.
+ *   X     device, m x k of dtype xt, row stride ldx (as tq_prerotate)
+ *   xrot  device, tq_prefill_xrot_bytes(m, k) bytes, 16-byte aligned
+ *         (written; read by tensor-memory-accelerator copies afterwards)
+ *
+ * tq_gemm_prefill_xrot -- the tensor-core product of tq_gemm_prefill over an
+ * xrot written by tq_prerotate_plain (same m and k).  The workspace needs
+ * only its 256-byte header (>= 256 bytes, 256-byte aligned); a one-thread
+ * launch clears its status word first.  Y, yt, ldy as tq_gemm.
+ */
+TQ_API size_t tq_prefill_xrot_bytes(int64_t m, int64_t k);
+TQ_API tq_status tq_prerotate_plain(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
+                                    void *stream);
+TQ_API tq_status tq_gemm_prefill_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
+                                      const uint16_t *xrot, int64_t m, void *Y, tq_dtype yt, int64_t ldy,
+                                      void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * tq_gemm_xrot -- the product with an activation already pre-rotated by
  * tq_prerotate (one xrot shared by every matrix that consumes the same
  * input, e.g. q/k/v).  m <= 32.  Same workspace rules as tq_gemm (a

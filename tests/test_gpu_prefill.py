@@ -137,3 +137,56 @@ def test_prefill_full_size_sampled(cuda_lib):
     # per activation row over the sampled outputs, and per sampled output over all rows
     assert _rel_l2(got, Y_ref).max() <= REL_L2_TOL
     assert _rel_l2(got.T, Y_ref.T).max() <= REL_L2_TOL
+
+
+@pytest.mark.parametrize("m,k", [(1, 32), (3, 160), (2, 4096)])
+def test_prerotate_plain_values(cuda_lib, m, k):
+    """Row-major fp16 H(s .* x)/32 per 32-block, within one fp16 ulp of the
+    fp64 rotation."""
+    X = _w(m, k, BF16, seed=69, std=1.0)
+    xr = cuda_lib.prerotate_plain(X.to(DEV))
+    torch.cuda.synchronize()
+    assert xr.dtype == F16 and tuple(xr.shape) == (m, k)
+    got = xr.cpu().numpy().astype(np.float64)
+    s = oracle.sign(np.arange(k)).astype(np.float64)
+    ref = (oracle.fwht32((_host_f32(X).astype(np.float64) * s).reshape(m, k // 32, 32)) / 32).reshape(m, k)
+    ulp = np.spacing(np.abs(ref.astype(np.float16))).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= ulp + 1e-12)
+
+
+def test_prefill_xrot_shared_by_three_matrices(cuda_lib):
+    """One plain pre-rotation serves three weight matrices of different n
+    (q/k/v-like); each product equals tq_gemm_prefill's bit for bit."""
+    m, k = 300, 512
+    X = _w(m, k, BF16, seed=70, std=1.0).to(DEV)
+    xr = cuda_lib.prerotate_plain(X)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    for i, n in enumerate((256, 64, 130)):
+        W = _w(n, k, BF16, seed=71 + i)
+        codes, scales = cuda_lib.quantize(W.to(DEV))
+        a = cuda_lib.gemm_prefill_xrot(codes, scales, n, k, xr, ws=ws)
+        b = cuda_lib.gemm_prefill(codes, scales, n, k, X)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b)
+        assert cuda_lib.workspace_status(ws) == 0
+        c_ref, s_ref = oracle.quantize(_host_f32(W))
+        Y_ref = oracle.gemm(c_ref, s_ref, n, k, _host_f32(X))
+        assert _rel_l2(a.cpu().numpy(), Y_ref).max() <= REL_L2_TOL
+
+
+def test_prefill_xrot_argument_errors(cuda_lib):
+    m, n, k = 64, 32, 128
+    codes, scales = cuda_lib.quantize(_w(n, k, BF16).to(DEV))
+    xr = torch.zeros((m * k + 8,), dtype=F16, device=DEV)
+    Y = torch.zeros((m, n), dtype=F32, device=DEV)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert cuda_lib.tq_prefill_xrot_bytes(m, k) == m * k * 2
+    call = lambda x, nbytes: cuda_lib.tq_gemm_prefill_xrot(codes.data_ptr(), scales.data_ptr(), n, k, x, m,
+                                                            Y.data_ptr(), 0, n, ws.data_ptr(), nbytes, stream)
+    assert call(xr.data_ptr(), 255) == 5          # TQ_ERR_WORKSPACE
+    assert call(xr.data_ptr() + 2, 256) == 3      # TQ_ERR_ALIGNMENT (xrot not 16-byte aligned)
+    assert call(0, 256) == 1                      # TQ_ERR_INVALID_ARG
+    assert call(xr.data_ptr(), 256) == 0
+    torch.cuda.synchronize()
+    assert cuda_lib.workspace_status(ws) == 0
