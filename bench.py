@@ -74,7 +74,7 @@ def parse_args(argv=None):
     p.add_argument("--skip-prefill", action="store_true", help="omit the large-M tensor-core product line")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     p.add_argument("--cpu-sample-rows", type=int, default=None,
-                   help="rows per matrix for the CPU oracle sample (default: 1/8 of each matrix)")
+                   help="rows per matrix for the CPU oracle sample (default: half of each matrix)")
     return p.parse_args(argv)
 
 
@@ -366,7 +366,7 @@ def cpu_oracle_sample(path, rows_per_matrix=None):
     weights = packed = 0
     for it in path.items:
         n, k = it["n"], it["k"]
-        r = rows_per_matrix if rows_per_matrix else max(1, n // 8)
+        r = min(n, rows_per_matrix) if rows_per_matrix else max(1, n // 2)
         W = it["W"][:r].float().cpu().numpy()
         x = it["x"].float().cpu().numpy().reshape(1, -1).astype(np.float64)
         t0 = time.perf_counter()
@@ -383,7 +383,7 @@ def cpu_oracle_sample(path, rows_per_matrix=None):
         packed += c.nbytes + s.nbytes
     return {"gemv_gbs": packed / tg / 1e9, "quantize_gweights_per_s": weights / tq_w / 1e9,
             "dequantize_gweights_per_s": weights / td / 1e9, "seconds": tq_w + td + tg,
-            "sample": f"first {rows_per_matrix or '1/8 of the'} rows of each of the {len(path.items)} matrices "
+            "sample": f"first {rows_per_matrix or 'half of the'} rows of each of the {len(path.items)} matrices "
                       f"({weights / 1e6:.1f} M weights): quantise, dequantise, GEMV"}
 
 
