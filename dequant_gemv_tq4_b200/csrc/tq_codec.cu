@@ -43,14 +43,41 @@ __device__ __forceinline__ size_t unit_row(int row, int sb, int nsb) {
     return ((size_t)(row >> 4) * nsb + sb) * 16 + (row & 15);
 }
 
-// #{j : a > t_j} for ascending t (binary search over the seven thresholds).
-__device__ __forceinline__ uint32_t magnitude_rank(float a, const float (&t)[7]) {
-    const bool b2 = a > t[3];
-    const float tm = b2 ? t[5] : t[1];
-    const bool b1 = a > tm;
-    const float tl = b2 ? (b1 ? t[6] : t[4]) : (b1 ? t[2] : t[0]);
-    const bool b0 = a > tl;
-    return (b2 ? 4u : 0u) | (b1 ? 2u : 0u) | (b0 ? 1u : 0u);
+// Compare to an all-ones / all-zeros mask (no predicate register).
+__device__ __forceinline__ uint32_t mask_gt(float a, float b) {
+    uint32_t r;
+    asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t mask_lt(float a, float b) {
+    uint32_t r;
+    asm("set.lt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// m ? x : y on the bits (m all ones or all zeros).
+__device__ __forceinline__ float mask_pick(uint32_t m, float x, float y) {
+    return __uint_as_float((m & __float_as_uint(x)) | (~m & __float_as_uint(y)));
+}
+
+// Code of one rotated value y against the ascending thresholds t of its half,
+// added into `word` at nibble position `sh`: bit 3 = [y < 0], bits 0..2 =
+// #{j : |y| > t_j} by a three-compare binary search.  The compares give masks
+// (0 or 0xffffffff), the next threshold is a bitwise pick, and each bit enters
+// the word as mask * (-bit): an integer multiply-add (the ALU pipe keeps only
+// the compares and picks).
+__device__ __forceinline__ uint32_t add_code(uint32_t word, float y, const float (&t)[7], int sh) {
+    const float a = fabsf(y);
+    const uint32_t m2 = mask_gt(a, t[3]);
+    const uint32_t m1 = mask_gt(a, mask_pick(m2, t[5], t[1]));
+    const float tl = mask_pick(m2, mask_pick(m1, t[6], t[4]), mask_pick(m1, t[2], t[0]));
+    const uint32_t m0 = mask_gt(a, tl);
+    const uint32_t ms = mask_lt(y, 0.0f);
+    word = m2 * (0u - (4u << sh)) + word;
+    word = m1 * (0u - (2u << sh)) + word;
+    word = m0 * (0u - (1u << sh)) + word;
+    return ms * (0u - (8u << sh)) + word;
 }
 
 // -------------------------------------------------------------------------
@@ -207,10 +234,7 @@ __global__ void __launch_bounds__(kCodecThreads) quantize_kernel(const char *__r
 #pragma unroll
             for (int i = 0; i < 7; ++i) t[i] = __fmul_rn(thr[i], D[h]);
 #pragma unroll
-            for (int e = 16 * h; e < 16 * h + 16; ++e) {
-                const uint32_t code = (v[e] < 0.0f ? 8u : 0u) | magnitude_rank(fabsf(v[e]), t);
-                lw[e >> 3] |= code << (4 * (e & 7));
-            }
+            for (int e = 16 * h; e < 16 * h + 16; ++e) lw[e >> 3] = add_code(lw[e >> 3], v[e], t, 4 * (e & 7));
         }
         if (exists) {
             uint32_t sw[4];
@@ -370,10 +394,11 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     in.xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
 }
 
-int rows_grid(int64_t n, int64_t segs, int sm_count) {
-    // aim for ~4 resident CTAs (32 warps) per SM in total
-    int64_t target = (int64_t)sm_count * 4;
-    int64_t gy = (target + segs - 1) / segs;
+// Row groups per column segment: one wave of the CTAs that fit on the GPU at
+// once (`per_sm` resident per SM), each striding the rows.
+int rows_grid(int64_t n, int64_t segs, int sm_count, int per_sm) {
+    int64_t target = (int64_t)sm_count * (per_sm > 0 ? per_sm : 1);
+    int64_t gy = target / segs;
     int64_t max_gy = (((n + 15) & ~(int64_t)15) + kCodecWarps - 1) / kCodecWarps;
     if (gy > max_gy) gy = max_gy;
     if (gy > 65535) gy = 65535;
@@ -383,6 +408,30 @@ int rows_grid(int64_t n, int64_t segs, int sm_count) {
 
 }  // namespace
 
+// Resident CTAs per SM of a kernel (queried once per kernel).
+template <typename K>
+int resident_per_sm(K kernel, int *cache) {
+    if (*cache <= 0) {
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, kCodecThreads, 0) != cudaSuccess || nb < 1)
+            nb = 1;
+        *cache = nb;
+    }
+    return *cache;
+}
+
+template <int DT>
+int quantize_per_sm() {
+    static int cache = 0;
+    return resident_per_sm(quantize_kernel<DT>, &cache);
+}
+
+template <int DT>
+int dequantize_per_sm() {
+    static int cache = 0;
+    return resident_per_sm(dequantize_kernel<DT>, &cache);
+}
+
 cudaError_t launch_quantize(const void *w, int dtype, int64_t n, int64_t k, int64_t ldw, uint8_t *codes,
                             uint16_t *scales, cudaStream_t stream) {
     DeviceInfo di;
@@ -390,7 +439,9 @@ cudaError_t launch_quantize(const void *w, int dtype, int64_t n, int64_t k, int6
     if (err != cudaSuccess) return err;
     const int64_t nb = k / 32, nsb = superblocks(k);
     const int64_t segs = (nsb * kSbBlocks + 31) / 32;
-    dim3 grid((unsigned)segs, (unsigned)rows_grid(n, segs, di.sm_count));
+    const int per_sm = dtype == kF32 ? quantize_per_sm<kF32>() : dtype == kBF16 ? quantize_per_sm<kBF16>()
+                                                                                 : quantize_per_sm<kF16>();
+    dim3 grid((unsigned)segs, (unsigned)rows_grid(n, segs, di.sm_count, per_sm));
     auto *c = reinterpret_cast<uint32_t *>(codes);
     auto *s = reinterpret_cast<uint32_t *>(scales);
     const char *wp = static_cast<const char *>(w);
@@ -410,7 +461,9 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int6
     if (err != cudaSuccess) return err;
     const int64_t nb = k / 32, nsb = superblocks(k);
     const int64_t segs = (nb + 31) / 32;
-    dim3 grid((unsigned)segs, (unsigned)rows_grid(n, segs, di.sm_count));
+    const int per_sm = dtype == kF32 ? dequantize_per_sm<kF32>() : dtype == kBF16 ? dequantize_per_sm<kBF16>()
+                                                                                   : dequantize_per_sm<kF16>();
+    dim3 grid((unsigned)segs, (unsigned)rows_grid(n, segs, di.sm_count, per_sm));
     auto *c = reinterpret_cast<const uint32_t *>(codes);
     auto *s = reinterpret_cast<const uint32_t *>(scales);
     char *o = static_cast<char *>(w_out);
