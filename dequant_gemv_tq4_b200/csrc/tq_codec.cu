@@ -43,41 +43,21 @@ __device__ __forceinline__ size_t unit_row(int row, int sb, int nsb) {
     return ((size_t)(row >> 4) * nsb + sb) * 16 + (row & 15);
 }
 
-// Compare to an all-ones / all-zeros mask (no predicate register).
-__device__ __forceinline__ uint32_t mask_gt(float a, float b) {
-    uint32_t r;
-    asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t mask_lt(float a, float b) {
-    uint32_t r;
-    asm("set.lt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
-    return r;
-}
-
-// m ? x : y on the bits (m all ones or all zeros).
-__device__ __forceinline__ float mask_pick(uint32_t m, float x, float y) {
-    return __uint_as_float((m & __float_as_uint(x)) | (~m & __float_as_uint(y)));
-}
-
 // Code of one rotated value y against the ascending thresholds t of its half,
 // added into `word` at nibble position `sh`: bit 3 = [y < 0], bits 0..2 =
-// #{j : |y| > t_j} by a three-compare binary search.  The compares give masks
-// (0 or 0xffffffff), the next threshold is a bitwise pick, and each bit enters
-// the word as mask * (-bit): an integer multiply-add (the ALU pipe keeps only
-// the compares and picks).
+// #{j : |y| > t_j} by a three-compare binary search.  Each bit is a
+// conditional add consumed right after its compare, so the compiler can
+// predicate the adds instead of materialising (or spilling) the predicates.
 __device__ __forceinline__ uint32_t add_code(uint32_t word, float y, const float (&t)[7], int sh) {
     const float a = fabsf(y);
-    const uint32_t m2 = mask_gt(a, t[3]);
-    const uint32_t m1 = mask_gt(a, mask_pick(m2, t[5], t[1]));
-    const float tl = mask_pick(m2, mask_pick(m1, t[6], t[4]), mask_pick(m1, t[2], t[0]));
-    const uint32_t m0 = mask_gt(a, tl);
-    const uint32_t ms = mask_lt(y, 0.0f);
-    word = m2 * (0u - (4u << sh)) + word;
-    word = m1 * (0u - (2u << sh)) + word;
-    word = m0 * (0u - (1u << sh)) + word;
-    return ms * (0u - (8u << sh)) + word;
+    const bool b2 = a > t[3];
+    const bool b1 = a > (b2 ? t[5] : t[1]);
+    const bool b0 = a > (b1 ? (b2 ? t[6] : t[2]) : (b2 ? t[4] : t[0]));
+    if (b2) word += 4u << sh;
+    if (b1) word += 2u << sh;
+    if (b0) word += 1u << sh;
+    if (y < 0.0f) word += 8u << sh;
+    return word;
 }
 
 // -------------------------------------------------------------------------
