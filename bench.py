@@ -27,7 +27,9 @@ Reported:
   cpu_baseline  the CPU oracle (single thread) on a bounded row sample;
   prefill    the large-M tensor-core product on an 8192 x 8192 weight times
              2048 activation rows: whole call and product alone, TFLOP/s
-             against the measured dense bf16 tensor peak.
+             against the measured dense bf16 tensor peak;
+  codec_comparison  NVFP4 next to TQ4_1S on the layer, and the TQ4_1S
+             skinny sweep (1, 2, 4, 8, 16, 32 activation rows).
 
 Multi-GPU (torchrun): every rank runs its own layer (independent problems,
 no collective on the data path, weak scaling); times are the max over ranks.
@@ -517,16 +519,17 @@ def run_ours(args, world, rank, local):
 def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, world):
     """NVFP4 next to TQ4_1S on the same layer: reconstruction rel-L2 over the
     layer, quantise Gweights/s and fused-product GB/s at M = 1 and M = 16
+    (TQ4_1S also at M = 2, 4, 8 and 32: the skinny sweep)
     (steady state, passes alternating with a shadow layer as for the main
     metric).  GB/s counts each codec's own packed bytes."""
     from dequant_gemv_tq4_b200 import inputs
 
     R = 10
     smats, _, _ = make_workload("llama3_8b_layer", rank + 1000, device)
-    x16 = {}
+    x32 = {}
     for aid, act in enumerate(("attn", "attn_out", "ffn", "ffn_mid")):
         k = 14336 if act == "ffn_mid" else 4096
-        x16[act] = inputs.gaussian_matrix(1, 300 + aid, 16, k, 1.0, torch.bfloat16, device)
+        x32[act] = inputs.gaussian_matrix(1, 300 + aid, 32, k, 1.0, torch.bfloat16, device)
     act_of = inputs.LLAMA3_8B_INPUTS
 
     def nv_pack(mats):
@@ -541,7 +544,7 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
         out = []
         for (c, s), (label, W, _) in zip(packs, mats):
             n, k = W.shape
-            X = x16[act_of[label]][:m]
+            X = x32[act_of[label]][:m]
             out.append((c, s, n, k, X, torch.empty((m, n), dtype=torch.float32, device=device)))
         return out
 
@@ -549,7 +552,7 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
         out = []
         for (c, s, t), (label, W, _) in zip(packs, mats):
             n, k = W.shape
-            X = x16[act_of[label]][:m]
+            X = x32[act_of[label]][:m]
             out.append((c, s, t, n, k, X, torch.empty((m, n), dtype=torch.float32, device=device)))
         return out
 
@@ -569,7 +572,8 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
         else:
             packed = sum(c.numel() + s.numel() + t.numel() * 4 for c, s, t in nv_layer)
             entry["bits_per_weight"] = 4.5
-        for m in (1, 16):
+        # the skinny sweep (1..32 activation rows) for TQ4_1S, m = 1 and 16 for NVFP4
+        for m in ((1, 2, 4, 8, 16, 32) if codec == "tq4_1s" else (1, 16)):
             if codec == "tq4_1s":
                 a, b = items_tq(tq_layer, layer_mats, m), items_tq(tq_shadow, smats, m)
                 da, db = tq.batch_descs(a), tq.batch_descs(b)
@@ -590,6 +594,7 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
             (ms,) = max_over_ranks([ms], world)
             entry[f"gemm_m{m}_us"] = round(1e3 * ms, 2)
             entry[f"gemm_m{m}_gbs"] = round(job_gbs(packed, world, ms), 1)
+            entry[f"gemm_m{m}_tflops"] = round(2.0 * m * path.weights() * world / (ms * 1e-3) / 1e12, 2)
         if codec == "tq4_1s":
             qfn = path.quantize
         else:
