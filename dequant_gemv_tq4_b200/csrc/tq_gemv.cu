@@ -52,9 +52,9 @@ namespace tq {
 namespace {
 
 // Warps per CTA: one-row products keep few registers live and take 20 warps;
-// the multi-row kernels (more accumulators) take 16 so that they fit 128
-// registers per thread without spilling.
-__host__ __device__ constexpr int warps_for(bool one_row) { return one_row ? 20 : 16; }
+// up to 16 rows take 16 (128 registers per thread); 17..32 rows take 12, whose
+// three or four accumulator tiles need up to 168 registers without spilling.
+__host__ __device__ constexpr int warps_for(bool one_row, int nt = 1) { return one_row ? 20 : (nt >= 3 ? 12 : 16); }
 constexpr int kStages = 2;  // ring stages per warp
 constexpr int kPerStage = 2;  // consecutive units per stage
 constexpr int kUnitCodeBytes = 1024;
@@ -634,8 +634,8 @@ __device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0,
 }
 
 template <int NT, bool M1, int OT, int CODEC>
-__global__ void __launch_bounds__(warps_for(M1) * 32, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
-    using G = Geometry<warps_for(M1)>;
+__global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
+    using G = Geometry<warps_for(M1, NT)>;
     using CT = CodecTraits<CODEC>;
     constexpr int SB = CT::kScaleBytes;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -810,7 +810,7 @@ uint32_t dynamic_smem_base() {
 
 template <int NT, bool M1, int CODEC>
 cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programmatic, cudaStream_t stream) {
-    using G = Geometry<warps_for(M1)>;
+    using G = Geometry<warps_for(M1, NT)>;
     const uint32_t smem = G::smem_bytes_for_base(dynamic_smem_base());
     const int kSmemBytes = (int)smem;
     cudaLaunchConfig_t cfg = {};
@@ -856,7 +856,7 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
         pl.units += tiles(n[i]) * superblocks(k[i]);
     }
     // one activation row runs the one-row kernel (see launch_group_codec)
-    const int kWarps = warps_for(m == 1);
+    const int kWarps = warps_for(m == 1, (int)((m > 32 ? 32 : (m < 1 ? 1 : m)) + 7) / 8);
     int64_t want = (pl.units + kWarps - 1) / kWarps;  // at least one unit per warp
     if (want > sm_count) want = sm_count;
     if (want < 1) want = 1;
@@ -905,7 +905,7 @@ cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, i
     const int nt = plan.mcap / 8;
     const bool one_row = m == 1 && nt == 1;
     // the plan's warps must all exist in the launched grid
-    if (plan.total_warps > (int64_t)plan.grid * warps_for(one_row)) return cudaErrorInvalidValue;
+    if (plan.total_warps > (int64_t)plan.grid * warps_for(one_row, nt)) return cudaErrorInvalidValue;
     if (one_row) return launch_nt<1, true, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
     switch (nt) {
         case 1: return launch_nt<1, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
