@@ -148,7 +148,7 @@ def test_prerotate_values_and_layout(cuda_lib, m, k):
 GEMM_CASES = [
     (1, 1, 32), (1, 15, 96), (1, 16, 128), (1, 17, 4096), (1, 1024, 4096), (2, 33, 256), (3, 64, 160),
     (5, 40, 1024), (8, 16, 8192), (9, 48, 512), (16, 100, 384), (31, 17, 1024), (32, 64, 2048),
-    (33, 20, 256), (40, 64, 128), (4, 3, 16384),
+    (33, 20, 256), (40, 64, 128), (4, 3, 16384), (20, 50, 640), (24, 33, 1056), (17, 300, 4096),
 ]
 
 
@@ -273,7 +273,7 @@ def test_llama3_8b_layer_full_size(cuda_lib):
         assert _rel_l2(y.cpu().numpy()[rows], y_ref)[0] <= REL_L2_TOL, name
 
 
-@pytest.mark.parametrize("m", [1, 2, 4, 8, 16, 32])
+@pytest.mark.parametrize("m", [1, 2, 4, 8, 16, 24, 32])
 def test_ffn_70b_skinny_sweep_full_size(cuda_lib, m):
     n, k = inputs.FFN_70B["gate"]
     W = inputs.gaussian_matrix(2, 0, n, k, 0.015, BF16, DEV)
