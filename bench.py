@@ -481,7 +481,9 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 in, fp16 tensor-core operands, fp32 accumulate",
+        "vs_baseline": None, "dtype": "f16",
+        "dtype_detail": "fused product: f16 tensor-core operands (centroids, pre-rotated x), f32 accumulate and "
+                        "scales; codec: f32 (bit-exact order); inputs bf16",
         "data": "synthetic (seeded counter-based generator; no checkpoints)",
         "config": dict(desc, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                        l2="flushed (256 MB write) before every timed phase replay; step loop inputs > L2",
