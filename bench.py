@@ -797,7 +797,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
             "steps": max(1, args.steps), "warmup": max(3, args.warmup),
             "ms_per_step": round(1e3 * wall / max(1, args.steps), 2), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp32 codec / fp64 product (CPU oracle)",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "dtype_detail": "CPU oracle: f32 codec in the codec order, f64 product",
             "data": "synthetic (seeded counter-based generator; no checkpoints)",
             "config": {"workload": args.workload, "sample": "first 1/64 of the rows of every matrix per step"},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
