@@ -158,9 +158,8 @@ tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t
 // the tcgen05 prefill kernel.
 constexpr int64_t kSkinnyMaxM = 32;
 
-// Prefill workspace: header | split area (the last wave's K halves) | plain xrot.
 static size_t prefill_workspace(int64_t m, int64_t k) {
-    return kStatusBytes + tq::prefill_split_bytes() + tq::prefill_xrot_bytes(m < 1 ? 1 : m, k);
+    return kStatusBytes + tq::prefill_xrot_bytes(m < 1 ? 1 : m, k);
 }
 
 size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
@@ -199,11 +198,9 @@ static tq_status run_prefill(const uint8_t *codes, const uint16_t *scales, int64
     if ((st = check_workspace(workspace, ws_bytes, prefill_workspace(m, k))) != TQ_OK) return st;
     if ((m + 255) / 256 > 65535) return TQ_ERR_SHAPE;
     char *ws = static_cast<char *>(workspace);
-    const size_t split_bytes = tq::prefill_split_bytes();
-    const cudaError_t e = tq::launch_prefill(codes, scales, n, k, X, xt, m, ldx,
-                                             reinterpret_cast<uint16_t *>(ws + kStatusBytes + split_bytes), Y, yt,
-                                             ldy, reinterpret_cast<unsigned *>(ws), ws + kStatusBytes, split_bytes,
-                                             (cudaStream_t)stream);
+    const cudaError_t e =
+        tq::launch_prefill(codes, scales, n, k, X, xt, m, ldx, reinterpret_cast<uint16_t *>(ws + kStatusBytes), Y, yt,
+                           ldy, reinterpret_cast<unsigned *>(ws), (cudaStream_t)stream);
     if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
     return from_cuda(e);
 }
@@ -307,9 +304,7 @@ tq_status tq_gemm_prefill_xrot(const uint8_t *codes, const uint16_t *scales, int
     cudaStream_t s = (cudaStream_t)stream;
     unsigned *header = static_cast<unsigned *>(workspace);
     if (tq::launch_prepare_header(header, s) != cudaSuccess) return TQ_ERR_CUDA;
-    char *ws = static_cast<char *>(workspace);
-    const cudaError_t e = tq::launch_prefill_product(codes, scales, n, k, xrot, m, Y, yt, ldy, header,
-                                                     ws + kStatusBytes, ws_bytes - kStatusBytes, s);
+    const cudaError_t e = tq::launch_prefill_product(codes, scales, n, k, xrot, m, Y, yt, ldy, header, s);
     if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
     return from_cuda(e);
 }

@@ -105,15 +105,9 @@ cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydt
 // (prefill_xrot_bytes), then one CTA per 128 weight rows x 256 activation rows
 // decodes the weight tile into shared memory and multiplies on the tensor cores.
 size_t prefill_xrot_bytes(int64_t m, int64_t k);
-// Area for splitting the last wave's tiles into K halves: kPrefillMeetBytes of
-// meeting words, then two fp32 128 x 256 partial tiles per split tile (up to
-// half the SM count of the current device).  Null / too small: no split.
-constexpr size_t kPrefillMeetBytes = 1024;
-size_t prefill_split_bytes_for(int64_t tiles);
-size_t prefill_split_bytes();
 cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
                            int xdtype, int64_t m, int64_t ldx, uint16_t *xrot, void *y, int ydtype, int64_t ldy,
-                           unsigned *header, void *split_area, size_t split_bytes, cudaStream_t stream);
+                           unsigned *header, cudaStream_t stream);
 // The two steps of launch_prefill on their own: the plain pre-rotation (header
 // may be null; otherwise it clears the status word and advances the call tag)
 // and the product over an xrot it wrote.
@@ -121,7 +115,7 @@ cudaError_t launch_prerotate_plain(const void *X, int xdtype, int64_t m, int64_t
                                    unsigned *header, cudaStream_t stream);
 cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
                                    const uint16_t *xrot, int64_t m, void *y, int ydtype, int64_t ldy,
-                                   unsigned *header, void *split_area, size_t split_bytes, cudaStream_t stream);
+                                   unsigned *header, cudaStream_t stream);
 
 // ---- NVFP4 comparison codec ---------------------------------------------------
 // Same fused product over NVFP4 planes (E2M1 codes in the TQ4_1S unit layout,

@@ -178,15 +178,6 @@ __device__ __forceinline__ uint32_t p_lds_u32(uint32_t a) {
     return v;
 }
 
-__device__ __forceinline__ void p_sts_u32(uint32_t a, uint32_t v) {
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
-}
-
-// Barrier `id` among `count` threads (whole warps) of the CTA.
-__device__ __forceinline__ void p_named_barrier(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 __device__ __forceinline__ void p_sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
@@ -207,17 +198,8 @@ struct PrefillParams {
     int nk;                 // 64-column stages: ceil(k / 64)
     char *y;
     int64_t ldy;
-    unsigned *header;       // workspace header (status word, call tag)
+    unsigned *header;       // workspace header (status word)
     uint64_t timeout_ns;
-    // grid: CTA b < full_ctas computes tile b over all of K; the last
-    // split_tiles tiles are computed as two K halves by CTAs full_ctas + 2 j + h
-    // (tile full_ctas + j, half h), which exchange fp32 partial tiles through
-    // `partials` and meet through `meet` (one word per split tile)
-    int tiles_x;            // weight-row tiles: ceil(n / 128)
-    int full_ctas;
-    int split_tiles;
-    float *partials;        // [split_tiles][2][128 rows][256 columns]
-    unsigned *meet;         // [split_tiles]
 };
 
 // One weight row's superblock slot: its four 16-byte code chunks (chunk b,
@@ -316,18 +298,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         return;
     }
     const uint32_t abase = (base + 1023u) & ~1023u;
-    // this CTA's tile and K range (whole tiles first, then K halves of the last
-    // tiles so that the final wave fills the GPU)
-    const int b = blockIdx.x;
-    const bool split = b >= P.full_ctas;
-    const int tile = split ? P.full_ctas + ((b - P.full_ctas) >> 1) : b;
-    const int half = split ? ((b - P.full_ctas) & 1) : 0;
-    const int n0 = (tile % P.tiles_x) * kPM, m0 = (tile / P.tiles_x) * kPN;
-    const int nsb_all = (P.nk + 1) / 2;        // superblocks touched by the stages
-    const int sb_mid = nsb_all / 2;            // the halves split at a superblock boundary
-    const int sb_lo = split && half == 1 ? sb_mid : 0;
-    const int sb_hi = split && half == 0 ? sb_mid : nsb_all;
-    const int kt_lo = 2 * sb_lo, kt_hi = min(2 * sb_hi, P.nk);
+    const int n0 = blockIdx.x * kPM, m0 = blockIdx.y * kPN;
     auto a_tile = [&](int s) { return abase + (uint32_t)s * kATile; };
     auto b_tile = [&](int s) { return kPBTiles + (uint32_t)s * kBTile; };
     auto full_a = [&](int s) { return kPBars + 8u * s; };
@@ -373,10 +344,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // ---- activation tiles by TMA ----------------------------------------
         if (lane == 0) {
             int issued = 0;
-            for (int kt = kt_lo; kt < kt_hi; ++kt) {
-                const int it = kt - kt_lo;
-                const int s = it % kPStages;
-                const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+            for (int kt = 0; kt < P.nk; ++kt) {
+                const int s = kt % kPStages;
+                const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
                 if (!p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns)) {
                     atomicOr(P.header, kPStatusTimeout);
                     break;
@@ -393,9 +363,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     } else if (warp == 1) {
         // ---- MMA issue ----------------------------------------------------------
         if (lane == 0) {
-            for (int it = 0; it < kt_hi - kt_lo; ++it) {
-                const int s = it % kPStages;
-                const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+            for (int kt = 0; kt < P.nk; ++kt) {
+                const int s = kt % kPStages;
+                const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
                 if (!p_mbar_wait(full_a(s), ph, P.timeout_ns) || !p_mbar_wait(full_b(s), ph, P.timeout_ns)) {
                     atomicOr(P.header, kPStatusTimeout);
                     break;
@@ -404,7 +374,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kPK / 16; ++kk)  // 16 columns = 32 bytes along the swizzled row
                     p_mma(tmem, p_smem_desc(a_tile(s) + 32u * kk), p_smem_desc(b_tile(s) + 32u * kk),
-                          (it | kk) != 0 ? 1u : 0u);
+                          (kt | kk) != 0 ? 1u : 0u);
                 p_mma_commit(empty(s));  // the stage is free once these MMAs have read it
             }
             p_mma_commit(accum);  // the accumulator is final once every MMA has completed
@@ -419,20 +389,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // unrolled by kAhead so that every ring index is a constant)
         RowSlot w[kAhead];
 #pragma unroll
-        for (int i = 0; i < kAhead; ++i) w[i] = load_slot(P, n0 + row, sb_lo + i < sb_hi ? sb_lo + i : P.nsb);
+        for (int i = 0; i < kAhead; ++i) w[i] = load_slot(P, n0 + row, i);
+        const int nsb_stages = (P.nk + 1) / 2;  // superblocks touched by the stages
         bool ok = true;
-        for (int sb0 = sb_lo; sb0 < sb_hi && ok; sb0 += kAhead) {
+        for (int sb0 = 0; sb0 < nsb_stages && ok; sb0 += kAhead) {
 #pragma unroll
             for (int i = 0; i < kAhead; ++i) {
                 const int sb = sb0 + i;
-                if (sb >= sb_hi || !ok) break;
+                if (sb >= nsb_stages || !ok) break;
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {  // the superblock's two stages
                     const int kt = 2 * sb + hb;
-                    if (kt >= kt_hi) break;
-                    const int it = kt - kt_lo;
-                    const int s = it % kPStages;
-                    const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+                    if (kt >= P.nk) break;
+                    const int s = kt % kPStages;
+                    const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
                     // (warp-uniform decision: the epilogue below runs warp-synchronous loads)
                     if (!__all_sync(kFull, p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns))) {
                         if (lane == 0) atomicOr(P.header, kPStatusTimeout);
@@ -443,65 +413,21 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     p_fence_proxy_async();
                     p_mbar_arrive(full_a(s));
                 }
-                w[i] = load_slot(P, n0 + row, sb + kAhead < sb_hi ? sb + kAhead : P.nsb);
+                w[i] = load_slot(P, n0 + row, sb + kAhead);
             }
         }
         // ---- epilogue: tensor memory -> Y ------------------------------------
         const int q = warp & 3;                 // this warp's quarter of the 128 lanes
         const int wrow = n0 + q * 32 + lane;    // weight row = accumulator lane
         const int c0 = ((warp - 2) >> 2) * (kPN / 64);  // two warps per quarter: half of the columns each
-        const bool acc_ok = __all_sync(kFull, p_mbar_wait(accum, 0u, P.timeout_ns));
-        if (!acc_ok && lane == 0) atomicOr(P.header, kPStatusTimeout);
-        if (acc_ok) p_tc_fence_after();
-        // a K half: publish this half's sums; the half that finishes second
-        // adds the other's (half 0 + half 1, the same order either way).  All
-        // eight epilogue warps pass both named barriers whatever happened.
-        bool store_y = acc_ok;
-        const float *other = nullptr;
-        if (split) {
-            const int j = tile - P.full_ctas;
-            if (acc_ok) {
-                float *mine = P.partials + ((size_t)(2 * j + half) * kPM + q * 32 + lane) * kPN;
-#pragma unroll 1
-                for (int c = c0; c < c0 + kPN / 64; ++c) {
-                    uint32_t v[32];
-                    p_tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<uint4 *>(mine + c * 32 + e) = make_uint4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                }
-            }
-            __threadfence();
-            p_named_barrier(1, 32 * kDecodeWarps);
-            if (threadIdx.x == 64) {  // warp 2, lane 0
-                const unsigned tag = *reinterpret_cast<volatile const unsigned *>(P.header + kHeaderTag);
-                const unsigned prev = atomicExch(P.meet + j, tag);
-                p_sts_u32(kPTmemSlot + 4u, prev == tag ? 1u : 0u);  // second to arrive
-            }
-            p_named_barrier(1, 32 * kDecodeWarps);
-            store_y = acc_ok && p_lds_u32(kPTmemSlot + 4u) != 0u;
-            __threadfence();
-            other = P.partials + ((size_t)(2 * j + (half ^ 1)) * kPM + q * 32 + lane) * kPN;
-        }
-        if (store_y) {
+        if (!__all_sync(kFull, p_mbar_wait(accum, 0u, P.timeout_ns))) {
+            if (lane == 0) atomicOr(P.header, kPStatusTimeout);
+        } else {
+            p_tc_fence_after();
 #pragma unroll 1
             for (int c = c0; c < c0 + kPN / 64; ++c) {
                 uint32_t v[32];
                 p_tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
-                if (other) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const float4 o = __ldcg(reinterpret_cast<const float4 *>(other + c * 32 + e));
-                        const float mine4[4] = {__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                                __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])};
-                        const float oth4[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float lo = half == 0 ? mine4[i] : oth4[i], hi = half == 0 ? oth4[i] : mine4[i];
-                            v[e + i] = __float_as_uint(lo + hi);
-                        }
-                    }
-                }
                 if (wrow < P.n) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -647,16 +573,6 @@ cudaError_t launch_plain_rotation(const PlainRotParams &r, cudaStream_t stream) 
 
 size_t prefill_xrot_bytes(int64_t m, int64_t k) { return round_up((size_t)m * (size_t)k * 2u, 256); }
 
-size_t prefill_split_bytes_for(int64_t tiles) {
-    return kPrefillMeetBytes + (size_t)tiles * 2u * (size_t)(kPM * kPN) * sizeof(float);
-}
-
-size_t prefill_split_bytes() {
-    DeviceInfo di;
-    if (device_info(&di) != cudaSuccess) return 0;
-    return prefill_split_bytes_for(di.sm_count / 2);
-}
-
 cudaError_t launch_prerotate_plain(const void *X, int xdtype, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
                                    unsigned *header, cudaStream_t stream) {
     if (m < 1 || k < 32 || k % 32 != 0) return cudaErrorInvalidValue;
@@ -671,23 +587,10 @@ cudaError_t launch_prerotate_plain(const void *X, int xdtype, int64_t m, int64_t
 
 cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
                                    const uint16_t *xrot, int64_t m, void *y, int ydtype, int64_t ldy,
-                                   unsigned *header, void *split_area, size_t split_bytes, cudaStream_t stream) {
+                                   unsigned *header, cudaStream_t stream) {
     if (n < 1 || m < 1 || k < 32 || k % 32 != 0) return cudaErrorInvalidValue;
     const int64_t grid_y = (m + kPN - 1) / kPN, grid_x = (n + kPM - 1) / kPM;
     if (grid_y > 65535 || grid_x > 0x7fffffff) return cudaErrorInvalidValue;
-    DeviceInfo di;
-    cudaError_t derr = device_info(&di);
-    if (derr != cudaSuccess) return derr;
-    // the last, partial wave of tiles: split each into two K halves when that
-    // still fits one wave (one CTA per SM) and the split area holds them
-    const int64_t tiles_all = grid_x * grid_y;
-    const int64_t rem = tiles_all % di.sm_count;
-    const int64_t nsb = superblocks(k);
-    int64_t split_tiles = 0;
-    if (rem > 0 && 2 * rem <= di.sm_count && rem <= (int64_t)(kPrefillMeetBytes / 4) && nsb >= 4 && split_area &&
-        split_bytes >= prefill_split_bytes_for(rem))
-        split_tiles = rem;
-    if (tiles_all + split_tiles > 0x7fffffff) return cudaErrorInvalidValue;
     EncodeTiled encode = encode_tiled();
     if (!encode) return cudaErrorNotSupported;
     // the tensor map of xrot: k x m fp16, rows of k*2 bytes, boxes of
@@ -713,15 +616,10 @@ cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales,
     prm.ldy = ldy;
     prm.header = header;
     prm.timeout_ns = 1000000000ull;
-    prm.tiles_x = (int)grid_x;
-    prm.full_ctas = (int)(tiles_all - split_tiles);
-    prm.split_tiles = (int)split_tiles;
-    prm.meet = split_tiles ? static_cast<unsigned *>(split_area) : nullptr;
-    prm.partials = split_tiles ? reinterpret_cast<float *>(static_cast<char *>(split_area) + kPrefillMeetBytes) : nullptr;
     const uint32_t base = prefill_smem_base();
     if (base > kPMaxBase) return cudaErrorInvalidValue;
     const uint32_t smem = kPEnd - base;
-    const dim3 grid((unsigned)(tiles_all + split_tiles));
+    const dim3 grid((unsigned)grid_x, (unsigned)grid_y);
     switch (ydtype) {
         case kF32: return launch_prefill_kernel<kF32>(map, prm, grid, smem, stream);
         case kBF16: return launch_prefill_kernel<kBF16>(map, prm, grid, smem, stream);
@@ -732,7 +630,7 @@ cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales,
 
 cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
                            int xdtype, int64_t m, int64_t ldx, uint16_t *xrot, void *y, int ydtype, int64_t ldy,
-                           unsigned *header, void *split_area, size_t split_bytes, cudaStream_t stream) {
+                           unsigned *header, cudaStream_t stream) {
     if (n < 1 || m < 1 || k < 32 || k % 32 != 0) return cudaErrorInvalidValue;
     if ((m + kPN - 1) / kPN > 65535) return cudaErrorInvalidValue;
     if (!encode_tiled()) return cudaErrorNotSupported;
@@ -740,8 +638,7 @@ cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t
     cudaError_t err = launch_prerotate_plain(X, xdtype, m, k, ldx, xrot, header, stream);
     if (err != cudaSuccess) return err;
     // 2. the product
-    return launch_prefill_product(codes, scales, n, k, xrot, m, y, ydtype, ldy, header, split_area, split_bytes,
-                                  stream);
+    return launch_prefill_product(codes, scales, n, k, xrot, m, y, ydtype, ldy, header, stream);
 }
 
 }  // namespace tq

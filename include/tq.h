@@ -190,14 +190,8 @@ TQ_API tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n
  * more rounding per weight (relative 2^-11).  Same operand rules as tq_gemm;
  * any m >= 1 (m <= 16,776,960).  Returns TQ_ERR_UNSUPPORTED if the driver
  * offers no tensor-map encoder.
- *   workspace  >= tq_gemm_prefill_workspace_bytes(m, k) bytes, 256-byte
- *              aligned: a 256-byte header; room for the last wave's tiles
- *              split into two K halves (1 KB of meeting words and two fp32
- *              128 x 256 partial tiles for up to half the SM count of the
- *              current device, so the final wave fills the GPU); then m*k
- *              fp16.  Zero-fill a new workspace once (see above).
- * The halves of a split tile are added in a fixed order, so results are
- * deterministic; they differ from an unsplit tile's only by fp32 rounding.
+ *   workspace  >= tq_gemm_prefill_workspace_bytes(m, k) bytes (256-byte
+ *              header + m*k fp16), 256-byte aligned
  */
 TQ_API size_t tq_gemm_prefill_workspace_bytes(int64_t m, int64_t k);
 TQ_API tq_status tq_gemm_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,
@@ -219,12 +213,9 @@ TQ_API tq_status tq_gemm_prefill(const uint8_t *codes, const uint16_t *scales, i
  *         (written; read by tensor-memory-accelerator copies afterwards)
  *
  * tq_gemm_prefill_xrot -- the tensor-core product of tq_gemm_prefill over an
- * xrot written by tq_prerotate_plain (same m and k).  The workspace needs its
- * 256-byte header (>= 256 bytes, 256-byte aligned); bytes beyond it serve as
- * the split area described under tq_gemm_prefill when there are enough of
- * them (a tq_gemm_prefill workspace always has enough), else every tile is
- * computed whole.  A one-thread launch clears the status word first.  Y, yt,
- * ldy as tq_gemm.
+ * xrot written by tq_prerotate_plain (same m and k).  The workspace needs
+ * only its 256-byte header (>= 256 bytes, 256-byte aligned); a one-thread
+ * launch clears its status word first.  Y, yt, ldy as tq_gemm.
  */
 TQ_API size_t tq_prefill_xrot_bytes(int64_t m, int64_t k);
 TQ_API tq_status tq_prerotate_plain(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
