@@ -13,28 +13,31 @@
 // fp16 pre-rotation H(s .* x)/32.
 //
 // B200 design:
-//  * One CTA per output tile of 128 weight rows x 256 activation rows (one
-//    tcgen05.mma of M = 128, N = 256, K = 16 per 16 columns; fp32 accumulator
-//    of 128 lanes x 256 columns in tensor memory).  Both operands are K-major
-//    in shared memory with the 128-byte swizzle.
+//  * One CTA per output tile of 256 weight rows x 256 activation rows: two
+//    tcgen05.mma of M = 128, N = 256, K = 16 per 16 columns (one per 128-row
+//    half of the weight tile) share the activation operand, each into its own
+//    fp32 accumulator of 128 lanes x 256 columns; together they fill the 512
+//    columns of tensor memory.  Both operands are K-major in shared memory
+//    with the 128-byte swizzle.  Two weight halves per activation tile halve
+//    the activation bytes each flop needs from L2, which sets the pace.
 //  * The activation tile (256 rows x 64 columns of fp16 per stage) arrives by
-//    TMA (cp.async.bulk.tensor, no multicast).
-//  * The weight tile (128 rows x 64 columns per stage) is decoded by eight
+//    TMA (cp.async.bulk.tensor, no multicast); four stages.
+//  * The weight tile (256 rows x 64 columns per stage) is decoded by sixteen
 //    warps, one row and one 32-column block per thread: each thread reads its
 //    row's 64-byte superblock slot with 16-byte loads (neighbouring threads,
 //    neighbouring slots), three superblocks ahead in registers; a 4x4 byte
-//    transpose restores element
-//    order, a lane-replicated shared table turns each code byte into an fp16
-//    pair, one fp16 multiply applies the half-block scale, and 16-byte stores
-//    write the swizzled rows.  A proxy fence then publishes them to the tensor
-//    cores.
+//    transpose restores element order; byte permutes against register tables
+//    of the fp16 magnitudes, with the sign bits merged in by two more
+//    permutes, give fp16 centroid pairs; one fp16 multiply applies the
+//    half-block scale and 16-byte stores write the swizzled rows.  A proxy
+//    fence then publishes them to the tensor cores.  Three stages.
 //  * One thread issues the MMAs; tcgen05.commit releases each stage to its
-//    producers and finally signals the epilogue.  The eight decode warps then
-//    read the accumulator (tcgen05.ld, one weight row per thread, two warps per
-//    32-lane quarter) and store Y with consecutive threads on consecutive
-//    columns.
-//  * Three stages; every mbarrier wait is bounded in time and reports through
-//    the workspace status word.
+//    producers and finally signals the epilogue.  The sixteen decode warps
+//    then read the accumulators (tcgen05.ld, one weight row per thread, four
+//    warps per 32-lane quarter: accumulator half and 128 columns each) and
+//    store Y with consecutive threads on consecutive columns.
+//  * Every mbarrier wait is bounded in time and reports through the
+//    workspace status word.
 #include <cuda.h>
 
 #include <mutex>
@@ -46,35 +49,35 @@ namespace tq {
 
 namespace {
 
-constexpr int kPM = 128;                 // weight rows per tile (MMA M)
+constexpr int kPM = 256;                 // weight rows per tile (two MMA halves of 128)
+constexpr int kMmaM = 128;               // rows of one MMA (cta_group::1 takes M = 64 or 128)
 constexpr int kPN = 256;                 // activation rows per tile (MMA N)
 constexpr int kPK = 64;                  // columns per stage: one 128-byte swizzle row of fp16
-constexpr int kPStages = 3;
-constexpr int kATile = kPM * kPK * 2;    // 16 KB
+constexpr int kSA = 3;                   // weight-tile stages
+constexpr int kSB = 4;                   // activation-tile stages
+constexpr int kATile = kPM * kPK * 2;    // 32 KB (half h at + 16 KB * h)
+constexpr int kAHalf = kATile / 2;
 constexpr int kBTile = kPN * kPK * 2;    // 32 KB
-constexpr int kDecodeWarps = 8;          // warps 2..9: (row, block) per thread
+constexpr int kDecodeWarps = 16;         // warps 2..17: (row, block) per thread
 constexpr int kPThreads = (2 + kDecodeWarps) * 32;
-constexpr int kTmemCols = 256;
+constexpr int kTmemCols = 512;           // two accumulators of 256 fp32 columns
 constexpr int kAhead = 3;       // superblocks of row slots held in registers ahead of the decode
 
-// Shared-memory map (addresses in the CTA's shared window; the dynamic
-// allocation starts at a base B <= kPMaxBase):
-//   [align1024(B), + 3 x 16 KB)   weight tiles (A)
-//   [0x10000, 0x20000)            code-pair table (entry v, lane l at 256 v + 4 l)
-//   [0x20000, 0x38000)            activation tiles (B), 3 x 32 KB
-//   [0x38000, ...)                mbarriers, tensor-memory address
-constexpr uint32_t kPLut = 0x10000;
-constexpr uint32_t kPBTiles = 0x20000;
-constexpr uint32_t kPBars = kPBTiles + kPStages * kBTile;  // full_a[3] full_b[3] empty[3] accum
-constexpr uint32_t kPTmemSlot = kPBars + 16 * 8;
-constexpr uint32_t kPEnd = kPTmemSlot + 16;
-constexpr uint32_t kPMaxBase = 0x10000 - kPStages * kATile - 1024;
-static_assert(kPEnd - 1024 <= 227 * 1024, "dynamic shared memory per CTA");
+// Shared-memory map (offsets from the 1024-aligned start of the dynamic
+// allocation): weight stages, activation stages, then the mbarriers
+// full_a[kSA] full_b[kSB] empty_a[kSA] empty_b[kSB] accum and the
+// tensor-memory address slot.
+constexpr uint32_t kPAOff = 0;
+constexpr uint32_t kPBOff = kPAOff + kSA * kATile;
+constexpr uint32_t kPBarOff = kPBOff + kSB * kBTile;
+constexpr uint32_t kPTmemOff = kPBarOff + 8 * (2 * kSA + 2 * kSB + 1);
+constexpr uint32_t kPEndOff = kPTmemOff + 16;
+constexpr uint32_t kPMaxBase = 1024;     // dynamic shared memory starts at most here
+static_assert(kPEndOff + kPMaxBase - 1024 <= 227 * 1024, "dynamic shared memory per CTA");
 
 constexpr unsigned kPStatusTimeout = 1u;
 constexpr unsigned kPStatusLayout = 2u;
-
-__constant__ uint16_t c_pmag_f16[8] = TQ_MAG_F16_INIT;
+constexpr unsigned kPStatusTmem = 4u;  // tensor-memory base not at lane 0, column 0
 
 // ---- PTX wrappers -----------------------------------------------------------
 __device__ __forceinline__ uint64_t p_global_ns() {
@@ -143,7 +146,7 @@ __device__ __forceinline__ uint64_t p_smem_desc(uint32_t addr) {
 
 // Instruction descriptor: fp32 accumulator, fp16 A and B, both K-major,
 // N = 256, M = 128.
-constexpr uint32_t kPIdesc = (1u << 4) | ((uint32_t)(kPN >> 3) << 17) | ((uint32_t)(kPM >> 4) << 24);
+constexpr uint32_t kPIdesc = (1u << 4) | ((uint32_t)(kPN >> 3) << 17) | ((uint32_t)(kMmaM >> 4) << 24);
 
 __device__ __forceinline__ void p_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
     asm volatile(
@@ -262,15 +265,49 @@ __device__ __forceinline__ void p_transpose4(const uint32_t (&w)[4], uint32_t (&
     o[3] = prmt(c, d, 0x7632u);
 }
 
+// fp16 Lloyd-Max magnitudes as byte tables for PRMT: low bytes of magnitudes
+// 0..3 / 4..7 and high bytes of magnitudes 0..3 / 4..7.
+constexpr uint16_t kPMag[8] = TQ_MAG_F16_INIT;
+constexpr uint32_t mag_bytes(int i0, bool hi) {
+    uint32_t v = 0;
+    for (int i = 0; i < 4; ++i) v |= (uint32_t)((hi ? kPMag[i0 + i] >> 8 : kPMag[i0 + i]) & 0xFF) << (8 * i);
+    return v;
+}
+constexpr uint32_t kMagLo0 = mag_bytes(0, false), kMagLo1 = mag_bytes(4, false);
+constexpr uint32_t kMagHi0 = mag_bytes(0, true), kMagHi1 = mag_bytes(4, true);
+
+// Eight codes (one logical word: element 2L in the low nibble of byte L,
+// element 2L+1 in the high nibble) to four fp16 pairs of signed centroids.
+//  * magnitudes: PRMT with the three magnitude bits of four codes as its
+//    selector nibbles picks their low (high) bytes from the byte tables;
+//  * signs: a code's sign is bit 3 of its nibble, i.e. the top bit of a byte
+//    of w (odd elements) or of w << 4 (even elements); PRMT in sign-replicate
+//    mode turns those top bits into 0xFF / 0x00 bytes, one per code, whose
+//    top bit is merged into the high bytes;
+//  * two more PRMTs interleave low and high bytes into fp16 pairs.
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t (&o)[4]) {
+    const uint32_t m = w & 0x77777777u;  // magnitude ranks (PRMT reads the low 16 bits)
+    const uint32_t m2 = m >> 16;
+    const uint32_t w4 = w << 4;
+    // byte j of the mask: sign of element j (selector nibbles: 8 | byte, a = w4, b = w)
+    const uint32_t s03 = prmt(w4, w, 0xD9C8u), s47 = prmt(w4, w, 0xFBEAu);
+    const uint32_t lo03 = prmt(kMagLo0, kMagLo1, m), lo47 = prmt(kMagLo0, kMagLo1, m2);
+    const uint32_t hi03 = prmt(kMagHi0, kMagHi1, m) | (s03 & 0x80808080u);
+    const uint32_t hi47 = prmt(kMagHi0, kMagHi1, m2) | (s47 & 0x80808080u);
+    o[0] = prmt(lo03, hi03, 0x5140u);  // elements 0, 1
+    o[1] = prmt(lo03, hi03, 0x7362u);  // elements 2, 3
+    o[2] = prmt(lo47, hi47, 0x5140u);  // elements 4, 5
+    o[3] = prmt(lo47, hi47, 0x7362u);  // elements 6, 7
+}
+
 // Decode one row's 32-column block jj of the stage into the swizzled weight
 // tile.  In a row's 64-byte superblock slot, logical byte L of block j sits at
 // chunk L % 4, word j, byte L / 4; so the block's four chunk words, byte-
-// transposed, give logical words i = 0..3, each holding elements 8i .. 8i+7
-// (element 2L in the low nibble of byte L).  Logical word i lands in 16-byte
+// transposed, give logical words i = 0..3, each holding elements 8i .. 8i+7.
+// The half-block scale multiplies in fp16.  Logical word i lands in 16-byte
 // chunk 4 jj + i of the tile row, stored at chunk (4 jj + i) xor (row % 8)
 // (the 128-byte swizzle).
-__device__ __forceinline__ void decode_block(const BlockWords &w, int row, int jj, uint32_t atile,
-                                             uint32_t lut_lane) {
+__device__ __forceinline__ void decode_block(const BlockWords &w, int row, int jj, uint32_t atile) {
     const uint32_t rbase = atile + (uint32_t)row * 128u;
     uint32_t L[4];
     p_transpose4(w.c, L);
@@ -278,12 +315,10 @@ __device__ __forceinline__ void decode_block(const BlockWords &w, int row, int j
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t d = i < 2 ? d0 : d1;  // elements 0..15 take d0, 16..31 d1
-        const uint32_t o0 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7604u)), d);
-        const uint32_t o1 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7614u)), d);
-        const uint32_t o2 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7624u)), d);
-        const uint32_t o3 = p_hmul2(p_lds_u32(prmt(L[i], lut_lane, 0x7634u)), d);
+        uint32_t v[4];
+        decode_word(L[i], v);
         const uint32_t chunk = (uint32_t)(4 * jj + i) ^ (uint32_t)(row & 7);
-        p_sts128(rbase + chunk * 16u, o0, o1, o2, o3);
+        p_sts128(rbase + chunk * 16u, p_hmul2(v[0], d), p_hmul2(v[1], d), p_hmul2(v[2], d), p_hmul2(v[3], d));
     }
 }
 
@@ -297,37 +332,33 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (threadIdx.x == 0) atomicOr(P.header, kPStatusLayout);
         return;
     }
-    const uint32_t abase = (base + 1023u) & ~1023u;
+    const uint32_t sbase = (base + 1023u) & ~1023u;
     const int n0 = blockIdx.x * kPM, m0 = blockIdx.y * kPN;
-    auto a_tile = [&](int s) { return abase + (uint32_t)s * kATile; };
-    auto b_tile = [&](int s) { return kPBTiles + (uint32_t)s * kBTile; };
-    auto full_a = [&](int s) { return kPBars + 8u * s; };
-    auto full_b = [&](int s) { return kPBars + 24u + 8u * s; };
-    auto empty = [&](int s) { return kPBars + 48u + 8u * s; };
-    const uint32_t accum = kPBars + 72u;
+    auto a_tile = [&](int s) { return sbase + kPAOff + (uint32_t)s * kATile; };
+    auto b_tile = [&](int s) { return sbase + kPBOff + (uint32_t)s * kBTile; };
+    const uint32_t bars = sbase + kPBarOff;
+    auto full_a = [&](int s) { return bars + 8u * s; };
+    auto full_b = [&](int s) { return bars + 8u * (kSA + s); };
+    auto empty_a = [&](int s) { return bars + 8u * (kSA + kSB + s); };
+    auto empty_b = [&](int s) { return bars + 8u * (2 * kSA + kSB + s); };
+    const uint32_t accum = bars + 8u * (2 * kSA + 2 * kSB);
+    const uint32_t tmem_slot = sbase + kPTmemOff;
 
-    // ---- set-up: barriers, code-pair table, tensor memory ------------------
+    // ---- set-up: barriers, tensor memory -------------------------------------
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kPStages; ++s) {
+        for (int s = 0; s < kSA; ++s) {
             p_mbar_init(full_a(s), 32 * kDecodeWarps);
+            p_mbar_init(empty_a(s), 1);
+        }
+        for (int s = 0; s < kSB; ++s) {
             p_mbar_init(full_b(s), 1);
-            p_mbar_init(empty(s), 1);
+            p_mbar_init(empty_b(s), 1);
         }
         p_mbar_init(accum, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    {
-        uint4 *lut = reinterpret_cast<uint4 *>(smem + (kPLut - base));
-        for (int idx = threadIdx.x; idx < 256 * 8; idx += kPThreads) {  // entry v: 8 x 16 bytes
-            const int v = idx >> 3;
-            const uint32_t lo = c_pmag_f16[v & 7] | ((v & 8) ? 0x8000u : 0u);
-            const uint32_t hi = c_pmag_f16[(v >> 4) & 7] | ((v & 0x80) ? 0x8000u : 0u);
-            const uint32_t e = lo | (hi << 16);
-            lut[v * 16 + (idx & 7)] = make_uint4(e, e, e, e);
-        }
-    }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(kPTmemSlot),
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tmem_slot),
                      "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -335,7 +366,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
     p_tc_fence_before();
     __syncthreads();
     p_tc_fence_after();
-    const uint32_t tmem = p_lds_u32(kPTmemSlot);
+    const uint32_t tmem = p_lds_u32(tmem_slot);
+    // both accumulators need the whole of tensor memory: checked, never expected
+    const bool tmem_ok = tmem == 0u;
+    if (!tmem_ok && threadIdx.x == 0) atomicOr(P.header, kPStatusTmem);
     // the activation tiles are the pre-rotation's output
     grid_dependency_wait();
     grid_dependents_launch();
@@ -345,9 +379,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (lane == 0) {
             int issued = 0;
             for (int kt = 0; kt < P.nk; ++kt) {
-                const int s = kt % kPStages;
-                const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
-                if (!p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns)) {
+                const int s = kt % kSB;
+                const uint32_t ph = (uint32_t)(kt / kSB) & 1u;
+                if (!p_mbar_wait(empty_b(s), ph ^ 1u, P.timeout_ns)) {
                     atomicOr(P.header, kPStatusTimeout);
                     break;
                 }
@@ -356,35 +390,39 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 ++issued;
             }
             // no copy may still be in flight when the CTA exits
-            for (int kt = issued > kPStages ? issued - kPStages : 0; kt < issued; ++kt)
-                p_mbar_wait(full_b(kt % kPStages), (uint32_t)(kt / kPStages) & 1u, P.timeout_ns);
+            for (int kt = issued > kSB ? issued - kSB : 0; kt < issued; ++kt)
+                p_mbar_wait(full_b(kt % kSB), (uint32_t)(kt / kSB) & 1u, P.timeout_ns);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---- MMA issue ----------------------------------------------------------
         if (lane == 0) {
             for (int kt = 0; kt < P.nk; ++kt) {
-                const int s = kt % kPStages;
-                const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
-                if (!p_mbar_wait(full_a(s), ph, P.timeout_ns) || !p_mbar_wait(full_b(s), ph, P.timeout_ns)) {
+                const int sa = kt % kSA, sb = kt % kSB;
+                const uint32_t pa = (uint32_t)(kt / kSA) & 1u, pb = (uint32_t)(kt / kSB) & 1u;
+                if (!p_mbar_wait(full_a(sa), pa, P.timeout_ns) || !p_mbar_wait(full_b(sb), pb, P.timeout_ns)) {
                     atomicOr(P.header, kPStatusTimeout);
                     break;
                 }
                 p_tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < kPK / 16; ++kk)  // 16 columns = 32 bytes along the swizzled row
-                    p_mma(tmem, p_smem_desc(a_tile(s) + 32u * kk), p_smem_desc(b_tile(s) + 32u * kk),
-                          (kt | kk) != 0 ? 1u : 0u);
-                p_mma_commit(empty(s));  // the stage is free once these MMAs have read it
+                for (int kk = 0; kk < kPK / 16 && tmem_ok; ++kk) {  // 16 columns = 32 bytes along the swizzled row
+                    const uint64_t bdesc = p_smem_desc(b_tile(sb) + 32u * kk);
+                    const uint32_t acc = (kt | kk) != 0 ? 1u : 0u;
+                    p_mma(tmem, p_smem_desc(a_tile(sa) + 32u * kk), bdesc, acc);                  // rows 0..127
+                    p_mma(tmem + (uint32_t)kPN, p_smem_desc(a_tile(sa) + kAHalf + 32u * kk), bdesc, acc);  // 128..255
+                }
+                // the stages are free once these MMAs have read them
+                p_mma_commit(empty_a(sa));
+                p_mma_commit(empty_b(sb));
             }
-            p_mma_commit(accum);  // the accumulator is final once every MMA has completed
+            p_mma_commit(accum);  // the accumulators are final once every MMA has completed
         }
         __syncwarp();
     } else {
         // ---- weight tiles: decode (thread = one row, one 32-column block) ---------
         const int td = (warp - 2) * 32 + lane;
         const int row = td & (kPM - 1), jj = td / kPM;
-        const uint32_t lut_lane = kPLut | ((uint32_t)lane * 4u);
         // row slots kAhead superblocks ahead, in a register ring (the loop is
         // unrolled by kAhead so that every ring index is a constant)
         RowSlot w[kAhead];
@@ -401,40 +439,46 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 for (int hb = 0; hb < 2; ++hb) {  // the superblock's two stages
                     const int kt = 2 * sb + hb;
                     if (kt >= P.nk) break;
-                    const int s = kt % kPStages;
-                    const uint32_t ph = (uint32_t)(kt / kPStages) & 1u;
+                    const int s = kt % kSA;
+                    const uint32_t ph = (uint32_t)(kt / kSA) & 1u;
                     // (warp-uniform decision: the epilogue below runs warp-synchronous loads)
-                    if (!__all_sync(kFull, p_mbar_wait(empty(s), ph ^ 1u, P.timeout_ns))) {
+                    if (!__all_sync(kFull, p_mbar_wait(empty_a(s), ph ^ 1u, P.timeout_ns))) {
                         if (lane == 0) atomicOr(P.header, kPStatusTimeout);
                         ok = false;
                         break;
                     }
-                    decode_block(block_of(w[i], 2 * hb + jj), row, jj, a_tile(s), lut_lane);
+                    decode_block(block_of(w[i], 2 * hb + jj), row, jj, a_tile(s));
                     p_fence_proxy_async();
                     p_mbar_arrive(full_a(s));
                 }
                 w[i] = load_slot(P, n0 + row, sb + kAhead);
             }
         }
-        // ---- epilogue: tensor memory -> Y ------------------------------------
-        const int q = warp & 3;                 // this warp's quarter of the 128 lanes
-        const int wrow = n0 + q * 32 + lane;    // weight row = accumulator lane
-        const int c0 = ((warp - 2) >> 2) * (kPN / 64);  // two warps per quarter: half of the columns each
-        if (!__all_sync(kFull, p_mbar_wait(accum, 0u, P.timeout_ns))) {
-            if (lane == 0) atomicOr(P.header, kPStatusTimeout);
-        } else {
-            p_tc_fence_after();
+        // ---- epilogue: tensor memory -> Y (all sixteen decode warps) ---------
+        // warp w may read lanes 32 (w % 4) .. +31; four warps per quarter, each
+        // reads four 32-column chunks of one accumulator (h = weight-row half)
+        if (tmem_ok) {
+            const int q = warp & 3;
+            const int iq = (warp - 2) >> 2;          // 0..3 within the quarter
+            const int h = iq >> 1;
+            const int c0 = (iq & 1) * (kPN / 64);
+            const int wrow = n0 + h * 128 + q * 32 + lane;
+            if (!__all_sync(kFull, p_mbar_wait(accum, 0u, P.timeout_ns))) {
+                if (lane == 0) atomicOr(P.header, kPStatusTimeout);
+            } else {
+                p_tc_fence_after();
 #pragma unroll 1
-            for (int c = c0; c < c0 + kPN / 64; ++c) {
-                uint32_t v[32];
-                p_tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
-                if (wrow < P.n) {
+                for (int c = c0; c < c0 + kPN / 64; ++c) {
+                    uint32_t v[32];
+                    p_tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kPN + c * 32), v);
+                    if (wrow < P.n) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int mrow = m0 + c * 32 + e;
-                        if (mrow < P.m)
-                            store1<OT>(P.y + ((int64_t)mrow * P.ldy + wrow) * ElemSize<OT>::value,
-                                       __uint_as_float(v[e]));
+                        for (int e = 0; e < 32; ++e) {
+                            const int mrow = m0 + c * 32 + e;
+                            if (mrow < P.m)
+                                store1<OT>(P.y + ((int64_t)mrow * P.ldy + wrow) * ElemSize<OT>::value,
+                                           __uint_as_float(v[e]));
+                        }
                     }
                 }
             }
@@ -618,7 +662,7 @@ cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales,
     prm.timeout_ns = 1000000000ull;
     const uint32_t base = prefill_smem_base();
     if (base > kPMaxBase) return cudaErrorInvalidValue;
-    const uint32_t smem = kPEnd - base;
+    const uint32_t smem = ((base + 1023u) & ~1023u) + kPEndOff - base;
     const dim3 grid((unsigned)grid_x, (unsigned)grid_y);
     switch (ydtype) {
         case kF32: return launch_prefill_kernel<kF32>(map, prm, grid, smem, stream);
