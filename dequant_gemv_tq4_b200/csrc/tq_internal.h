@@ -102,7 +102,7 @@ cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydt
 
 // ---- large-M product on tcgen05 (tq_prefill.cu) ---------------------------------
 // Y = X w~^T for any m: X is first pre-rotated into plain row-major fp16 xrot
-// (prefill_xrot_bytes), then one CTA per 128 weight rows x 256 activation rows
+// (prefill_xrot_bytes), then one CTA per 256 weight rows x 256 activation rows
 // decodes the weight tile into shared memory and multiplies on the tensor cores.
 size_t prefill_xrot_bytes(int64_t m, int64_t k);
 cudaError_t launch_prefill(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X,

@@ -182,10 +182,11 @@ TQ_API tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n
  * the fifth-generation tensor cores (TQ page, 解码速度 section: rotate the
  * activation once, then every weight is centroid times scale).  X is first
  * pre-rotated into a plain row-major fp16 matrix in the workspace; then each
- * CTA takes 128 weight rows x 256 activation rows: it decodes its weight rows
+ * CTA takes 256 weight rows x 256 activation rows: it decodes its weight rows
  * 64 columns at a time into shared memory (centroid x half-block scale, fp16),
  * receives the matching activation columns by TMA, and accumulates
- * tcgen05.mma products (fp16 operands, fp32 accumulator in tensor memory).
+ * tcgen05.mma products (fp16 operands, two fp32 accumulators in tensor
+ * memory, one per 128-row half of the weight tile).
  * Compared with tq_gemm's skinny path the weight enters as fp16(c * d), one
  * more rounding per weight (relative 2^-11).  Same operand rules as tq_gemm;
  * any m >= 1 (m <= 16,776,960).  Returns TQ_ERR_UNSUPPORTED if the driver
