@@ -443,7 +443,10 @@ def run_ours(args, world, rank, local):
     barrier(world)
     t_q = time_replays(q_run, steps, flush)
     t_d = time_replays(d_run, steps, flush)
-    t_g = time_replays(g_run, steps, flush)
+    # the GEMV passes alternate between two layers whose packed weights
+    # together exceed L2, so they need no flush (a write flush would leave
+    # 126 MB of dirty lines for the first pass to write back)
+    t_g = time_replays(g_run, steps)
     per_matrix = {}
     for i, it in enumerate(path.items):
         run_i = capture(path.gemv_one(i), use_graph)
@@ -486,7 +489,9 @@ def run_ours(args, world, rank, local):
                         "scales; codec: f32 (bit-exact order); inputs bf16",
         "data": "synthetic (seeded counter-based generator; no checkpoints)",
         "config": dict(desc, parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                       l2="flushed (256 MB write) before every timed phase replay; step loop inputs > L2",
+                       l2="quantise / dequantise phases: flushed (256 MB write) before every replay; GEMV "
+                          "phase and codec comparison: inputs > L2 (passes alternate between two layers, "
+                          "2 x 136.5 MB packed), no flush; step loop: inputs > L2",
                        graph=use_graph, hbm_peak_source=hbm_kind),
         "pct_of_hbm_peak": round(100 * value / world / hbm, 2),
         "quantize_gweights_per_s": round(quant_gw, 2),
@@ -558,12 +563,12 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
             out.append((c, s, t, n, k, X, torch.empty((m, n), dtype=torch.float32, device=device)))
         return out
 
-    def timed(fn, passes):
+    def timed(fn, passes, fl=None):
         run = capture(fn, use_graph, passes)
         for _ in range(warmup):
             run()
         torch.cuda.synchronize()
-        return time_replays(run, steps, flush) / (steps * passes)
+        return time_replays(run, steps, fl) / (steps * passes)
 
     result = {}
     for codec in ("tq4_1s", "nvfp4"):
@@ -592,7 +597,7 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
                 def pair(a=a, b=b, da=da, db=db, wa=wa, wb=wb, m=m):
                     tq.nvfp4_gemm_batch(a, m=m, ws=wa, descs=da)
                     tq.nvfp4_gemm_batch(b, m=m, ws=wb, descs=db)
-            ms = timed(pair, R // 2) / 2
+            ms = timed(pair, R // 2) / 2  # two layers alternate: packed bytes together > L2, no flush
             (ms,) = max_over_ranks([ms], world)
             entry[f"gemm_m{m}_us"] = round(1e3 * ms, 2)
             entry[f"gemm_m{m}_gbs"] = round(job_gbs(packed, world, ms), 1)
@@ -607,7 +612,7 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
                                               t.data_ptr(), torch.cuda.current_stream().cuda_stream)
                     if st != 0:
                         raise tq.TQError(st, "tq_nvfp4_quantize")
-        ms_q = timed(qfn, R)
+        ms_q = timed(qfn, R, flush)
         (ms_q,) = max_over_ranks([ms_q], world)
         entry["quantize_gweights_per_s"] = round(job_gbs(path.weights(), world, ms_q), 2)
         # reconstruction error over the layer: ||W~ - W|| / ||W||

@@ -17,7 +17,8 @@
 //    The units of all matrices in the group form one index space, split evenly
 //    over every warp of a one-CTA-per-SM grid (stream-K style), so each warp
 //    streams one contiguous stretch of memory.
-//  * Each warp keeps a ring of two stages of two units each in shared memory,
+//  * Each warp keeps a ring of two stages of four units (one activation row)
+//    or two units (more rows) in shared memory,
 //    filled by cp.async.bulk (TMA bulk copies, one lane issues, an mbarrier
 //    per stage counts the bytes).  No registers are spent on loads in flight;
 //    waits are bounded in time and report a timeout through a status word.
@@ -51,40 +52,51 @@ namespace tq {
 
 namespace {
 
-// Warps per CTA: one-row products keep few registers live and take 20 warps;
-// up to 16 rows take 16 (128 registers per thread); 17..32 rows take 12, whose
-// three or four accumulator tiles need up to 168 registers without spilling.
-__host__ __device__ constexpr int warps_for(bool one_row, int nt = 1) { return one_row ? 20 : (nt >= 3 ? 12 : 16); }
+// Warps per CTA and units per ring stage.  One activation row: 12 warps of up
+// to 168 registers, four units per stage (fewer, longer-lived warps with deeper
+// stages beat 16 or 20 warps of two or three units: the per-stage loop and
+// copy bookkeeping is paid once per four units, and each warp's stretch of the
+// unit space is longer).  Up to 16 rows: 16 warps (128 registers), two units
+// per stage; 17..32 rows: 12 warps, whose three or four accumulator tiles need
+// up to 168 registers without spilling.
+__host__ __device__ constexpr int warps_for(bool one_row, int nt = 1) { return one_row ? 12 : (nt >= 3 ? 12 : 16); }
 constexpr int kStages = 2;  // ring stages per warp
-constexpr int kPerStage = 2;  // consecutive units per stage
 constexpr int kUnitCodeBytes = 1024;
 constexpr int kUnitScaleBytes = 256;  // TQ4_1S: 16 rows x 4 blocks x 2 fp16; NVFP4 uses 128 (16 x 8 E4M3)
 constexpr int kUnitBytes = kUnitCodeBytes + kUnitScaleBytes;
-// stage = [codes of unit A | codes of unit B | scales of A | scales of B]
-constexpr int kStageScaleOff = kPerStage * kUnitCodeBytes;
-constexpr int kStageBytes = kPerStage * kUnitBytes;    // 2560 (room for either codec)
-constexpr int kRingWarpBytes = kStages * kStageBytes;  // 5120
+// stage = [codes of units 0 .. P-1 | scales of units 0 .. P-1]
+template <bool M1>
+struct Ring {
+    static constexpr int kPerStage = M1 ? 4 : 2;  // consecutive units per stage
+    static constexpr int kStageScaleOff = kPerStage * kUnitCodeBytes;
+    static constexpr int kStageBytes = kPerStage * kUnitBytes;  // room for either codec
+    static constexpr int kRingWarpBytes = kStages * kStageBytes;
+};
 // Shared-memory map (addresses in the CTA's shared window; the dynamic
 // allocation starts at a small base B <= kMaxSmemBase):
-//   [B, B + W/2 rings)          rings of the first half of the W warps
+//   [kBarAddr, kLowRings)       the mbarriers
+//   [kLowRings, 0x10000)        rings of the first kLowWarps warps
 //   [0x10000, 0x20000)          lookup table, 64 KB aligned so that one PRMT
 //                               yields the full address of an entry
-//   [0x20000, + W/2 rings)      rings of the second half
-//   then the mbarriers
+//   [0x20000, kTop)             rings of the other warps
 constexpr uint32_t kLutAddr = 0x10000;
 constexpr uint32_t kHighRings = 0x20000;
-template <int W>
+template <int W, bool M1>
 struct Geometry {
     static constexpr int kWarps = W;
     static constexpr int kThreads = W * 32;
-    static constexpr int kLowWarps = W / 2;
-    static constexpr uint32_t kMaxSmemBase = 0x10000 - kLowWarps * kRingWarpBytes;
-    static constexpr uint32_t kBarAddr = kHighRings + (W - kLowWarps) * kRingWarpBytes;
+    static constexpr int kRingWarpBytes = Ring<M1>::kRingWarpBytes;
     static constexpr uint32_t kBarBytes = W * kStages * 8;
-    static_assert(kMaxSmemBase >= 1024 && kMaxSmemBase < 0x10000, "ring placement below the table");
-    static_assert(kBarAddr + kBarBytes - 1024 <= 227 * 1024, "dynamic shared memory per CTA");
+    static constexpr int kLowFit = (int)((0x10000u - 1024u - kBarBytes) / kRingWarpBytes);
+    static constexpr int kLowWarps = W < kLowFit ? W : kLowFit;
+    static constexpr uint32_t kLowRings = 0x10000u - kLowWarps * kRingWarpBytes;
+    static constexpr uint32_t kBarAddr = kLowRings - kBarBytes;
+    static constexpr uint32_t kMaxSmemBase = kBarAddr;
+    static constexpr uint32_t kTop = kHighRings + (W - kLowWarps) * kRingWarpBytes;
+    static_assert(kMaxSmemBase >= 1024, "barriers and rings below the table");
+    static_assert(kTop - 1024 <= 227 * 1024, "dynamic shared memory per CTA");
     // dynamic shared memory to request for a dynamic base of `base` bytes
-    static uint32_t smem_bytes_for_base(uint32_t base) { return kBarAddr + kBarBytes - base; }
+    static uint32_t smem_bytes_for_base(uint32_t base) { return kTop - base; }
 };
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusLayout = 2u;
@@ -286,18 +298,18 @@ __device__ __forceinline__ void cursor_step(const GroupParams &P, Cursor &cu, in
 // Copy the next `cnt` (1 or 2) units of the cursor into a stage.  Units of one
 // tile are contiguous in both planes, so a pair is one copy per plane; a pair
 // that straddles two tiles takes one copy per unit and plane.
-template <int SB>  // scale bytes per unit
+template <int SB, int SOFF>  // scale bytes per unit, offset of the scales in a stage
 __device__ __forceinline__ void issue_stage(const GroupParams &P, Cursor &cu, int cnt, uint32_t dst, uint32_t bar,
                                             uint32_t leader) {
     arrive_expect_tx_pred(leader, bar, (uint32_t)(cnt * (kUnitCodeBytes + SB)));
     if (cu.sb_left >= cnt) {
         bulk_copy_pred(leader, dst, cu.c, (uint32_t)(cnt * kUnitCodeBytes), bar);
-        bulk_copy_pred(leader, dst + kStageScaleOff, cu.s, (uint32_t)(cnt * SB), bar);
+        bulk_copy_pred(leader, dst + SOFF, cu.s, (uint32_t)(cnt * SB), bar);
         cursor_step<SB>(P, cu, cnt);
     } else {
         for (int h = 0; h < cnt; ++h) {
             bulk_copy_pred(leader, dst + h * kUnitCodeBytes, cu.c, kUnitCodeBytes, bar);
-            bulk_copy_pred(leader, dst + kStageScaleOff + h * SB, cu.s, SB, bar);
+            bulk_copy_pred(leader, dst + SOFF + h * SB, cu.s, SB, bar);
             cursor_step<SB>(P, cu, 1);
         }
     }
@@ -549,7 +561,10 @@ __device__ __forceinline__ void unit_product_m1(uint32_t sc, uint32_t ss, uint2 
     const uint4 c1 = lds128(sc + off_c + 512);
     const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
     const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
-    float d[4];
+    // two accumulator chains, first halves (even columns) in d, second halves
+    // (odd columns) in e: half the dependent-mma depth, and lane (g, t) reads
+    // column 2t from d and column 2t + 1 from e
+    float d[4], e[4];
 #pragma unroll
     for (int j = 0; j < kSbBlocks; ++j) {
         // code byte b of word cw: logical byte t + 4b of the block
@@ -562,17 +577,27 @@ __device__ __forceinline__ void unit_product_m1(uint32_t sc, uint32_t ss, uint2 
         const uint32_t a12 = lds_lut(prmt(cw0[j], lut_lane, 0x7634u));
         const uint32_t a13 = lds_lut(prmt(cw1[j], lut_lane, 0x7634u));
         const bool p0 = g == 2 * j, p1 = g == 2 * j + 1;
-        if (j == 0)
+        if (j == 0) {
             mma_nv(d, a00, a01, a02, a03, p0 ? xv.x : 0u, p0 ? xv.y : 0u);
-        else
+            mma_nv(e, a10, a11, a12, a13, p1 ? xv.x : 0u, p1 ? xv.y : 0u);
+        } else {
             mma_acc(d, a00, a01, a02, a03, p0 ? xv.x : 0u, p0 ? xv.y : 0u);
-        mma_acc(d, a10, a11, a12, a13, p1 ? xv.x : 0u, p1 ? xv.y : 0u);
+            mma_acc(e, a10, a11, a12, a13, p1 ? xv.x : 0u, p1 ? xv.y : 0u);
+        }
     }
     const float2 sg = CT::block(ss, g, t), sg8 = CT::block(ss, g + 8, t);
     acc[0][0] = fmaf(d[0], sg.x, acc[0][0]);
-    acc[0][1] = fmaf(d[1], sg.y, acc[0][1]);
+    acc[0][1] = fmaf(e[1], sg.y, acc[0][1]);
     acc[0][2] = fmaf(d[2], sg8.x, acc[0][2]);
-    acc[0][3] = fmaf(d[3], sg8.y, acc[0][3]);
+    acc[0][3] = fmaf(e[3], sg8.y, acc[0][3]);
+}
+
+// One-row unit with its activation words already loaded (a no-op for the
+// multi-row kernels, which never take that path).
+template <int NT, bool M1, typename CT>
+__device__ __forceinline__ void unit_xv(uint32_t sc, uint32_t ss, uint2 xv, uint32_t lut_lane, uint32_t off_c, int g,
+                                        int t, float (&acc)[NT][4]) {
+    if constexpr (M1) unit_product_m1<CT>(sc, ss, xv, lut_lane, off_c, g, t, acc);
 }
 
 // One unit's products; the activation fragments of its superblock start at
@@ -635,9 +660,11 @@ __device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0,
 
 template <int NT, bool M1, int OT, int CODEC>
 __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
-    using G = Geometry<warps_for(M1, NT)>;
+    using G = Geometry<warps_for(M1, NT), M1>;
+    using RG = Ring<M1>;
     using CT = CodecTraits<CODEC>;
     constexpr int SB = CT::kScaleBytes;
+    constexpr int kPerStage = RG::kPerStage, kStageBytes = RG::kStageBytes, kStageScaleOff = RG::kStageScaleOff;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gw = blockIdx.x * G::kWarps + warp;
@@ -647,7 +674,7 @@ __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(c
         return;
     }
     const uint32_t ring =
-        warp < G::kLowWarps ? base + warp * kRingWarpBytes : kHighRings + (warp - G::kLowWarps) * kRingWarpBytes;
+        warp < G::kLowWarps ? G::kLowRings + warp * G::kRingWarpBytes : kHighRings + (warp - G::kLowWarps) * G::kRingWarpBytes;
     const uint32_t bars = G::kBarAddr + warp * (kStages * 8);
     const bool active = gw < P.total_warps;
     const int U = (int)P.units;
@@ -670,7 +697,7 @@ __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(c
         for (int i = 0; i < kStages && pv < u1; ++i) {
             const int cnt = min(kPerStage, u1 - pv);
             const bool skip = P.inject_skip && gw == 0 && i == 0;
-            issue_stage<SB>(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0 && !skip);
+            issue_stage<SB, kStageScaleOff>(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0 && !skip);
             pv += cnt;
         }
     }
@@ -758,15 +785,21 @@ __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(c
         }
         const int cnt = min(kPerStage, u1 - u);  // units held by this stage
         if (M1 && cnt == kPerStage && u + kPerStage <= seg_end) {
-            // common one-row case: both units belong to the current tile
-            // segment (the multi-row kernels take the loop below, which keeps
-            // one unit's operands live at a time)
-            unit_any<NT, M1, CT>(st, st + kStageScaleOff, xcur, 0, lut_lane, off_c, off_x, g, t, acc);
-            unit_any<NT, M1, CT>(st + kUnitCodeBytes, st + kStageScaleOff + SB, xcur, 128, lut_lane, off_c, off_x, g,
-                                 t, acc);
+            // common one-row case: every unit of the stage belongs to the
+            // current tile segment; their activation words are loaded first
+            // (the multi-row kernels take the loop below, which keeps one
+            // unit's operands live at a time)
+            const char *xb = reinterpret_cast<const char *>(xcur[0]) + off_x;
+            uint2 xv[kPerStage];
 #pragma unroll
-            for (int a = 0; a < NT; ++a) xcur[a] += 256;
-            u += 2;
+            for (int h = 0; h < kPerStage; ++h) xv[h] = ldg64(xb + 256 * h);  // 128 halves per superblock
+#pragma unroll
+            for (int h = 0; h < kPerStage; ++h)
+                unit_xv<NT, M1, CT>(st + h * kUnitCodeBytes, st + kStageScaleOff + h * SB, xv[h], lut_lane, off_c, g,
+                                    t, acc);
+#pragma unroll
+            for (int a = 0; a < NT; ++a) xcur[a] += 128 * kPerStage;
+            u += kPerStage;
             if (u == seg_end)
                 end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, tag, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
         } else {
@@ -783,7 +816,7 @@ __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(c
         __syncwarp();  // every lane has read the stage: it may be refilled
         if (pv < u1) {
             const int c2 = min(kPerStage, u1 - pv);
-            issue_stage<SB>(P, cu, c2, st, bar, lane == 0);
+            issue_stage<SB, kStageScaleOff>(P, cu, c2, st, bar, lane == 0);
             pv += c2;
         }
         stage = (stage == kStages - 1) ? 0 : stage + 1;
@@ -810,7 +843,7 @@ uint32_t dynamic_smem_base() {
 
 template <int NT, bool M1, int CODEC>
 cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programmatic, cudaStream_t stream) {
-    using G = Geometry<warps_for(M1, NT)>;
+    using G = Geometry<warps_for(M1, NT), M1>;
     const uint32_t smem = G::smem_bytes_for_base(dynamic_smem_base());
     const int kSmemBytes = (int)smem;
     cudaLaunchConfig_t cfg = {};
