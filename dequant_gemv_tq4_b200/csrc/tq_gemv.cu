@@ -60,6 +60,10 @@ namespace {
 // per stage; 17..32 rows: 12 warps, whose three or four accumulator tiles need
 // up to 168 registers without spilling.
 __host__ __device__ constexpr int warps_for(bool one_row, int nt = 1) { return one_row ? 12 : (nt >= 3 ? 12 : 16); }
+// Activation rows per half-block-combination kernel for m rows (1, 2 or 4; 0:
+// the multi-row kernel).  3 rows run the 4-row kernel with the last row
+// repeated (never stored).
+constexpr int combo_rows(int64_t m) { return m == 1 ? 1 : m == 2 ? 2 : (m == 3 || m == 4) ? 4 : 0; }
 constexpr int kStages = 2;  // ring stages per warp
 constexpr int kUnitCodeBytes = 1024;
 constexpr int kUnitScaleBytes = 256;  // TQ4_1S: 16 rows x 4 blocks x 2 fp16; NVFP4 uses 128 (16 x 8 E4M3)
@@ -389,10 +393,33 @@ struct AccTile {
     float v[NT][4];
 };
 
+// Activation row of accumulator v[a][b] of lane (g, t) once a tile segment is
+// complete, or 32 (never below m) for an entry that carries nothing.  CM = 0:
+// the multi-row kernel (column 2t + (b & 1) of n-tile a).  CM = 1, 2, 4: the
+// half-block-combination kernels for 1, 2 and 4 activation rows, whose sums
+// end in entries b = 0 (weight row g) and b = 2 (row g + 8) of the lanes that
+// own an activation row: t = 0 (CM = 1), t = 0 and 2 (CM = 2), every t (CM = 4).
+template <int CM>
+__device__ __forceinline__ int acc_xrow(int a, int b, int t) {
+    if constexpr (CM == 0) return 8 * a + 2 * t + (b & 1);
+    else if constexpr (CM == 1) return (b & 1) ? 32 : 2 * t;
+    else if constexpr (CM == 2) return ((b & 1) || (t & 1)) ? 32 : (t >> 1);
+    else return (b & 1) ? 32 : t;
+}
+
+// Activation row whose fragments lane group g loads (rows past m repeat row
+// m - 1; their results are never stored).  CM = 0: row 8a + g of n-tile a;
+// CM = 1, 2, 4: the activation row of the B column g, g / (8 / CM).
+template <int CM>
+__device__ __forceinline__ int lane_xrow(int a, int g, int m) {
+    if constexpr (CM == 0) return min(8 * a + g, m - 1);
+    else return min(g / (8 / CM), m - 1);
+}
+
 // The first contributor of a split tile: its own sums plus those of warps
 // gw+1 .. last, the owner of the tile's last unit (the largest w with
 // floor(w*U/W) <= x), added in warp order once each word carries the tag.
-template <int NT, bool M1, int OT>
+template <int NT, int CM, int OT>
 __device__ __noinline__ void reduce_first(const GroupParams &P, int q, int r, int tile_hi, int gw, uint32_t tag,
                                           AccTile<NT> acc) {
     constexpr int kMcap = 8 * NT;
@@ -408,8 +435,7 @@ __device__ __noinline__ void reduce_first(const GroupParams &P, int q, int r, in
     for (int a = 0; a < NT; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-            if (M1 && (b & 1)) continue;
-            const int xrow = 8 * a + 2 * t + (b & 1);
+            const int xrow = acc_xrow<CM>(a, b, t);
             const int wl = g + ((b & 2) ? 8 : 0);
             if (xrow >= P.m) continue;
             const uint64_t *src = base + xrow * 16 + wl;
@@ -448,7 +474,7 @@ __device__ __noinline__ void reduce_first(const GroupParams &P, int q, int r, in
 // call tag), with no fence and no atomic, and gw0 adds them (own part first,
 // then warp order: deterministic), polling until each word carries this
 // call's tag.  The wait is bounded in time and reports a timeout.
-template <int NT, bool M1, int OT>
+template <int NT, int CM, int OT>
 __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
                                            int u1, int gw, uint32_t tag, const float (&acc_in)[NT][4]) {
     constexpr int kMcap = 8 * NT;
@@ -467,8 +493,7 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
         for (int a = 0; a < NT; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                if (M1 && (b & 1)) continue;
-                const int xrow = 8 * a + 2 * t + (b & 1);
+                const int xrow = acc_xrow<CM>(a, b, t);
                 const int wrow = (b & 2) ? row_g8 : row_g;
                 if (xrow < P.m && wrow < pr.n)
                     store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, acc[a][b]);
@@ -482,7 +507,7 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
         for (int a = 0; a < NT; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const int xrow = 8 * a + 2 * t + (b & 1);
+                const int xrow = acc_xrow<CM>(a, b, t);
                 const int wrow = g + ((b & 2) ? 8 : 0);
                 if (xrow < P.m) st_relaxed_u64(slot + xrow * 16 + wrow, tag_hi | __float_as_uint(acc[a][b]));
             }
@@ -494,13 +519,13 @@ __device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r
     for (int a = 0; a < NT; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) own.v[a][b] = acc[a][b];
-    reduce_first<NT, M1, OT>(P, q, r, tile_hi, gw, tag, own);
+    reduce_first<NT, CM, OT>(P, q, r, tile_hi, gw, tag, own);
 }
 
 // Products of one unit (16 rows x 128 columns) accumulated into acc: the
 // unit's codes at shared address sc, its scales at ss, the activation
 // fragments at xcur[a] + xoff.
-template <int NT, bool M1, typename CT>
+template <int NT, typename CT>
 __device__ __forceinline__ void unit_product(uint32_t sc, uint32_t ss, const uint16_t *const (&xcur)[NT], int xoff,
                                              uint32_t lut_lane, uint32_t off_c, int g, float (&acc)[NT][4]) {
     const uint4 c0 = lds128(sc + off_c);
@@ -531,17 +556,13 @@ __device__ __forceinline__ void unit_product(uint32_t sc, uint32_t ss, const uin
             mma_nv(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
             acc[a][0] = fmaf(d[0], dg.x, acc[a][0]);
             acc[a][2] = fmaf(d[2], dg8.x, acc[a][2]);
-            if (!M1) {
-                acc[a][1] = fmaf(d[1], dg.x, acc[a][1]);
-                acc[a][3] = fmaf(d[3], dg8.x, acc[a][3]);
-            }
+            acc[a][1] = fmaf(d[1], dg.x, acc[a][1]);
+            acc[a][3] = fmaf(d[3], dg8.x, acc[a][3]);
             mma_nv(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
             acc[a][0] = fmaf(d[0], dg.y, acc[a][0]);
             acc[a][2] = fmaf(d[2], dg8.y, acc[a][2]);
-            if (!M1) {
-                acc[a][1] = fmaf(d[1], dg.y, acc[a][1]);
-                acc[a][3] = fmaf(d[3], dg8.y, acc[a][3]);
-            }
+            acc[a][1] = fmaf(d[1], dg.y, acc[a][1]);
+            acc[a][3] = fmaf(d[3], dg8.y, acc[a][3]);
         }
     }
 }
@@ -592,48 +613,121 @@ __device__ __forceinline__ void unit_product_m1(uint32_t sc, uint32_t ss, uint2 
     acc[0][3] = fmaf(e[3], sg8.y, acc[0][3]);
 }
 
-// One-row unit with its activation words already loaded (a no-op for the
-// multi-row kernels, which never take that path).
-template <int NT, bool M1, typename CT>
-__device__ __forceinline__ void unit_xv(uint32_t sc, uint32_t ss, uint2 xv, uint32_t lut_lane, uint32_t off_c, int g,
-                                        int t, float (&acc)[NT][4]) {
-    if constexpr (M1) unit_product_m1<CT>(sc, ss, xv, lut_lane, off_c, g, t, acc);
+// Two or four activation rows (CM): the eight B columns hold CM rows x S = 8 /
+// CM half-block slots.  Block j of the unit goes to accumulator chain k = j %
+// CM and slot pair u = j / CM (its halves in slots 2u and 2u + 1), so column
+// n = S * row + 2u + h carries half h of block u * CM + k of activation row
+// `row`; the CM chains are independent, 8 / CM dependent MMAs deep each, and
+// keep their half-block sums apart.  Lane (g, t) feeds column g:
+// in chain k it supplies its words of block (g % S) / 2 * CM + k, half g % 2,
+// of activation row g / S (xv[k], loaded by the caller), and zero in the
+// other slots.  It ends with, per chain k, columns 2t and 2t + 1: the two
+// halves of block (t % (S / 2)) * CM + k of activation row 2t / S, which it
+// scales by that block's (d0, d1).
+template <int CM, typename CT>
+__device__ __forceinline__ void unit_product_cm(uint32_t sc, uint32_t ss, const uint2 (&xv)[CM], uint32_t lut_lane,
+                                                uint32_t off_c, int g, int t, float (&acc)[1][4]) {
+    static_assert(CM == 2 || CM == 4, "two or four activation rows");
+    constexpr int S = 8 / CM;
+    const uint4 c0 = lds128(sc + off_c);
+    const uint4 c1 = lds128(sc + off_c + 512);
+    const uint32_t cw0[4] = {c0.x, c0.y, c0.z, c0.w};
+    const uint32_t cw1[4] = {c1.x, c1.y, c1.z, c1.w};
+    const int slot = g % S;  // this lane's B column slot
+    float d[CM][4];
+#pragma unroll
+    for (int j = 0; j < kSbBlocks; ++j) {
+        const uint32_t a00 = lds_lut(prmt(cw0[j], lut_lane, 0x7604u));
+        const uint32_t a01 = lds_lut(prmt(cw1[j], lut_lane, 0x7604u));
+        const uint32_t a02 = lds_lut(prmt(cw0[j], lut_lane, 0x7614u));
+        const uint32_t a03 = lds_lut(prmt(cw1[j], lut_lane, 0x7614u));
+        const uint32_t a10 = lds_lut(prmt(cw0[j], lut_lane, 0x7624u));
+        const uint32_t a11 = lds_lut(prmt(cw1[j], lut_lane, 0x7624u));
+        const uint32_t a12 = lds_lut(prmt(cw0[j], lut_lane, 0x7634u));
+        const uint32_t a13 = lds_lut(prmt(cw1[j], lut_lane, 0x7634u));
+        const int k = j % CM, u = j / CM;
+        const bool p0 = slot == 2 * u, p1 = slot == 2 * u + 1;
+        if (u == 0)
+            mma_nv(d[k], a00, a01, a02, a03, p0 ? xv[k].x : 0u, p0 ? xv[k].y : 0u);
+        else
+            mma_acc(d[k], a00, a01, a02, a03, p0 ? xv[k].x : 0u, p0 ? xv[k].y : 0u);
+        mma_acc(d[k], a10, a11, a12, a13, p1 ? xv[k].x : 0u, p1 ? xv[k].y : 0u);
+    }
+#pragma unroll
+    for (int k = 0; k < CM; ++k) {
+        const int blk = (t % (S / 2)) * CM + k;
+        const float2 sg = CT::block(ss, g, blk), sg8 = CT::block(ss, g + 8, blk);
+        acc[0][0] = fmaf(d[k][0], sg.x, acc[0][0]);
+        acc[0][1] = fmaf(d[k][1], sg.y, acc[0][1]);
+        acc[0][2] = fmaf(d[k][2], sg8.x, acc[0][2]);
+        acc[0][3] = fmaf(d[k][3], sg8.y, acc[0][3]);
+    }
+}
+
+// Activation words a half-block-combination lane needs per unit (CM = 1, 2,
+// 4): one 8-byte word per chain.
+template <int CM>
+struct XWords {
+    uint2 w[CM == 0 ? 1 : CM];
+};
+
+// Half-block-combination unit with its activation words already loaded (a
+// no-op for the multi-row kernels, which never take that path).
+template <int NT, int CM, typename CT>
+__device__ __forceinline__ void unit_xv(uint32_t sc, uint32_t ss, const XWords<CM> &xv, uint32_t lut_lane,
+                                        uint32_t off_c, int g, int t, float (&acc)[NT][4]) {
+    if constexpr (CM == 1) unit_product_m1<CT>(sc, ss, xv.w[0], lut_lane, off_c, g, t, acc);
+    else if constexpr (CM == 2 || CM == 4) unit_product_cm<CM, CT>(sc, ss, xv.w, lut_lane, off_c, g, t, acc);
+}
+
+// The activation words of one unit for a half-block-combination lane: chain k
+// at byte offset 64 k from the lane's first word (xb).
+template <int CM>
+__device__ __forceinline__ XWords<CM> load_xwords(const char *xb) {
+    XWords<CM> xv;
+#pragma unroll
+    for (int k = 0; k < (CM == 0 ? 1 : CM); ++k) xv.w[k] = ldg64(xb + 64 * k);
+    return xv;
 }
 
 // One unit's products; the activation fragments of its superblock start at
 // xcur[a] + xoff.
-template <int NT, bool M1, typename CT>
+template <int NT, int CM, typename CT>
 __device__ __forceinline__ void unit_any(uint32_t sc, uint32_t ss, const uint16_t *const (&xcur)[NT], int xoff,
                                          uint32_t lut_lane, uint32_t off_c, uint32_t off_x, int g, int t,
                                          float (&acc)[NT][4]) {
-    if constexpr (M1) {
-        static_assert(NT == 1, "one activation row uses one n-tile");
-        // this lane's four activation values of half-block g
-        const uint2 xv = ldg64(reinterpret_cast<const char *>(xcur[0] + xoff) + off_x);
-        unit_product_m1<CT>(sc, ss, xv, lut_lane, off_c, g, t, acc);
+    if constexpr (CM > 0) {
+        static_assert(NT == 1, "the half-block-combination kernels use one n-tile");
+        const XWords<CM> xv = load_xwords<CM>(reinterpret_cast<const char *>(xcur[0] + xoff) + off_x);
+        unit_xv<NT, CM, CT>(sc, ss, xv, lut_lane, off_c, g, t, acc);
     } else {
-        unit_product<NT, M1, CT>(sc, ss, xcur, xoff, lut_lane, off_c, g, acc);
+        unit_product<NT, CT>(sc, ss, xcur, xoff, lut_lane, off_c, g, acc);
     }
 }
 
 // The tile segment ending at unit u is complete: write it out, reset the
 // accumulators and move the segment state to the tile of unit u.
-template <int NT, bool M1, int OT, int CODEC>
+template <int NT, int CM, int OT, int CODEC>
 __device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0, int u1, int gw, int g, int t,
                                          uint32_t tag, int &q,
                                          int &prob_end, int &nsb, int &r, int &tile_lo, int &seg_end,
                                          const uint16_t *(&xcur)[NT], float (&acc)[NT][4]) {
-    if constexpr (M1) {
-        // rows g, g + 8: add the two halves, then the four blocks (lanes t)
+    if constexpr (CM > 0) {
+        // weight rows g, g + 8: add the two halves, then the blocks the lanes
+        // of one activation row share (four lanes for CM = 1, two for CM = 2)
         float vg = acc[0][0] + acc[0][1], vg8 = acc[0][2] + acc[0][3];
-        vg += __shfl_xor_sync(kFull, vg, 1);
-        vg8 += __shfl_xor_sync(kFull, vg8, 1);
-        vg += __shfl_xor_sync(kFull, vg, 2);
-        vg8 += __shfl_xor_sync(kFull, vg8, 2);
+        if constexpr (CM <= 2) {
+            vg += __shfl_xor_sync(kFull, vg, 1);
+            vg8 += __shfl_xor_sync(kFull, vg8, 1);
+        }
+        if constexpr (CM == 1) {
+            vg += __shfl_xor_sync(kFull, vg, 2);
+            vg8 += __shfl_xor_sync(kFull, vg8, 2);
+        }
         acc[0][0] = vg;
         acc[0][2] = vg8;
     }
-    flush_segment<NT, M1, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, tag, acc);
+    flush_segment<NT, CM, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, tag, acc);
 #pragma unroll
     for (int a = 0; a < NT; ++a)
 #pragma unroll
@@ -652,16 +746,16 @@ __device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0,
         seg_end = min(tile_lo + nsb, u1);
 #pragma unroll
         for (int a = 0; a < NT; ++a) {  // back to superblock 0 of the activation
-            const int xrow = min(8 * a + g, P.m - 1);
+            const int xrow = lane_xrow<CM>(a, g, P.m);
             xcur[a] = P.prob[q].xrot + (int64_t)xrow * nsb * 128 + t * 8;
         }
     }
 }
 
-template <int NT, bool M1, int OT, int CODEC>
-__global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
-    using G = Geometry<warps_for(M1, NT), M1>;
-    using RG = Ring<M1>;
+template <int NT, int CM, int OT, int CODEC>
+__global__ void __launch_bounds__(warps_for(CM > 0, NT) * 32, 1) gemv_group_kernel(const __grid_constant__ GroupParams P) {
+    using G = Geometry<warps_for(CM > 0, NT), (CM > 0)>;
+    using RG = Ring<(CM > 0)>;
     using CT = CodecTraits<CODEC>;
     constexpr int SB = CT::kScaleBytes;
     constexpr int kPerStage = RG::kPerStage, kStageBytes = RG::kStageBytes, kStageScaleOff = RG::kStageScaleOff;
@@ -725,10 +819,12 @@ __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(c
     const uint32_t lut_lane = kLutAddr | ((uint32_t)lane * 4u);
     // this lane's 16 code bytes of rows g and g+8 in a unit
     const uint32_t off_c = g * 64 + t * 16;
-    // one activation row: byte offset of this lane's 8 bytes of half-block g
-    // (block g/2, half g%2) in a superblock's fragments [4 blocks][4 t][8
-    // halves], relative to xcur (which already holds t)
-    const uint32_t off_x = (g >> 1) * 64 + (g & 1) * 8;
+    // half-block-combination kernels: byte offset of this lane's first 8-byte
+    // activation word (block (g % S) / 2 * CM, half g % 2, S = 8 / CM) in a
+    // superblock's fragments [4 blocks][4 t][8 halves], relative to xcur
+    // (which already holds t); chain k adds 64 k
+    constexpr int kSlots = 8 / (CM == 0 ? 1 : CM);
+    const uint32_t off_x = ((g % kSlots) >> 1) * (CM == 0 ? 1 : CM) * 64 + (g & 1) * 8;
 
     // ---- segment state: the tile the current unit belongs to ---------------
     int q = problem_of(P, u0);
@@ -748,7 +844,7 @@ __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(c
     const uint16_t *xcur[NT];
 #pragma unroll
     for (int a = 0; a < NT; ++a) {
-        const int xrow = min(8 * a + g, P.m - 1);
+        const int xrow = lane_xrow<CM>(a, g, P.m);
         xcur[a] = P.prob[q].xrot + ((int64_t)xrow * nsb + sb) * 128 + t * 8;
     }
 
@@ -784,33 +880,33 @@ __global__ void __launch_bounds__(warps_for(M1, NT) * 32, 1) gemv_group_kernel(c
             }
         }
         const int cnt = min(kPerStage, u1 - u);  // units held by this stage
-        if (M1 && cnt == kPerStage && u + kPerStage <= seg_end) {
-            // common one-row case: every unit of the stage belongs to the
-            // current tile segment; their activation words are loaded first
-            // (the multi-row kernels take the loop below, which keeps one
-            // unit's operands live at a time)
+        if (CM > 0 && cnt == kPerStage && u + kPerStage <= seg_end) {
+            // common half-block-combination case: every unit of the stage
+            // belongs to the current tile segment; their activation words are
+            // loaded first (the multi-row kernels take the loop below, which
+            // keeps one unit's operands live at a time)
             const char *xb = reinterpret_cast<const char *>(xcur[0]) + off_x;
-            uint2 xv[kPerStage];
+            XWords<CM> xv[kPerStage];
 #pragma unroll
-            for (int h = 0; h < kPerStage; ++h) xv[h] = ldg64(xb + 256 * h);  // 128 halves per superblock
+            for (int h = 0; h < kPerStage; ++h) xv[h] = load_xwords<CM>(xb + 256 * h);  // 128 halves per superblock
 #pragma unroll
             for (int h = 0; h < kPerStage; ++h)
-                unit_xv<NT, M1, CT>(st + h * kUnitCodeBytes, st + kStageScaleOff + h * SB, xv[h], lut_lane, off_c, g,
+                unit_xv<NT, CM, CT>(st + h * kUnitCodeBytes, st + kStageScaleOff + h * SB, xv[h], lut_lane, off_c, g,
                                     t, acc);
 #pragma unroll
             for (int a = 0; a < NT; ++a) xcur[a] += 128 * kPerStage;
             u += kPerStage;
             if (u == seg_end)
-                end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, tag, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
+                end_segment<NT, CM, OT, CODEC>(P, u, u0, u1, gw, g, t, tag, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
         } else {
             for (int h = 0; h < cnt; ++h) {
-                unit_any<NT, M1, CT>(st + h * kUnitCodeBytes, st + kStageScaleOff + h * SB, xcur, 0, lut_lane, off_c,
+                unit_any<NT, CM, CT>(st + h * kUnitCodeBytes, st + kStageScaleOff + h * SB, xcur, 0, lut_lane, off_c,
                                      off_x, g, t, acc);
 #pragma unroll
                 for (int a = 0; a < NT; ++a) xcur[a] += 128;
                 ++u;
                 if (u == seg_end)
-                    end_segment<NT, M1, OT, CODEC>(P, u, u0, u1, gw, g, t, tag, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
+                    end_segment<NT, CM, OT, CODEC>(P, u, u0, u1, gw, g, t, tag, q, prob_end, nsb, r, tile_lo, seg_end, xcur, acc);
             }
         }
         __syncwarp();  // every lane has read the stage: it may be refilled
@@ -841,9 +937,9 @@ uint32_t dynamic_smem_base() {
     return cached[dev];
 }
 
-template <int NT, bool M1, int CODEC>
+template <int NT, int CM, int CODEC>
 cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programmatic, cudaStream_t stream) {
-    using G = Geometry<warps_for(M1, NT), M1>;
+    using G = Geometry<warps_for(CM > 0, NT), (CM > 0)>;
     const uint32_t smem = G::smem_bytes_for_base(dynamic_smem_base());
     const int kSmemBytes = (int)smem;
     cudaLaunchConfig_t cfg = {};
@@ -859,20 +955,20 @@ cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programm
     cudaError_t err;
     switch (dtype) {
         case kF32:
-            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kF32, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(gemv_group_kernel<NT, CM, kF32, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
             if (err != cudaSuccess) return err;
-            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kF32, CODEC>, prm);
+            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, CM, kF32, CODEC>, prm);
         case kBF16:
-            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kBF16, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(gemv_group_kernel<NT, CM, kBF16, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
             if (err != cudaSuccess) return err;
-            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kBF16, CODEC>, prm);
+            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, CM, kBF16, CODEC>, prm);
         case kF16:
-            err = cudaFuncSetAttribute(gemv_group_kernel<NT, M1, kF16, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(gemv_group_kernel<NT, CM, kF16, CODEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
             if (err != cudaSuccess) return err;
-            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, M1, kF16, CODEC>, prm);
+            return cudaLaunchKernelEx(&cfg, gemv_group_kernel<NT, CM, kF16, CODEC>, prm);
         default:
             return cudaErrorInvalidValue;
     }
@@ -888,8 +984,9 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
         pl.tiles += tiles(n[i]);
         pl.units += tiles(n[i]) * superblocks(k[i]);
     }
-    // one activation row runs the one-row kernel (see launch_group_codec)
-    const int kWarps = warps_for(m == 1, (int)((m > 32 ? 32 : (m < 1 ? 1 : m)) + 7) / 8);
+    // up to four activation rows run a half-block-combination kernel (see
+    // launch_group_codec)
+    const int kWarps = warps_for(combo_rows(m) > 0, (int)((m > 32 ? 32 : (m < 1 ? 1 : m)) + 7) / 8);
     int64_t want = (pl.units + kWarps - 1) / kWarps;  // at least one unit per warp
     if (want > sm_count) want = sm_count;
     if (want < 1) want = 1;
@@ -936,15 +1033,17 @@ cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, i
     prm.timeout_ns = prm.inject_skip ? kDebugTimeoutNs : kTimeoutNs;
     // the partial-slot stride is 16 * 8 * NT floats: NT must match plan.mcap
     const int nt = plan.mcap / 8;
-    const bool one_row = m == 1 && nt == 1;
+    const int cm = nt == 1 ? combo_rows(m) : 0;
     // the plan's warps must all exist in the launched grid
-    if (plan.total_warps > (int64_t)plan.grid * warps_for(one_row, nt)) return cudaErrorInvalidValue;
-    if (one_row) return launch_nt<1, true, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+    if (plan.total_warps > (int64_t)plan.grid * warps_for(cm > 0, nt)) return cudaErrorInvalidValue;
+    if (cm == 1) return launch_nt<1, 1, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+    if (cm == 2) return launch_nt<1, 2, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+    if (cm == 4) return launch_nt<1, 4, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
     switch (nt) {
-        case 1: return launch_nt<1, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
-        case 2: return launch_nt<2, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
-        case 3: return launch_nt<3, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
-        case 4: return launch_nt<4, false, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+        case 1: return launch_nt<1, 0, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+        case 2: return launch_nt<2, 0, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+        case 3: return launch_nt<3, 0, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
+        case 4: return launch_nt<4, 0, CODEC>(prm, ydtype, plan.grid, programmatic, stream);
         default: return cudaErrorInvalidValue;
     }
 }

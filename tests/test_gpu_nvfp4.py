@@ -120,7 +120,8 @@ def test_nvfp4_dequantize_within_bound(cuda_lib, n, k, out_dtype):
 
 
 GEMM_CASES = [(1, 1, 32), (1, 17, 4096), (1, 1024, 4096), (2, 33, 256), (5, 40, 1024), (8, 16, 8192),
-              (16, 100, 384), (16, 300, 1056), (31, 17, 1024), (32, 64, 2048)]
+              (16, 100, 384), (16, 300, 1056), (31, 17, 1024), (32, 64, 2048),
+              (2, 40, 4096), (3, 100, 2048), (4, 17, 8192)]
 
 
 @pytest.mark.parametrize("m,n,k", GEMM_CASES)

@@ -149,6 +149,8 @@ GEMM_CASES = [
     (1, 1, 32), (1, 15, 96), (1, 16, 128), (1, 17, 4096), (1, 1024, 4096), (2, 33, 256), (3, 64, 160),
     (5, 40, 1024), (8, 16, 8192), (9, 48, 512), (16, 100, 384), (31, 17, 1024), (32, 64, 2048),
     (33, 20, 256), (40, 64, 128), (4, 3, 16384), (20, 50, 640), (24, 33, 1056), (17, 300, 4096),
+    # two to four rows: the half-block-combination kernels, with split tiles and ragged edges
+    (2, 1, 32), (2, 40, 4096), (3, 100, 2048), (4, 17, 8192), (4, 300, 640), (3, 2000, 160),
 ]
 
 
@@ -287,7 +289,7 @@ def test_ffn_70b_skinny_sweep_full_size(cuda_lib, m):
     assert _rel_l2(Y.cpu().numpy()[:, rows], Y_ref).max() <= REL_L2_TOL
 
 
-@pytest.mark.parametrize("m", [1, 5])
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5])
 def test_gemm_batch_shares_prerotation(cuda_lib, m):
     """Six matrices with three distinct inputs in one batch (q/k/v-style and
     gate/up-style sharing) against the oracle and the one-matrix path."""
