@@ -37,9 +37,11 @@
 //    columns idle.  Instead column c carries half-block c of the superblock
 //    (four blocks x two halves): the B fragment is the activation in the four
 //    lanes of column c and zero elsewhere, so the eight mmas of a unit chain
-//    into one accumulator whose columns stay separate half-block sums.  Each
+//    into accumulators whose columns stay separate half-block sums.  Each
 //    lane then applies two scales per row pair per unit (not sixteen), and the
-//    four lanes of a row add their blocks once per tile.
+//    four lanes of a row add their blocks once per tile.  Two and four
+//    activation rows share the eight columns the same way (four and two
+//    half-block slots per row).
 //  * Tiles split across warps combine fixed-order partial sums: the later
 //    contributors store (value, call tag) words without fences or atomics,
 //    and the tile's first warp, which reaches its part of the tile last, adds
