@@ -513,33 +513,53 @@ __global__ void __launch_bounds__(256) prerotate_plain_kernel(const __grid_const
         R.header[kHeaderStatus] = 0u;
         R.header[kHeaderTag] += 1u;
     }
+    // Warp w owns superblock w % nsb of every (w / nsb + i * groups)-th row,
+    // groups = (warps in the grid) / nsb >= 1: the lane's sign masks are
+    // computed once, and each step loads kRows rows before rotating any, so
+    // several loads per lane are in flight.
+    constexpr int kRows = 4;
     const int lane = threadIdx.x & 31;
     const int j = lane >> 3, p = lane & 7;
-    const int64_t warps = (int64_t)gridDim.x * 8;
-    for (int64_t wu = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); wu < R.m * R.nsb; wu += warps) {
-        const int64_t row = wu / R.nsb;
-        const int sb = (int)(wu - row * R.nsb);
-        const uint32_t col0 = (uint32_t)sb * 128u + 32u * j + 4u * p;
-        const bool valid = (int)col0 < R.k;  // k is a multiple of 32: whole blocks
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) load4<DT>(R.x + (row * R.ldx + col0) * ElemSize<DT>::value, v);
+    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int64_t groups = (int64_t)gridDim.x * 8 / R.nsb;
+    const int64_t r0 = gw / R.nsb;
+    if (r0 >= groups) return;  // past the last whole set of superblocks (warp-uniform)
+    const int sb = (int)(gw - r0 * R.nsb);
+    const uint32_t col0 = (uint32_t)sb * 128u + 32u * j + 4u * p;
+    const bool valid = (int)col0 < R.k;  // k is a multiple of 32: whole blocks
+    uint32_t msk[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = flip(v[i], sign_mask(col0 + i));
-        butterfly_local4(v);
+    for (int i = 0; i < 4; ++i) msk[i] = sign_mask(col0 + i);
+    for (int64_t row = r0; row < R.m; row += kRows * groups) {
+        float v[kRows][4];
 #pragma unroll
-        for (int st = 0; st < 3; ++st) {
-            const int xo = 1 << st;
-            const bool upper = (p & xo) != 0;
+        for (int u = 0; u < kRows; ++u) {
+            const int64_t r = row + u * groups;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = butterfly_xlane(v[i], xo, upper);
+            for (int i = 0; i < 4; ++i) v[u][i] = 0.f;
+            if (valid && r < R.m) load4<DT>(R.x + (r * R.ldx + col0) * ElemSize<DT>::value, v[u]);
         }
-        if (valid) {
-            const __half2 lo = __floats2half2_rn(__fmul_rn(v[0], 0.03125f), __fmul_rn(v[1], 0.03125f));
-            const __half2 hi = __floats2half2_rn(__fmul_rn(v[2], 0.03125f), __fmul_rn(v[3], 0.03125f));
-            uint2 o;
-            o.x = *reinterpret_cast<const uint32_t *>(&lo);
-            o.y = *reinterpret_cast<const uint32_t *>(&hi);
-            *reinterpret_cast<uint2 *>(R.xrot + row * R.k + col0) = o;
+#pragma unroll
+        for (int u = 0; u < kRows; ++u) {
+            const int64_t r = row + u * groups;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[u][i] = flip(v[u][i], msk[i]);
+            butterfly_local4(v[u]);
+#pragma unroll
+            for (int st = 0; st < 3; ++st) {
+                const int xo = 1 << st;
+                const bool upper = (p & xo) != 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) v[u][i] = butterfly_xlane(v[u][i], xo, upper);
+            }
+            if (valid && r < R.m) {
+                const __half2 lo = __floats2half2_rn(__fmul_rn(v[u][0], 0.03125f), __fmul_rn(v[u][1], 0.03125f));
+                const __half2 hi = __floats2half2_rn(__fmul_rn(v[u][2], 0.03125f), __fmul_rn(v[u][3], 0.03125f));
+                uint2 o;
+                o.x = *reinterpret_cast<const uint32_t *>(&lo);
+                o.y = *reinterpret_cast<const uint32_t *>(&hi);
+                *reinterpret_cast<uint2 *>(R.xrot + r * R.k + col0) = o;
+            }
         }
     }
 }
@@ -599,10 +619,17 @@ cudaError_t launch_prefill_kernel(const CUtensorMap &map, const PrefillParams &p
 
 template <int DT>
 cudaError_t launch_plain_rotation(const PlainRotParams &r, cudaStream_t stream) {
-    const int64_t warps = r.m * r.nsb;
-    int64_t grid = (warps + 7) / 8;
-    if (grid > 148 * 16) grid = 148 * 16;
-    if (grid < 1) grid = 1;
+    // one (row, superblock) step per warp and four rows per step at most,
+    // about one resident wave (8 CTAs of 8 warps per SM), and at least one
+    // warp per superblock
+    DeviceInfo di;
+    const cudaError_t err = device_info(&di);
+    if (err != cudaSuccess) return err;
+    int64_t grid = (r.m * r.nsb + 31) / 32;
+    if (grid > (int64_t)di.sm_count * 8) grid = (int64_t)di.sm_count * 8;
+    const int64_t min_grid = (r.nsb + 7) / 8;
+    if (grid < min_grid) grid = min_grid;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(256);
