@@ -32,7 +32,9 @@
 //    pre-rotated activation fragment (X rows as the n dimension, 8 per mma,
 //    NT n-tiles for m <= 8*NT).  One k16 step is exactly one half-block, so the
 //    fp16 half-block scale multiplies the fp32 mma result before it joins the
-//    accumulator.
+//    accumulator; with four n-tiles (m > 24) it multiplies the decoded
+//    centroids instead (fp16(c * d), shared by the n-tiles) and the mmas
+//    accumulate directly.
 //  * One activation row (the decode case) would leave seven of the eight mma
 //    columns idle.  Instead column c carries half-block c of the superblock
 //    (four blocks x two halves): the B fragment is the activation in the four
@@ -177,6 +179,12 @@ __device__ __forceinline__ void mma_acc(float (&d)[4], uint32_t a0, uint32_t a1,
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// fp16x2 product, round to nearest even
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     uint32_t v;
@@ -341,9 +349,11 @@ struct CodecTraits<kCodecTQ4> {
     __device__ static uint4 load(uint32_t ss, int row) { return lds128(ss + row * 16); }
     // (scale of half 0, scale of half 1) of 32-column block j
     __device__ static float2 pair(const uint4 &w, int j) {
-        const uint32_t v = j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w;
+        const uint32_t v = pair_h2(w, j);
         return __half22float2(*reinterpret_cast<const __half2 *>(&v));
     }
+    // the same pair as one fp16x2 word
+    __device__ static uint32_t pair_h2(const uint4 &w, int j) { return j == 0 ? w.x : j == 1 ? w.y : j == 2 ? w.z : w.w; }
     // (d0, d1) of block j of row `row`
     __device__ static float2 block(uint32_t ss, int row, int j) {
         const uint32_t v = lds32(ss + row * 16 + j * 4);
@@ -363,11 +373,16 @@ struct CodecTraits<kCodecNVFP4> {
     }
     // 32-column block j covers 16-element blocks 2j (half 0) and 2j+1 (half 1)
     __device__ static float2 pair(const uint4 &w, int j) {
+        const uint32_t h = pair_h2(w, j);
+        return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+    }
+    // the same pair as one fp16x2 word (E4M3 values are exact in fp16)
+    __device__ static uint32_t pair_h2(const uint4 &w, int j) {
         const uint32_t word = (j < 2) ? w.x : w.y;
         const uint16_t two = (uint16_t)(word >> (16 * (j & 1)));
         uint32_t h;
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
-        return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+        return h;
     }
     // block scales of the two halves of 32-column block j of row `row`
     __device__ static float2 block(uint32_t ss, int row, int j) {
@@ -550,21 +565,39 @@ __device__ __forceinline__ void unit_product(uint32_t sc, uint32_t ss, const uin
         const uint32_t a11 = lds_lut(prmt(cw1[j], lut_lane, 0x7624u));
         const uint32_t a12 = lds_lut(prmt(cw0[j], lut_lane, 0x7634u));
         const uint32_t a13 = lds_lut(prmt(cw1[j], lut_lane, 0x7634u));
-        const float2 dg = CT::pair(s0, j);
-        const float2 dg8 = CT::pair(s1, j);
+        if constexpr (NT >= 4) {
+            // four n-tiles share A: scale the decoded centroids once, fp16(c *
+            // d) (the prefill kernel's operand), and let the tensor cores
+            // accumulate every half-block in fp32 (no FFMA per n-tile; with
+            // fewer n-tiles the dependent-mma chains this makes cost more than
+            // the FFMAs they save)
+            const uint32_t pg = CT::pair_h2(s0, j), pg8 = CT::pair_h2(s1, j);
+            const uint32_t g0 = prmt(pg, pg, 0x1010u), g1 = prmt(pg, pg, 0x3232u);    // (d0, d0), (d1, d1) of row g
+            const uint32_t e0 = prmt(pg8, pg8, 0x1010u), e1 = prmt(pg8, pg8, 0x3232u);  // the same for row g + 8
+            const uint32_t b00 = hmul2(a00, g0), b01 = hmul2(a01, e0), b02 = hmul2(a02, g0), b03 = hmul2(a03, e0);
+            const uint32_t b10 = hmul2(a10, g1), b11 = hmul2(a11, e1), b12 = hmul2(a12, g1), b13 = hmul2(a13, e1);
 #pragma unroll
-        for (int a = 0; a < NT; ++a) {
-            float d[4];
-            mma_nv(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
-            acc[a][0] = fmaf(d[0], dg.x, acc[a][0]);
-            acc[a][2] = fmaf(d[2], dg8.x, acc[a][2]);
-            acc[a][1] = fmaf(d[1], dg.x, acc[a][1]);
-            acc[a][3] = fmaf(d[3], dg8.x, acc[a][3]);
-            mma_nv(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
-            acc[a][0] = fmaf(d[0], dg.y, acc[a][0]);
-            acc[a][2] = fmaf(d[2], dg8.y, acc[a][2]);
-            acc[a][1] = fmaf(d[1], dg.y, acc[a][1]);
-            acc[a][3] = fmaf(d[3], dg8.y, acc[a][3]);
+            for (int a = 0; a < NT; ++a) {
+                mma_acc(acc[a], b00, b01, b02, b03, xb[a].x, xb[a].y);
+                mma_acc(acc[a], b10, b11, b12, b13, xb[a].z, xb[a].w);
+            }
+        } else {
+            const float2 dg = CT::pair(s0, j);
+            const float2 dg8 = CT::pair(s1, j);
+#pragma unroll
+            for (int a = 0; a < NT; ++a) {
+                float d[4];
+                mma_nv(d, a00, a01, a02, a03, xb[a].x, xb[a].y);
+                acc[a][0] = fmaf(d[0], dg.x, acc[a][0]);
+                acc[a][2] = fmaf(d[2], dg8.x, acc[a][2]);
+                acc[a][1] = fmaf(d[1], dg.x, acc[a][1]);
+                acc[a][3] = fmaf(d[3], dg8.x, acc[a][3]);
+                mma_nv(d, a10, a11, a12, a13, xb[a].z, xb[a].w);
+                acc[a][0] = fmaf(d[0], dg.y, acc[a][0]);
+                acc[a][2] = fmaf(d[2], dg8.y, acc[a][2]);
+                acc[a][1] = fmaf(d[1], dg.y, acc[a][1]);
+                acc[a][3] = fmaf(d[3], dg8.y, acc[a][3]);
+            }
         }
     }
 }
