@@ -97,6 +97,14 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# Operations the TQ4_1S codec defines per 32-element block when it quantises:
+# sign flip 32, five butterfly stages 5 x 32, half-block RMS (32 squares, 2 x
+# 15 adds, 2 x (scale by 1/16, square root, fp16 rounding)) 68, thresholds
+# scaled by each half's scale 2 x 7, three threshold compares and the sign
+# test per element 4 x 32, one nibble insert per element 32: 434 per block.
+QUANT_OPS_PER_WEIGHT = 434 / 32
+LANES_PER_SM = 128  # fp32 / integer lanes of one SM (4 partitions x 32)
+
 PROFILE_FILES = {  # phase -> committed ncu summary and the sources its kernel is built from
     "quantize": ("quantize_kernel_llama3_8b_down.md", ("tq_device.cuh", "tq_codec.cu")),
     "dequantize": ("dequantize_kernel_llama3_8b_down.md", ("tq_device.cuh", "tq_codec.cu")),
@@ -480,6 +488,20 @@ def run_ours(args, world, rank, local):
                          "frac": round(ach / hbm, 4), "traffic": profile_traffic(ph, weights),
                          "bytes_per_step": nbytes, "ms": round(ms, 5), "launches": nl}
     dominant = max(("quantize", "dequantize", "gemv"), key=lambda ph: alg[ph][1])
+    # the quantise kernel is bound by its arithmetic, not by HBM: its ALU
+    # roofline counts the codec's defined operations against every lane of
+    # every SM at the highest SM clock seen
+    props = torch.cuda.get_device_properties(device)
+    max_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    alu_peak = props.multi_processor_count * LANES_PER_SM * max_mhz * 1e6 / 1e12
+    alu_ach = QUANT_OPS_PER_WEIGHT * weights / (ms_q * 1e-3) / 1e12
+    rooflines["quantize_alu"] = {"bound": "alu", "achieved": round(alu_ach, 3), "peak": round(alu_peak, 3),
+                                 "unit": "Tops/s", "frac": round(alu_ach / alu_peak, 4),
+                                 "traffic": rooflines["quantize"]["traffic"],
+                                 "ops_per_weight": round(QUANT_OPS_PER_WEIGHT, 4), "ms": round(ms_q, 5),
+                                 "peak_note": f"{props.multi_processor_count} SMs x {LANES_PER_SM} lanes x "
+                                              f"{max_mhz:.0f} MHz, one operation per lane per cycle"}
+    top = rooflines["quantize_alu"] if dominant == "quantize" else rooflines[dominant]
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps,
@@ -497,7 +519,8 @@ def run_ours(args, world, rank, local):
         "quantize_gweights_per_s": round(quant_gw, 2),
         "phases_ms": {"quantize": round(ms_q, 5), "dequantize": round(ms_d, 5), "gemv": round(ms_g, 5)},
         "gemv_single_matrix": per_matrix,
-        "roofline": dict(rooflines[dominant], kernel=dominant, peak_note=f"{hbm_kind} HBM copy bandwidth"),
+        "roofline": dict(top, kernel=dominant, **({} if dominant == "quantize" else
+                                                  {"peak_note": f"{hbm_kind} HBM copy bandwidth"})),
         "rooflines": rooflines,
         "clocks": clocks,
         "gpu_launches": launches_per_step * steps * R,
