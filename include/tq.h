@@ -157,7 +157,10 @@ TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * tq_gemm -- Y[i][r] = sum_k w~[r][k] X[i][k] for i < m, r < n, computed as
  * (1/32) sum_blocks sum_halves d * sum_e c_e xrot_e with the activation
  * pre-rotated once per call (TQ page, 解码速度 section).  Centroids and xrot
- * enter the tensor cores as fp16; products accumulate in fp32.
+ * enter the tensor cores as fp16; products accumulate in fp32.  For m = 25..32
+ * (and in the prefill product) the centroid enters already multiplied by its
+ * half-block scale, fp16(c * d), which overflows once d exceeds about 23,970
+ * (weights of magnitude around 4,000 and up).
  *   X          device, m x k of dtype xt, row stride ldx (as tq_prerotate)
  *   Y          device, m x n of dtype yt (F32, BF16 or F16), row stride ldy
  *              (ldy >= n)
