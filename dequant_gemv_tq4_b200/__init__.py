@@ -85,6 +85,7 @@ def load_library() -> ctypes.CDLL:
             "tq_workspace_status": ([P, I, P], I),
             "tq_debug_set_flags": ([ctypes.c_uint32], None),
             "tq_gemv_static_scratch": ([P, P, I64, I64, P, I, P, I, P], I),
+            "tq_static_scratch_status": ([I, P], I),
             "tq_gemm_prefill_workspace_bytes": ([I64, I64], SZ),
             "tq_gemm_prefill": ([P, P, I64, I64, P, I, I64, I64, P, I, I64, P, SZ, P], I),
             "tq_prefill_xrot_bytes": ([I64, I64], SZ),
@@ -178,6 +179,11 @@ def tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream) -> int:
     device memory: the scratch is a fixed array inside the library (see
     include/tq.h).  Calls that overlap on the GPU must not share it."""
     return load_library().tq_gemv_static_scratch(codes, scales, n, k, x, xt, y, yt, stream)
+
+
+def tq_static_scratch_status(clear, stream) -> int:
+    """Timeout flag of the last tq_gemv_static_scratch call (synchronises)."""
+    return load_library().tq_static_scratch_status(clear, stream)
 
 
 def tq_gemm_prefill_workspace_bytes(m: int, k: int) -> int:

@@ -514,24 +514,64 @@ namespace {
 static __device__ __align__(256) unsigned char g_static_scratch[TQ_STATIC_SCRATCH_BYTES];
 
 std::mutex g_scratch_mu;
-void *g_scratch_ptr[256];
+struct ScratchAddr {
+    unsigned long long ctx_id;  // the context the address belongs to (0: none yet)
+    void *ptr;
+};
+ScratchAddr g_scratch_addr[256];
 
-// Device address of g_static_scratch on the current device.  In host code the
+using CtxGetCurrent = int (*)(void **);
+using CtxGetId = int (*)(void *, unsigned long long *);
+
+// Unique id of the calling thread's current context (cuCtxGetId through the
+// runtime's driver entry point, no link to the driver library).  A device
+// reset or another context on the same device yields a new id.
+cudaError_t current_context_id(unsigned long long *id) {
+    static std::once_flag once;
+    static CtxGetCurrent get_current = nullptr;
+    static CtxGetId get_id = nullptr;
+    std::call_once(once, [] {
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa = cudaDriverEntryPointSymbolNotFound, qb = qa;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<CtxGetCurrent>(a);
+            get_id = reinterpret_cast<CtxGetId>(b);
+        }
+    });
+    if (!get_current || !get_id) return cudaErrorNotSupported;
+    void *ctx = nullptr;
+    if (get_current(&ctx) != 0 || !ctx) return cudaErrorDeviceUninitialized;
+    return get_id(ctx, id) == 0 ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
+
+// Device address of g_static_scratch in the current context.  In host code the
 // array's name is only a host-side stand-in, so the address is asked from the
-// runtime, once per device, with that device current.
+// runtime with the device current, once per context: the cache is keyed by
+// the context's unique id, so a device reset (which reloads the module, and
+// may place the array elsewhere) or a different context on the same device
+// looks the address up again.
 cudaError_t static_scratch_address(void **out) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        err = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (err != cudaSuccess) return err;
-        g_scratch_ptr[dev] = p;
+    unsigned long long id = 0;
+    void *p = nullptr;
+    if (current_context_id(&id) != cudaSuccess) {
+        // no current context yet: the runtime creates the device's primary
+        // context on its first call, here the address lookup itself
+        if ((err = cudaGetSymbolAddress(&p, g_static_scratch)) != cudaSuccess) return err;
+        if ((err = current_context_id(&id)) != cudaSuccess) return err;
+        g_scratch_addr[dev] = {id, p};
+    } else if (g_scratch_addr[dev].ctx_id != id || !g_scratch_addr[dev].ptr) {
+        if ((err = cudaGetSymbolAddress(&p, g_static_scratch)) != cudaSuccess) return err;
+        g_scratch_addr[dev] = {id, p};
     }
-    *out = g_scratch_ptr[dev];
+    *out = g_scratch_addr[dev].ptr;
     return cudaSuccess;
 }
 
@@ -560,4 +600,10 @@ extern "C" tq_status tq_gemv_static_scratch(const uint8_t *codes, const uint16_t
     e = tq::launch_group(&pb, 1, 1, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
                          reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
     return from_cuda(e);
+}
+
+extern "C" tq_status tq_static_scratch_status(int clear, void *stream) {
+    void *scratch = nullptr;
+    if (static_scratch_address(&scratch) != cudaSuccess) return TQ_ERR_CUDA;
+    return tq_workspace_status(scratch, clear, stream);
 }

@@ -982,11 +982,17 @@ cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programm
     cfg.blockDim = dim3(G::kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    // Cooperative: the whole grid (at most one CTA per SM) is resident at
+    // once, which the split-tile reduction relies on (a tile's first warp
+    // polls for the partial sums of later CTAs; a CTA that could not start
+    // until the first one exited would make that poll run out).
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = programmatic ? 1 : 0;
+    cfg.numAttrs = programmatic ? 2 : 1;
     cudaError_t err;
     switch (dtype) {
         case kF32:
@@ -1012,6 +1018,7 @@ cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programm
 }  // namespace
 
 void set_debug_flags(uint32_t flags) { g_debug_flags = flags; }
+uint32_t debug_flags() { return g_debug_flags; }
 
 GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, int sm_count) {
     GroupPlan pl = {};

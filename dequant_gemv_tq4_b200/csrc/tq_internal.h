@@ -93,9 +93,13 @@ struct GroupPlan {
 
 GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, int sm_count);
 
-// Debug hooks (tq_debug_set_flags): bit 0 makes one bulk copy go missing so
-// the kernel's bounded wait expires and reports a timeout.
+// Debug hooks (tq_debug_set_flags): bit 0 makes one bulk copy of the fused
+// GEMV go missing, bit 1 one activation-tile copy of the prefill product, so
+// that the kernel's bounded wait expires and reports a timeout.
+constexpr uint32_t kDebugSkipGemvCopy = 1u;
+constexpr uint32_t kDebugSkipPrefillCopy = 2u;
 void set_debug_flags(uint32_t flags);
+uint32_t debug_flags();
 
 cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
                          unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream);

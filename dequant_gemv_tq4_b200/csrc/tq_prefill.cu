@@ -203,6 +203,7 @@ struct PrefillParams {
     int64_t ldy;
     unsigned *header;       // workspace header (status word)
     uint64_t timeout_ns;
+    int inject_skip;        // test hook: CTA (0, 0) never issues its second activation-tile copy
 };
 
 // One weight row's superblock slot: its four 16-byte code chunks (chunk b,
@@ -384,6 +385,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 if (!p_mbar_wait(empty_b(s), ph ^ 1u, P.timeout_ns)) {
                     atomicOr(P.header, kPStatusTimeout);
                     break;
+                }
+                if (P.inject_skip && kt == 1 && blockIdx.x == 0 && blockIdx.y == 0) {
+                    // neither the copy nor its byte count: the stage never
+                    // completes, no copy is left in flight, and the MMA
+                    // thread's bounded wait on it runs out
+                    ++issued;
+                    continue;
                 }
                 p_mbar_expect_tx(full_b(s), kBTile);
                 p_tma_load_2d(b_tile(s), &xmap, kt * kPK, m0, full_b(s));
@@ -686,7 +694,8 @@ cudaError_t launch_prefill_product(const uint8_t *codes, const uint16_t *scales,
     prm.y = static_cast<char *>(y);
     prm.ldy = ldy;
     prm.header = header;
-    prm.timeout_ns = 1000000000ull;
+    prm.inject_skip = (debug_flags() & kDebugSkipPrefillCopy) ? 1 : 0;
+    prm.timeout_ns = prm.inject_skip ? 5000000ull : 1000000000ull;  // 5 ms under the test hook
     const uint32_t base = prefill_smem_base();
     if (base > kPMaxBase) return cudaErrorInvalidValue;
     const uint32_t smem = ((base + 1023u) & ~1023u) + kPEndOff - base;

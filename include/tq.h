@@ -278,9 +278,13 @@ TQ_API tq_status tq_workspace_status(void *workspace, int clear, void *stream);
 
 /*
  * tq_debug_set_flags -- test hook, process-wide, 0 by default.  Bit 0: in
- * later fused-product launches one bulk copy of the first warp is never
- * issued, so its bounded wait expires after ~5 ms and the timeout path runs
- * (status word set, kernel returns normally; no fault, no trap).
+ * later fused-product launches (m <= 32) one bulk copy of the first warp is
+ * never issued, so its bounded wait expires after ~5 ms and the timeout path
+ * runs (status word set, kernel returns normally; no fault, no trap).  Bit 1:
+ * the same for the tensor-core prefill product (tq_gemm_prefill and m > 32):
+ * the first CTA never issues its second activation-tile copy (nor counts its
+ * bytes), its waits expire after ~5 ms, every tensor-memory column is still
+ * released, and the status word is set.
  */
 TQ_API void tq_debug_set_flags(uint32_t flags);
 
@@ -299,17 +303,34 @@ TQ_API void tq_debug_set_flags(uint32_t flags);
  * routine) and returns TQ_ERR_SHAPE when the problem's scratch,
  * tq_gemm_workspace_bytes(1, n, k), exceeds TQ_STATIC_SCRATCH_BYTES.
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the array, and each starts by
- * clearing what must start at zero: calls that overlap on the GPU (other
- * streams, other host threads, without ordering between them) race and give
- * wrong results.  Run them in order on one stream, or use tq_gemv.
+ * The first call in a CUDA context looks up the array's device address
+ * (cudaGetSymbolAddress) with that context's device current; make that first
+ * call before any stream capture.  The address is cached per context (keyed
+ * by the driver's unique context id), so after cudaDeviceReset, or from
+ * another context on the same device, the next call looks it up again; do
+ * that call outside stream capture too.  All calls share the array, and each
+ * starts by clearing what must start at zero: calls that overlap on the GPU
+ * (other streams, other host threads, without ordering between them) race
+ * and give wrong results.  Run them in order on one stream (or order the
+ * streams with events), or use tq_gemv.
+ *
+ * A bounded wait that expires inside this call is recorded in the array's
+ * status word like tq_gemv's: read it with tq_static_scratch_status.
  */
 #define TQ_STATIC_SCRATCH_BYTES (4u << 20)
 
 TQ_API tq_status tq_gemv_static_scratch(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k,
                                         const void *x, tq_dtype xt, void *y, tq_dtype yt, void *stream);
+
+/*
+ * tq_static_scratch_status -- tq_workspace_status for the fixed array of
+ * tq_gemv_static_scratch in the current context: synchronises `stream`, then
+ * returns TQ_ERR_TIMEOUT if the last tq_gemv_static_scratch call on this
+ * device gave up a bounded wait (its y is then incomplete), else TQ_OK;
+ * clear != 0 resets the flag (the next call also resets it).  Allocates
+ * nothing.
+ */
+TQ_API tq_status tq_static_scratch_status(int clear, void *stream);
 
 /*
  * ---------------------------------------------------------------------------

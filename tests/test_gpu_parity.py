@@ -333,3 +333,70 @@ def test_timeout_path_reports_and_recovers(cuda_lib):
     y = cuda_lib.gemv(codes, scales, n, k, x, ws=ws)
     assert cuda_lib.workspace_status(ws) == 0
     assert torch.equal(y, y_good)
+
+
+def test_gemv_correct_while_another_stream_holds_the_sms(cuda_lib):
+    """The fused product relies on its whole grid being resident (a split
+    tile's first warp polls for the partial sums of later CTAs); it is launched
+    cooperatively, so a long kernel on another stream that occupies the SMs
+    delays it but cannot make that poll run out.  Status TQ_OK and output
+    identical to the solo run."""
+    n, k = 14336, 4096
+    W = inputs.gaussian_matrix(0, 5, n, k, 0.02, BF16, DEV)
+    x = inputs.gaussian_matrix(1, 5, 1, k, 1.0, BF16, DEV)[0]
+    codes, scales = cuda_lib.quantize(W)
+    ws = cuda_lib.workspace(1, n, k)
+    y_solo = cuda_lib.gemv(codes, scales, n, k, x, ws=ws).clone()
+    A = torch.randn(8192, 8192, dtype=BF16, device=DEV)
+    B = torch.randn(8192, 8192, dtype=BF16, device=DEV)
+    C = torch.empty(8192, 8192, dtype=BF16, device=DEV)
+    torch.cuda.synchronize()
+    busy = torch.cuda.Stream()
+    with torch.cuda.stream(busy):
+        for _ in range(40):  # a few tens of ms of dense matmuls on every SM
+            torch.matmul(A, B, out=C)
+    for _ in range(5):
+        y = cuda_lib.gemv(codes, scales, n, k, x, ws=ws)
+    assert cuda_lib.workspace_status(ws) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_solo)
+
+
+@pytest.mark.parametrize("m", [1, 3, 17])
+def test_gemm_writes_nothing_past_its_outputs(cuda_lib, m):
+    """Guard bands: with n inside the last 16-row tile (rows past n exist in
+    the packed planes) and ldy > n, every column past n and every row past m
+    keeps its sentinel."""
+    n, k = 77, 640
+    W = _w(n, k, BF16, seed=40)
+    X = _w(m, k, BF16, seed=41, std=1.0)
+    c_ref, s_ref = _oracle_quantize(W)
+    Y_ref = oracle.gemm(c_ref, s_ref, n, k, _host_f32(X))
+    codes, scales = cuda_lib.quantize(W.to(DEV))
+    ldy = 96
+    big = torch.full((m + 2, ldy), -777.0, dtype=F32, device=DEV)
+    ws = cuda_lib.workspace(m, n, k)
+    st = cuda_lib.tq_gemm(codes.data_ptr(), scales.data_ptr(), n, k, X.to(DEV).data_ptr(), 1, m, k, big.data_ptr(),
+                          0, ldy, ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    got = big.cpu().numpy()
+    assert _rel_l2(got[:m, :n], Y_ref).max() <= REL_L2_TOL
+    assert np.all(got[:m, n:] == -777.0)
+    assert np.all(got[m:] == -777.0)
+
+
+@pytest.mark.parametrize("m", [1, 8, 32])
+def test_gemm_small_weights(cuda_lib, m):
+    """Weights of std 1e-4: half-block scales d around 6e-4, so the products
+    fp16(c * d) of the smallest centroid fall near the bottom of the fp16
+    normal range (6.1e-5), and some below it."""
+    n, k = 256, 2048
+    W = _w(n, k, F32, seed=42, std=1e-4)
+    X = _w(m, k, BF16, seed=43, std=1.0)
+    c_ref, s_ref = _oracle_quantize(W)
+    Y_ref = oracle.gemm(c_ref, s_ref, n, k, _host_f32(X))
+    codes, scales = cuda_lib.quantize(W.to(DEV))
+    Y = cuda_lib.gemm(codes, scales, n, k, X.to(DEV))
+    torch.cuda.synchronize()
+    assert _rel_l2(Y.cpu().numpy(), Y_ref).max() <= REL_L2_TOL

@@ -190,3 +190,51 @@ def test_prefill_xrot_argument_errors(cuda_lib):
     assert call(xr.data_ptr(), 256) == 0
     torch.cuda.synchronize()
     assert cuda_lib.workspace_status(ws) == 0
+
+
+def test_prefill_timeout_path_reports_and_recovers(cuda_lib):
+    """Test hook bit 1: the first CTA never issues its second activation-tile
+    copy (nor counts its bytes).  Its bounded waits (5 ms under the hook)
+    expire, the status word reports TQ_ERR_TIMEOUT, every tensor-memory column
+    is released (the next launch allocates them again) and the next call is
+    bit-identical to a clean one."""
+    m, n, k = 300, 512, 1024  # several CTAs in both directions, 16 stages of 64 columns
+    W = _w(n, k, BF16, seed=71)
+    X = _w(m, k, BF16, seed=72, std=1.0).to(DEV)
+    codes, scales = cuda_lib.quantize(W.to(DEV))
+    ws = cuda_lib.prefill_workspace(m, k)
+    Y_good = cuda_lib.gemm_prefill(codes, scales, n, k, X, ws=ws).clone()
+    assert cuda_lib.workspace_status(ws) == 0
+    try:
+        cuda_lib.tq_debug_set_flags(2)
+        cuda_lib.gemm_prefill(codes, scales, n, k, X, ws=ws)
+        assert cuda_lib.workspace_status(ws) == 8  # TQ_ERR_TIMEOUT
+    finally:
+        cuda_lib.tq_debug_set_flags(0)
+    for _ in range(2):
+        Y = cuda_lib.gemm_prefill(codes, scales, n, k, X, ws=ws)
+        assert cuda_lib.workspace_status(ws) == 0
+        assert torch.equal(Y, Y_good)
+
+
+def test_prefill_writes_nothing_past_its_outputs(cuda_lib):
+    """Guard bands: Y rows of a larger buffer (ldy > n) and the rows past m
+    keep their sentinel; only the m x n block changes."""
+    m, n, k = 40, 130, 256
+    W = _w(n, k, BF16, seed=73)
+    X = _w(m, k, BF16, seed=74, std=1.0)
+    c_ref, s_ref = oracle.quantize(_host_f32(W))
+    Y_ref = oracle.gemm(c_ref, s_ref, n, k, _host_f32(X))
+    codes, scales = cuda_lib.quantize(W.to(DEV))
+    ldy = n + 14
+    big = torch.full((m + 3, ldy), 12345.0, dtype=F32, device=DEV)
+    ws = cuda_lib.prefill_workspace(m, k)
+    st = cuda_lib.tq_gemm_prefill(codes.data_ptr(), scales.data_ptr(), n, k, X.to(DEV).data_ptr(), 1, m, k,
+                                  big.data_ptr(), 0, ldy, ws.data_ptr(), ws.numel(),
+                                  torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    got = big.cpu().numpy()
+    assert _rel_l2(got[:m, :n], Y_ref).max() <= REL_L2_TOL
+    assert np.all(got[:m, n:] == 12345.0)
+    assert np.all(got[m:] == 12345.0)
