@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["tq_codec.cu", "tq_gemv.cu", "tq_nvfp4.cu", "tq_prefill.cu", "tq_capi.cu"]
+SOURCES = ["tq_codec.cu", "tq_gemv.cu", "tq_tcgemv.cu", "tq_nvfp4.cu", "tq_prefill.cu", "tq_capi.cu"]
 HEADERS = ["tq_device.cuh", "tq_internal.h", "tq_codebook.h", os.path.join("..", "..", "include", "tq.h")]
 
 NVCC_FLAGS = [

@@ -54,35 +54,89 @@ tq_status check_planes(const uint8_t *codes, const uint16_t *scales) {
 
 tq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 
-// Workspace of a fused-product call:
+// Workspace of a fused-product call (m <= 32):
 //   [0, 256)           header: status word (timeout flag of the last call),
 //                      call tag (advanced by every call)
-//   partial slots      (tiles + warps) * 16 * mcap tagged sums (8 bytes each)
-//   pre-rotated inputs one area per distinct activation (calls that rotate)
+//   tensor-memory kernel:
+//     counters         one call-tagged 64-bit counter per 128-row block
+//     partial slots    2 * CTAs * mld * 128 fp32 partial sums of split row blocks
+//   mma.sync kernel:
+//     partial slots    (tiles + warps) * 16 * mcap tagged sums (8 bytes each)
+//   pre-rotated inputs one area per distinct activation, in the layout of the
+//                      kernel that runs
 struct Layout {
-    size_t partial_off, xrot_off[tq::kMaxInputs], total;
+    size_t partial_off, counter_off, xrot_off[tq::kMaxInputs], total;
     int inputs;
-    tq::GroupPlan plan;
+    bool tc;             // the tensor-memory kernel runs the product
+    tq::GroupPlan plan;  // mma.sync kernel
+    tq::TcPlan tplan;    // tensor-memory kernel
 };
 
 constexpr size_t kStatusBytes = 256;
 
 tq_status make_layout(const int64_t *n, const int64_t *k, int count, const int64_t *input_k, int inputs, int64_t m,
-                      Layout *lay) {
+                      Layout *lay, bool allow_tc) {
     tq::DeviceInfo di;
     if (tq::device_info(&di) != cudaSuccess) return TQ_ERR_CUDA;
     const int64_t ms = m > 32 ? 32 : (m < 1 ? 1 : m);
-    lay->plan = tq::plan_group(n, k, count, ms, di.sm_count);
-    if (lay->plan.units >= ((int64_t)1 << 31)) return TQ_ERR_SHAPE;  // > 2^42 weights per call
-    lay->partial_off = kStatusBytes;
-    size_t off = lay->partial_off + lay->plan.partial_bytes;
     lay->inputs = inputs;
-    for (int i = 0; i < inputs; ++i) {
-        lay->xrot_off[i] = off;
-        off += tq::round_up(tq_xrot_bytes(ms, input_k[i]), 256);
+    lay->tc = allow_tc && tq::use_tc(ms);
+    size_t off;
+    if (lay->tc) {
+        lay->tplan = tq::plan_tc(n, k, count, ms, di.sm_count);
+        if (lay->tplan.units >= ((int64_t)1 << 31)) return TQ_ERR_SHAPE;  // > 2^41 weights per call
+        lay->counter_off = kStatusBytes;
+        lay->partial_off = lay->counter_off + lay->tplan.counter_bytes;
+        off = lay->partial_off + lay->tplan.partial_bytes;
+        for (int i = 0; i < inputs; ++i) {
+            lay->xrot_off[i] = off;
+            off += tq::round_up(tq::tc_xrot_bytes(ms, input_k[i]), 256);
+        }
+    } else {
+        lay->plan = tq::plan_group(n, k, count, ms, di.sm_count);
+        if (lay->plan.units >= ((int64_t)1 << 31)) return TQ_ERR_SHAPE;  // > 2^42 weights per call
+        lay->counter_off = 0;
+        lay->partial_off = kStatusBytes;
+        off = lay->partial_off + lay->plan.partial_bytes;
+        for (int i = 0; i < inputs; ++i) {
+            lay->xrot_off[i] = off;
+            off += tq::round_up(tq_xrot_bytes(ms, input_k[i]), 256);
+        }
     }
     lay->total = off;
     return TQ_OK;
+}
+
+// Bytes a product of these shapes needs whichever kernel runs it.
+tq_status workspace_need(const int64_t *n, const int64_t *k, int count, const int64_t *input_k, int inputs, int64_t m,
+                         size_t *need) {
+    Layout a, b;
+    tq_status st = make_layout(n, k, count, input_k, inputs, m, &a, false);
+    if (st != TQ_OK) return st;
+    st = make_layout(n, k, count, input_k, inputs, m, &b, true);
+    if (st != TQ_OK) return st;
+    *need = a.total > b.total ? a.total : b.total;
+    return TQ_OK;
+}
+
+// Pre-rotation (which also clears the status word and advances the call tag)
+// and product of a laid-out call: jobs[q] feeds the problems whose input is q.
+cudaError_t run_layout(const Layout &lay, const tq::RotJob *jobs, const tq::GemvProblem *pbs, int count, int64_t m,
+                       tq_dtype xt, tq_dtype yt, char *ws, cudaStream_t s) {
+    unsigned *header = reinterpret_cast<unsigned *>(ws);
+    if (lay.tc) {
+        const int np = lay.tplan.npad;
+        cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, header, s, true,
+                                             np == 0 ? tq::kRotPlain : tq::kRotCore, np);
+        if (e != cudaSuccess) return e;
+        return tq::launch_tc(pbs, count, m, yt, lay.tplan, header,
+                             reinterpret_cast<unsigned long long *>(ws + lay.counter_off),
+                             reinterpret_cast<float *>(ws + lay.partial_off), true, s);
+    }
+    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, header, s);
+    if (e != cudaSuccess) return e;
+    return tq::launch_group(pbs, count, m, yt, lay.plan, header, reinterpret_cast<uint64_t *>(ws + lay.partial_off),
+                            true, s);
 }
 
 }  // namespace
@@ -165,9 +219,9 @@ static size_t prefill_workspace(int64_t m, int64_t k) {
 size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
     if (m < 0 || check_nk(n, k) != TQ_OK) return 0;
     if (m > kSkinnyMaxM) return prefill_workspace(m, k);
-    Layout lay;
-    if (make_layout(&n, &k, 1, &k, 1, m, &lay) != TQ_OK) return 0;
-    return lay.total;
+    size_t need = 0;
+    if (workspace_need(&n, &k, 1, &k, 1, m, &need) != TQ_OK) return 0;
+    return need;
 }
 
 static tq_status check_gemm_common(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, int64_t m,
@@ -212,8 +266,8 @@ tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, 
     if (m > 32) return TQ_ERR_SHAPE;
     if (!xrot) return TQ_ERR_INVALID_ARG;
     if (!aligned(xrot, 16)) return TQ_ERR_ALIGNMENT;
-    Layout lay;
-    if ((st = make_layout(&n, &k, 1, nullptr, 0, m, &lay)) != TQ_OK) return st;
+    Layout lay;  // the activation is in the mma.sync kernel's fragment order: that kernel runs
+    if ((st = make_layout(&n, &k, 1, nullptr, 0, m, &lay, false)) != TQ_OK) return st;
     if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
     char *ws = static_cast<char *>(workspace);
     cudaStream_t s = (cudaStream_t)stream;
@@ -222,7 +276,7 @@ tq_status tq_gemm_xrot(const uint8_t *codes, const uint16_t *scales, int64_t n, 
     if (tq::launch_prepare_header(reinterpret_cast<unsigned *>(ws), s) != cudaSuccess) return TQ_ERR_CUDA;
     tq::GemvProblem pb = {codes, scales, xrot, Y, ldy, n, k};
     return from_cuda(tq::launch_group(&pb, 1, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
-                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s));
+                                      reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s));
 }
 
 tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *X, tq_dtype xt,
@@ -234,24 +288,12 @@ tq_status tq_gemm(const uint8_t *codes, const uint16_t *scales, int64_t n, int64
     if ((st = check_matrix_operand(X, ldx, k)) != TQ_OK) return st;
     if (m > kSkinnyMaxM) return run_prefill(codes, scales, n, k, X, xt, m, ldx, Y, yt, ldy, workspace, ws_bytes, stream);
     Layout lay;
-    if ((st = make_layout(&n, &k, 1, &k, 1, m, &lay)) != TQ_OK) return st;
+    if ((st = make_layout(&n, &k, 1, &k, 1, m, &lay, true)) != TQ_OK) return st;
     if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
     char *ws = static_cast<char *>(workspace);
-    auto *xrot = reinterpret_cast<uint16_t *>(ws + lay.xrot_off[0]);
-    const size_t xsize = xt == TQ_F32 ? 4 : 2, ysize = yt == TQ_F32 ? 4 : 2;
-    cudaStream_t s = (cudaStream_t)stream;
-    for (int64_t i0 = 0; i0 < m; i0 += 32) {
-        const int64_t ms = (m - i0) < 32 ? (m - i0) : 32;
-        tq::RotJob job = {static_cast<const char *>(X) + (size_t)i0 * (size_t)ldx * xsize, ldx, k, xrot};
-        // also clears the status word and advances the call tag
-        cudaError_t e = tq::launch_prerotate(&job, 1, xt, ms, reinterpret_cast<unsigned *>(ws), s);
-        if (e != cudaSuccess) return TQ_ERR_CUDA;
-        tq::GemvProblem pb = {codes, scales, xrot, static_cast<char *>(Y) + (size_t)i0 * (size_t)ldy * ysize, ldy, n, k};
-        e = tq::launch_group(&pb, 1, ms, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
-                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
-        if (e != cudaSuccess) return TQ_ERR_CUDA;
-    }
-    return TQ_OK;
+    const tq::RotJob job = {X, ldx, k, reinterpret_cast<uint16_t *>(ws + lay.xrot_off[0])};
+    const tq::GemvProblem pb = {codes, scales, job.xrot, Y, ldy, n, k};
+    return from_cuda(run_layout(lay, &job, &pb, 1, m, xt, yt, ws, (cudaStream_t)stream));
 }
 
 tq_status tq_gemv(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, const void *x, tq_dtype xt,
@@ -310,7 +352,8 @@ tq_status tq_gemm_prefill_xrot(const uint8_t *codes, const uint16_t *scales, int
 }
 
 // ---- batch: several matrices, one pre-rotation per distinct input ----------
-static tq_status batch_layout(const tq_gemm_desc *descs, int count, int64_t m, Layout *lay, int *input_of) {
+static tq_status batch_layout(const tq_gemm_desc *descs, int count, int64_t m, Layout *lay, int *input_of,
+                              bool allow_tc) {
     int64_t n[tq::kMaxProblems], k[tq::kMaxProblems], ik[tq::kMaxInputs];
     int inputs = 0;
     for (int i = 0; i < count; ++i) {
@@ -328,17 +371,18 @@ static tq_status batch_layout(const tq_gemm_desc *descs, int count, int64_t m, L
         }
         input_of[i] = found;
     }
-    return make_layout(n, k, count, ik, inputs, m, lay);
+    return make_layout(n, k, count, ik, inputs, m, lay, allow_tc);
 }
 
 size_t tq_gemm_batch_workspace_bytes(const tq_gemm_desc *descs, int count, int64_t m) {
     if (!descs || count < 1 || count > TQ_MAX_BATCH || m < 0 || m > 32) return 0;
     for (int i = 0; i < count; ++i)
         if (check_nk(descs[i].n, descs[i].k) != TQ_OK) return 0;
-    Layout lay;
+    Layout a, b;
     int input_of[tq::kMaxProblems];
-    if (batch_layout(descs, count, m, &lay, input_of) != TQ_OK) return 0;
-    return lay.total;
+    if (batch_layout(descs, count, m, &a, input_of, false) != TQ_OK) return 0;
+    if (batch_layout(descs, count, m, &b, input_of, true) != TQ_OK) return 0;
+    return a.total > b.total ? a.total : b.total;
 }
 
 tq_status tq_gemm_batch(const tq_gemm_desc *descs, int count, int64_t m, tq_dtype xt, tq_dtype yt, void *workspace,
@@ -358,7 +402,7 @@ tq_status tq_gemm_batch(const tq_gemm_desc *descs, int count, int64_t m, tq_dtyp
     if (m == 0) return TQ_OK;
     Layout lay;
     int input_of[tq::kMaxProblems];
-    if ((st = batch_layout(descs, count, m, &lay, input_of)) != TQ_OK) return st;
+    if ((st = batch_layout(descs, count, m, &lay, input_of, true)) != TQ_OK) return st;
     if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
     char *ws = static_cast<char *>(workspace);
     tq::RotJob jobs[tq::kMaxInputs];
@@ -369,12 +413,7 @@ tq_status tq_gemm_batch(const tq_gemm_desc *descs, int count, int64_t m, tq_dtyp
         jobs[q] = {descs[i].X, descs[i].ldx, descs[i].k, xrot};
         pbs[i] = {descs[i].codes, descs[i].scales, xrot, descs[i].Y, descs[i].ldy, descs[i].n, descs[i].k};
     }
-    cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws), s);
-    if (e != cudaSuccess) return TQ_ERR_CUDA;
-    e = tq::launch_group(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
-                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
-    return from_cuda(e);
+    return from_cuda(run_layout(lay, jobs, pbs, count, m, xt, yt, ws, (cudaStream_t)stream));
 }
 
 // ---- NVFP4 comparison codec -------------------------------------------------
@@ -450,7 +489,7 @@ tq_status tq_nvfp4_gemm_batch(const tq_nvfp4_gemm_desc *descs, int count, int64_
     if (m == 0) return TQ_OK;
     Layout lay;
     int input_of[tq::kMaxProblems];
-    if ((st = batch_layout(plain, count, m, &lay, input_of)) != TQ_OK) return st;
+    if ((st = batch_layout(plain, count, m, &lay, input_of, false)) != TQ_OK) return st;
     if ((st = check_workspace(workspace, ws_bytes, lay.total)) != TQ_OK) return st;
     char *ws = static_cast<char *>(workspace);
     tq::RotJob jobs[tq::kMaxInputs];
@@ -467,8 +506,7 @@ tq_status tq_nvfp4_gemm_batch(const tq_nvfp4_gemm_desc *descs, int count, int64_
     cudaError_t e = tq::launch_prerotate(jobs, lay.inputs, xt, m, reinterpret_cast<unsigned *>(ws), s, false);
     if (e != cudaSuccess) return TQ_ERR_CUDA;
     e = tq::launch_group_nvfp4(pbs, count, m, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
-                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true,
-                               s);
+                               reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
     return from_cuda(e);
 }
 
@@ -584,22 +622,16 @@ extern "C" tq_status tq_gemv_static_scratch(const uint8_t *codes, const uint16_t
     if (!valid_dtype(xt)) return TQ_ERR_DTYPE;
     if ((st = check_matrix_operand(x, k, k)) != TQ_OK) return st;
     Layout lay;
-    if ((st = make_layout(&n, &k, 1, &k, 1, 1, &lay)) != TQ_OK) return st;
+    if ((st = make_layout(&n, &k, 1, &k, 1, 1, &lay, true)) != TQ_OK) return st;
     if (lay.total > (size_t)TQ_STATIC_SCRATCH_BYTES) return TQ_ERR_SHAPE;  // does not fit the fixed scratch
     void *scratch = nullptr;
     if (static_scratch_address(&scratch) != cudaSuccess) return TQ_ERR_CUDA;
     char *ws = static_cast<char *>(scratch);
-    auto *xrot = reinterpret_cast<uint16_t *>(ws + lay.xrot_off[0]);
-    cudaStream_t s = (cudaStream_t)stream;
-    tq::RotJob job = {x, k, k, xrot};
+    const tq::RotJob job = {x, k, k, reinterpret_cast<uint16_t *>(ws + lay.xrot_off[0])};
+    const tq::GemvProblem pb = {codes, scales, job.xrot, y, n, n, k};
     // the pre-rotation launch also clears the status word and advances the
     // call tag: the array keeps whatever the previous call left in it
-    cudaError_t e = tq::launch_prerotate(&job, 1, xt, 1, reinterpret_cast<unsigned *>(ws), s);
-    if (e != cudaSuccess) return TQ_ERR_CUDA;
-    tq::GemvProblem pb = {codes, scales, xrot, y, n, n, k};
-    e = tq::launch_group(&pb, 1, 1, yt, lay.plan, reinterpret_cast<unsigned *>(ws),
-                         reinterpret_cast<uint64_t *>(ws + lay.partial_off), true, s);
-    return from_cuda(e);
+    return from_cuda(run_layout(lay, &job, &pb, 1, 1, xt, yt, ws, (cudaStream_t)stream));
 }
 
 extern "C" tq_status tq_static_scratch_status(int clear, void *stream) {

@@ -326,20 +326,29 @@ __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_
 }
 
 // -------------------------------------------------------------------------
-// Pre-rotation of activations into the fused kernel's fragment order:
-// element e of a block goes to slot t*8 + q with t = (e%8)/2, q = 2*(e/8) + e%2.
+// Pre-rotation of activations.  Output layouts (RotLayout):
+//  * kRotFragment: the mma.sync kernel's fragment order: element e of a block
+//    goes to slot t*8 + q with t = (e%8)/2, q = 2*(e/8) + e%2;
+//  * kRotPlain: row-major fp16 [rows][NSB*128], padding columns zero (the
+//    tensor-memory kernel's one-row operand);
+//  * kRotCore: the tensor-memory kernel's B operand for npad rows, in 16-byte
+//    core-matrix rows: [NSB][16 column groups of 8][npad rows][8], rows m ..
+//    npad-1 and padding columns zero.
 // Handles a list of inputs (one warp per (input, row, superblock)) and
 // prepares the header of the product that follows (status cleared, tag
 // advanced).
 // -------------------------------------------------------------------------
-template <int DT, bool ROTATE>
+template <int DT, bool ROTATE, int LAYOUT>
 __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_constant__ RotParams prm) {
     // Launched as a programmatic dependent of the previous kernel in the
-    // stream: wait until every earlier kernel has completed (and its memory is
-    // visible), then let the fused product that follows start its prologue,
-    // which reads packed weights that earlier kernels may have written.
-    grid_dependency_wait();
+    // stream.  The fused product that follows may launch at once: before its
+    // own dependency wait it only fills shared memory and copies packed
+    // weights, which no kernel still running writes (a product's weights are
+    // written by a quantise launch that completed before this kernel could
+    // start), so its CTAs can take the SMs that the previous product frees
+    // in its tail.  Then wait until every earlier kernel has completed.
     grid_dependents_launch();
+    grid_dependency_wait();
     if (prm.header && blockIdx.x == 0 && threadIdx.x == 0) {
         prm.header[kHeaderStatus] = 0u;
         prm.header[kHeaderTag] += 1u;  // the previous call (and its product) has completed
@@ -354,7 +363,7 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     const RotInput &in = prm.in[q];
     const int64_t local = unit - in.unit_begin;
     const int row = (int)(local / in.nsb), sb = (int)(local % in.nsb);
-    const bool valid = sb * kSbBlocks + j < in.nb;
+    const bool valid = sb * kSbBlocks + j < in.nb && row < prm.m;
     const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (valid) load4<DT>(in.x + ((int64_t)row * in.ldx + col0) * ElemSize<DT>::value, v);
@@ -367,11 +376,24 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     }
     const __half2 lo = __floats2half2_rn(v[0], v[1]);
     const __half2 hi = __floats2half2_rn(v[2], v[3]);
-    // elements 4p, 4p+1 -> t = 2(p&1), q = 2(p>>1) + {0,1}; 4p+2, 4p+3 -> t + 1
-    const size_t blk_words = ((size_t)local * kSbBlocks + j) * 16;  // 32 halves per block
-    const int t0 = 2 * (p & 1), q0 = 2 * (p >> 1);
-    in.xrot[blk_words + (t0 * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&lo);
-    in.xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
+    if constexpr (LAYOUT == kRotFragment) {
+        // elements 4p, 4p+1 -> t = 2(p&1), q = 2(p>>1) + {0,1}; 4p+2, 4p+3 -> t + 1
+        const size_t blk_words = ((size_t)local * kSbBlocks + j) * 16;  // 32 halves per block
+        const int t0 = 2 * (p & 1), q0 = 2 * (p >> 1);
+        in.xrot[blk_words + (t0 * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&lo);
+        in.xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
+    } else {
+        size_t half_off;
+        if constexpr (LAYOUT == kRotPlain) {
+            half_off = (size_t)row * in.nsb * kSbElems + col0;
+        } else {  // kRotCore: column group 4j + p/2, element 4(p&1) .. +3 of its 16-byte row
+            half_off = ((size_t)sb * 16 + 4 * j + (p >> 1)) * (size_t)prm.npad * 8 + (size_t)row * 8 + 4 * (p & 1);
+        }
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t *>(&lo);
+        o.y = *reinterpret_cast<const uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(in.xrot) + half_off) = o;
+    }
 }
 
 // Row groups per column segment: one wave of the CTAs that fit on the GPU at
@@ -459,8 +481,8 @@ cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int6
 namespace {
 
 __global__ void __launch_bounds__(32) prepare_header_kernel(unsigned *header) {
+    grid_dependents_launch();  // as in the pre-rotation: the product's prologue may overlap
     grid_dependency_wait();
-    grid_dependents_launch();
     if (threadIdx.x == 0) {
         header[kHeaderStatus] = 0u;
         header[kHeaderTag] += 1u;
@@ -483,8 +505,13 @@ cudaError_t launch_prepare_header(unsigned *header, cudaStream_t stream) {
 }
 
 cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *header,
-                             cudaStream_t stream, bool rotate) {
+                             cudaStream_t stream, bool rotate, int layout, int npad) {
     if (count < 1 || count > kMaxInputs) return cudaErrorInvalidValue;
+    if (layout == kRotCore && (npad < m || npad % 8 != 0)) return cudaErrorInvalidValue;
+    if (layout == kRotPlain && !rotate) return cudaErrorInvalidValue;
+    // rows written per input: m, or npad in the core-matrix layout (rows past
+    // m are written as zeros)
+    const int64_t rows = layout == kRotCore ? npad : m;
     RotParams prm = {};
     int64_t units = 0;
     for (int i = 0; i < count; ++i) {
@@ -495,11 +522,13 @@ cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m
         in.unit_begin = units;
         in.nb = (int)(jobs[i].k / 32);
         in.nsb = (int)superblocks(jobs[i].k);
-        units += m * in.nsb;
+        units += rows * in.nsb;
     }
     prm.count = count;
     prm.units = units;
     prm.header = header;
+    prm.m = (int)m;
+    prm.npad = npad;
     int64_t grid = (units + kCodecWarps - 1) / kCodecWarps;
     if (grid < 1) grid = 1;
     cudaLaunchConfig_t cfg = {};
@@ -511,13 +540,29 @@ cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (layout == kRotPlain) {
+        switch (dtype) {
+            case kF32: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, true, kRotPlain>, prm);
+            case kBF16: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, true, kRotPlain>, prm);
+            case kF16: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, true, kRotPlain>, prm);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    if (layout == kRotCore) {
+        switch (dtype * 2 + (rotate ? 1 : 0)) {
+            case kF32 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, true, kRotCore>, prm);
+            case kBF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, true, kRotCore>, prm);
+            case kF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, true, kRotCore>, prm);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (dtype * 2 + (rotate ? 1 : 0)) {
-        case kF32 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, true>, prm);
-        case kBF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, true>, prm);
-        case kF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, true>, prm);
-        case kF32 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, false>, prm);
-        case kBF16 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, false>, prm);
-        case kF16 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, false>, prm);
+        case kF32 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, true, kRotFragment>, prm);
+        case kBF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, true, kRotFragment>, prm);
+        case kF16 * 2 + 1: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, true, kRotFragment>, prm);
+        case kF32 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF32, false, kRotFragment>, prm);
+        case kBF16 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kBF16, false, kRotFragment>, prm);
+        case kF16 * 2: return cudaLaunchKernelEx(&cfg, prerotate_kernel<kF16, false, kRotFragment>, prm);
         default: return cudaErrorInvalidValue;
     }
 }

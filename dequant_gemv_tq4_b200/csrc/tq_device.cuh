@@ -185,6 +185,55 @@ __device__ __forceinline__ void mma_16816_zero(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// ---------------------------------------------------------------------------
+// Register-table decode of TQ4_1S codes (no shared-memory table): the eight
+// fp16 Lloyd-Max magnitudes as byte tables for PRMT.
+// ---------------------------------------------------------------------------
+// 4x4 byte transpose: out[i] byte b = in[b] byte i.
+__device__ __forceinline__ void transpose4(const uint32_t (&w)[4], uint32_t (&o)[4]) {
+    const uint32_t a = prmt(w[0], w[1], 0x5140u), b = prmt(w[2], w[3], 0x5140u);
+    const uint32_t c = prmt(w[0], w[1], 0x7362u), d = prmt(w[2], w[3], 0x7362u);
+    o[0] = prmt(a, b, 0x5410u);
+    o[1] = prmt(a, b, 0x7632u);
+    o[2] = prmt(c, d, 0x5410u);
+    o[3] = prmt(c, d, 0x7632u);
+}
+
+// fp16 Lloyd-Max magnitudes as byte tables for PRMT: low bytes of magnitudes
+// 0..3 / 4..7 and high bytes of magnitudes 0..3 / 4..7.
+constexpr uint16_t kMagF16[8] = TQ_MAG_F16_INIT;
+constexpr uint32_t mag_bytes(int i0, bool hi) {
+    uint32_t v = 0;
+    for (int i = 0; i < 4; ++i) v |= (uint32_t)((hi ? kMagF16[i0 + i] >> 8 : kMagF16[i0 + i]) & 0xFF) << (8 * i);
+    return v;
+}
+constexpr uint32_t kMagLo0 = mag_bytes(0, false), kMagLo1 = mag_bytes(4, false);
+constexpr uint32_t kMagHi0 = mag_bytes(0, true), kMagHi1 = mag_bytes(4, true);
+
+// Eight codes (one logical word: element 2L in the low nibble of byte L,
+// element 2L+1 in the high nibble) to four fp16 pairs of signed centroids.
+//  * magnitudes: PRMT with the three magnitude bits of four codes as its
+//    selector nibbles picks their low (high) bytes from the byte tables;
+//  * signs: a code's sign is bit 3 of its nibble, i.e. the top bit of a byte
+//    of w (odd elements) or of w << 4 (even elements); PRMT in sign-replicate
+//    mode turns those top bits into 0xFF / 0x00 bytes, one per code, whose
+//    top bit is merged into the high bytes;
+//  * two more PRMTs interleave low and high bytes into fp16 pairs.
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t (&o)[4]) {
+    const uint32_t m = w & 0x77777777u;  // magnitude ranks (PRMT reads the low 16 bits)
+    const uint32_t m2 = m >> 16;
+    const uint32_t w4 = w << 4;
+    // byte j of the mask: sign of element j (selector nibbles: 8 | byte, a = w4, b = w)
+    const uint32_t s03 = prmt(w4, w, 0xD9C8u), s47 = prmt(w4, w, 0xFBEAu);
+    const uint32_t lo03 = prmt(kMagLo0, kMagLo1, m), lo47 = prmt(kMagLo0, kMagLo1, m2);
+    const uint32_t hi03 = prmt(kMagHi0, kMagHi1, m) | (s03 & 0x80808080u);
+    const uint32_t hi47 = prmt(kMagHi0, kMagHi1, m2) | (s47 & 0x80808080u);
+    o[0] = prmt(lo03, hi03, 0x5140u);  // elements 0, 1
+    o[1] = prmt(lo03, hi03, 0x7362u);  // elements 2, 3
+    o[2] = prmt(lo47, hi47, 0x5140u);  // elements 4, 5
+    o[3] = prmt(lo47, hi47, 0x7362u);  // elements 6, 7
+}
+
 // Programmatic dependent launch: wait for the preceding grid's results / let
 // the next grid start its prologue.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -44,7 +44,12 @@ struct RotParams {
     int count;
     int64_t units;
     unsigned *header;  // product workspace header (see below), or nullptr
+    int m;             // activation rows (rows past m are written as zeros)
+    int npad;          // rows of the core-matrix layout
 };
+
+// Output layouts of the pre-rotation (see launch_prerotate).
+enum RotLayout : int { kRotFragment = 0, kRotPlain = 1, kRotCore = 2 };
 
 struct RotJob {  // host-side request
     const void *x;
@@ -62,9 +67,13 @@ constexpr int kHeaderTag = 1;
 
 // xrot for m rows of every job (same dtype); also prepares `header` (status
 // cleared, tag advanced) when it is not null.  With rotate = false the
-// activation is only converted to fp16 fragment order.
+// activation is only converted to fp16 (fragment or core-matrix order).
+// Layouts: kRotFragment (tq_xrot_bytes per input; the mma.sync kernel),
+// kRotPlain (one row, NSB*128 fp16 with zero padding; the tensor-memory
+// kernel for m = 1), kRotCore (npad rows, NSB*16*npad*16 bytes; the
+// tensor-memory kernel for m > 1).
 cudaError_t launch_prerotate(const RotJob *jobs, int count, int dtype, int64_t m, unsigned *header,
-                             cudaStream_t stream, bool rotate = true);
+                             cudaStream_t stream, bool rotate = true, int layout = kRotFragment, int npad = 0);
 
 // Only the header preparation (for products whose activation is already
 // pre-rotated).  Launched as a programmatic dependent like the pre-rotation.
@@ -98,11 +107,45 @@ GroupPlan plan_group(const int64_t *n, const int64_t *k, int count, int64_t m, i
 // that the kernel's bounded wait expires and reports a timeout.
 constexpr uint32_t kDebugSkipGemvCopy = 1u;
 constexpr uint32_t kDebugSkipPrefillCopy = 2u;
+// bits 2 and 3: run every product of m <= 32 on the tensor-memory kernel
+// (bit 2) or on the mma.sync kernel (bit 3) instead of choosing by m (lets
+// tests and measurements cover both kernels at every m)
+constexpr uint32_t kDebugUseTmem = 4u;
+constexpr uint32_t kDebugUseMmaSync = 8u;
 void set_debug_flags(uint32_t flags);
 uint32_t debug_flags();
 
 cudaError_t launch_group(const GemvProblem *probs, int count, int64_t m, int ydtype, const GroupPlan &plan,
                          unsigned *header, uint64_t *partials, bool programmatic, cudaStream_t stream);
+
+// ---- fused product on tcgen05 with the weights in tensor memory (tq_tcgemv.cu)
+// Big units of 128 weight rows x 128 columns split into equal ranges, one per
+// CTA; split row blocks combine through per-row-block call-tagged counters
+// (the last contributor adds the partial sums).  The activation operand is
+// the pre-rotation in kRotPlain layout (m = 1) or kRotCore layout with
+// npad = 16 (m <= 16) or 32 rows.
+struct TcPlan {
+    int64_t units;        // big units over all problems
+    int64_t rblocks;      // row blocks over all problems (counter slots)
+    int grid;             // CTAs (<= SM count)
+    int npad;             // activation rows of the operand: 0 (one row, plain layout), 16 or 32
+    int mld;              // accumulator columns read back per row: 1, 2, 4, 8, 16 or 32
+    size_t counter_bytes; // rblocks * 8, rounded up to 256
+    size_t partial_bytes; // 2 * grid * mld * 128 fp32, rounded up to 256
+};
+int tc_npad(int64_t m);
+int tc_mld(int64_t m);
+size_t tc_xrot_bytes(int64_t m, int64_t k);  // the activation operand of one input
+TcPlan plan_tc(const int64_t *n, const int64_t *k, int count, int64_t m, int sm_count);
+cudaError_t launch_tc(const GemvProblem *probs, int count, int64_t m, int ydtype, const TcPlan &plan,
+                      unsigned *header, unsigned long long *counters, float *partials, bool programmatic,
+                      cudaStream_t stream);
+// Which kernel runs a TQ4_1S product of m <= 32 activation rows: the mma.sync
+// kernel up to 8 rows, the tensor-memory kernel from 9 rows (measured on B200:
+// from 9 rows the mma.sync kernel reloads four activation fragments per unit
+// and falls below it); the test hooks kDebugUseTmem / kDebugUseMmaSync force
+// one kernel.
+bool use_tc(int64_t m);
 
 // ---- large-M product on tcgen05 (tq_prefill.cu) ---------------------------------
 // Y = X w~^T for any m: X is first pre-rotated into plain row-major fp16 xrot

@@ -157,10 +157,16 @@ TQ_API size_t tq_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * tq_gemm -- Y[i][r] = sum_k w~[r][k] X[i][k] for i < m, r < n, computed as
  * (1/32) sum_blocks sum_halves d * sum_e c_e xrot_e with the activation
  * pre-rotated once per call (TQ page, 解码速度 section).  Centroids and xrot
- * enter the tensor cores as fp16; products accumulate in fp32.  For m = 25..32
- * (and in the prefill product) the centroid enters already multiplied by its
- * half-block scale, fp16(c * d), which overflows once d exceeds about 23,970
- * (weights of magnitude around 4,000 and up).
+ * enter the tensor cores as fp16; products accumulate in fp32.
+ * Kernels: m <= 8 runs the mma.sync kernel (half-block sums scaled in fp32);
+ * m = 9..32 runs the tcgen05 kernel that stages the decoded weights in tensor
+ * memory; m > 32 runs the prefill product.  From m = 9 (and for m = 25..32
+ * on the mma.sync kernel when a test hook forces it) the centroid enters
+ * already multiplied by its half-block scale, fp16(c * d): that product
+ * overflows once d exceeds about 23,970 (weights of magnitude around 4,000
+ * and up) and becomes an fp16 subnormal, with coarser relative precision,
+ * once 0.128 * d falls below 6.1e-5, i.e. d below about 4.8e-4 (weights of
+ * RMS below about 1e-4).
  *   X          device, m x k of dtype xt, row stride ldx (as tq_prerotate)
  *   Y          device, m x n of dtype yt (F32, BF16 or F16), row stride ldy
  *              (ldy >= n)
@@ -278,9 +284,12 @@ TQ_API tq_status tq_workspace_status(void *workspace, int clear, void *stream);
 
 /*
  * tq_debug_set_flags -- test hook, process-wide, 0 by default.  Bit 0: in
- * later fused-product launches (m <= 32) one bulk copy of the first warp is
- * never issued, so its bounded wait expires after ~5 ms and the timeout path
- * runs (status word set, kernel returns normally; no fault, no trap).  Bit 1:
+ * later fused-product launches (m <= 32) the first copy of the first warp
+ * (mma.sync kernel) or of the first CTA (tensor-memory kernel) is never
+ * issued, so its bounded wait expires after ~5 ms and the timeout path runs
+ * (status word set, kernel returns normally; no fault, no trap).  Bits 2 and
+ * 3: every product with m <= 32 runs on the tensor-memory kernel (bit 2) or
+ * on the mma.sync kernel (bit 3) instead of the kernel chosen by m.  Bit 1:
  * the same for the tensor-core prefill product (tq_gemm_prefill and m > 32):
  * the first CTA never issues its second activation-tile copy (nor counts its
  * bytes), its waits expire after ~5 ms, every tensor-memory column is still

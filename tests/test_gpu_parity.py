@@ -23,6 +23,22 @@ DEV = "cuda:0"
 F32, BF16, F16 = torch.float32, torch.bfloat16, torch.float16
 
 
+USE_TMEM = 4  # tq_debug_set_flags bit 2: every m <= 32 on the tensor-memory kernel
+USE_MMA_SYNC = 8  # bit 3: every m <= 32 on the mma.sync kernel
+
+
+@pytest.fixture(params=["mma_sync", "tmem"])
+def kernel(request, cuda_lib):
+    """Runs a test on each fused-product kernel (m <= 32), whatever m: the
+    mma.sync kernel (the default up to 8 rows) and the tcgen05 kernel with the
+    weights in tensor memory (the default from 9 rows)."""
+    cuda_lib.tq_debug_set_flags(USE_TMEM if request.param == "tmem" else USE_MMA_SYNC)
+    try:
+        yield request.param
+    finally:
+        cuda_lib.tq_debug_set_flags(0)
+
+
 def _w(n, k, dtype, seed=0, std=0.02):
     return inputs.gaussian_matrix(seed, n * 7919 + k, n, k, std, dtype)
 
@@ -155,7 +171,7 @@ GEMM_CASES = [
 
 
 @pytest.mark.parametrize("m,n,k", GEMM_CASES)
-def test_gemm_rel_l2(cuda_lib, m, n, k):
+def test_gemm_rel_l2(cuda_lib, kernel, m, n, k):
     W = _w(n, k, BF16, seed=8)
     X = _w(m, k, BF16, seed=9, std=1.0)
     c_ref, s_ref = _oracle_quantize(W)
@@ -168,7 +184,7 @@ def test_gemm_rel_l2(cuda_lib, m, n, k):
 
 
 @pytest.mark.parametrize("out_dtype", [BF16, F16])
-def test_gemv_low_precision_outputs(cuda_lib, out_dtype):
+def test_gemv_low_precision_outputs(cuda_lib, kernel, out_dtype):
     n, k = 300, 1024
     W = _w(n, k, BF16, seed=10)
     x = _w(1, k, F32, seed=11, std=1.0)[0]
@@ -201,7 +217,7 @@ def test_gemv_single_matrix_workload(cuda_lib):
     assert _rel_l2(y.cpu().numpy(), y_ref)[0] <= REL_L2_TOL
 
 
-def test_gemv_deterministic_and_workspace_reuse(cuda_lib):
+def test_gemv_deterministic_and_workspace_reuse(cuda_lib, kernel):
     n, k = 4096, 4096
     W = inputs.gaussian_matrix(0, 1, n, k, 0.02, BF16, DEV)
     x = inputs.gaussian_matrix(1, 1, 1, k, 1.0, BF16, DEV)[0]
@@ -215,7 +231,10 @@ def test_gemv_deterministic_and_workspace_reuse(cuda_lib):
 
 
 def test_shared_prerotation_matches_gemm(cuda_lib):
-    """One pre-rotated activation shared by three matrices (q/k/v style)."""
+    """One pre-rotated activation shared by three matrices (q/k/v style).
+    tq_gemm_xrot takes the mma.sync kernel's fragment-ordered activation, so
+    it is compared bit for bit with tq_gemm on that (default) kernel, and with
+    the tensor-memory kernel within the product's bar."""
     k = 1024
     x = _w(1, k, BF16, seed=12, std=1.0).to(DEV)
     xr = cuda_lib.prerotate(x)
@@ -224,9 +243,15 @@ def test_shared_prerotation_matches_gemm(cuda_lib):
         codes, scales = cuda_lib.quantize(W)
         ws = cuda_lib.workspace(1, n, k)
         a = cuda_lib.gemm_xrot(codes, scales, n, k, xr, 1, ws=ws)
-        b = cuda_lib.gemm(codes, scales, n, k, x)
+        b = cuda_lib.gemm(codes, scales, n, k, x)  # one row: the mma.sync kernel
+        try:
+            cuda_lib.tq_debug_set_flags(USE_TMEM)
+            c = cuda_lib.gemm(codes, scales, n, k, x)
+        finally:
+            cuda_lib.tq_debug_set_flags(0)
         torch.cuda.synchronize()
         assert torch.equal(a, b)
+        assert _rel_l2(a.cpu().numpy(), c.cpu().numpy().astype(np.float64)).max() <= REL_L2_TOL
 
 
 def test_workspace_errors(cuda_lib):
@@ -237,8 +262,8 @@ def test_workspace_errors(cuda_lib):
     need = cuda_lib.tq_gemm_workspace_bytes(1, n, k)
     ws = torch.zeros(need + 512, dtype=torch.uint8, device=DEV)
     st = cuda_lib.tq_gemv(codes.data_ptr(), scales.data_ptr(), n, k, x.data_ptr(), 1, y.data_ptr(), 0,
-                          ws.data_ptr(), need - 1, torch.cuda.current_stream().cuda_stream)
-    assert st == 5
+                          ws.data_ptr(), 255, torch.cuda.current_stream().cuda_stream)
+    assert st == 5  # smaller than the header alone
     st = cuda_lib.tq_gemv(codes.data_ptr(), scales.data_ptr(), n, k, x.data_ptr(), 1, y.data_ptr(), 0,
                           ws.data_ptr() + 16, need, torch.cuda.current_stream().cuda_stream)
     assert st == 5
@@ -256,7 +281,7 @@ def _sample_rows(n, count=24, seed=0):
     return rows
 
 
-def test_llama3_8b_layer_full_size(cuda_lib):
+def test_llama3_8b_layer_full_size(cuda_lib, kernel):
     weights, acts = inputs.llama3_8b_layer(device=DEV)
     for name, W in weights.items():
         n, k = W.shape
@@ -276,7 +301,7 @@ def test_llama3_8b_layer_full_size(cuda_lib):
 
 
 @pytest.mark.parametrize("m", [1, 2, 4, 8, 16, 24, 32])
-def test_ffn_70b_skinny_sweep_full_size(cuda_lib, m):
+def test_ffn_70b_skinny_sweep_full_size(cuda_lib, kernel, m):
     n, k = inputs.FFN_70B["gate"]
     W = inputs.gaussian_matrix(2, 0, n, k, 0.015, BF16, DEV)
     X = inputs.gaussian_matrix(1, 100 + m, m, k, 1.0, BF16, DEV)
@@ -290,7 +315,7 @@ def test_ffn_70b_skinny_sweep_full_size(cuda_lib, m):
 
 
 @pytest.mark.parametrize("m", [1, 2, 3, 4, 5])
-def test_gemm_batch_shares_prerotation(cuda_lib, m):
+def test_gemm_batch_shares_prerotation(cuda_lib, kernel, m):
     """Six matrices with three distinct inputs in one batch (q/k/v-style and
     gate/up-style sharing) against the oracle and the one-matrix path."""
     shapes = [(256, 1024, "a"), (64, 1024, "a"), (64, 1024, "a"), (300, 512, "b"), (300, 512, "b"), (40, 2048, "c")]
@@ -313,7 +338,7 @@ def test_gemm_batch_shares_prerotation(cuda_lib, m):
         np.testing.assert_allclose(Y.cpu().numpy(), single.cpu().numpy(), rtol=1e-5, atol=1e-6)
 
 
-def test_timeout_path_reports_and_recovers(cuda_lib):
+def test_timeout_path_reports_and_recovers(cuda_lib, kernel):
     """Fault injection on the host side of the contract: one bulk copy is never
     issued, the kernel's bounded wait (5 ms under injection) expires, it sets
     the workspace status word and returns; the context stays usable."""
@@ -324,12 +349,13 @@ def test_timeout_path_reports_and_recovers(cuda_lib):
     ws = cuda_lib.workspace(1, n, k)
     y_good = cuda_lib.gemv(codes, scales, n, k, x, ws=ws).clone()
     assert cuda_lib.workspace_status(ws) == 0
+    base = USE_TMEM if kernel == "tmem" else USE_MMA_SYNC
     try:
-        cuda_lib.tq_debug_set_flags(1)
+        cuda_lib.tq_debug_set_flags(base | 1)
         cuda_lib.gemv(codes, scales, n, k, x, ws=ws)
         assert cuda_lib.workspace_status(ws) == 8  # TQ_ERR_TIMEOUT
     finally:
-        cuda_lib.tq_debug_set_flags(0)
+        cuda_lib.tq_debug_set_flags(base)
     y = cuda_lib.gemv(codes, scales, n, k, x, ws=ws)
     assert cuda_lib.workspace_status(ws) == 0
     assert torch.equal(y, y_good)
@@ -363,7 +389,7 @@ def test_gemv_correct_while_another_stream_holds_the_sms(cuda_lib):
 
 
 @pytest.mark.parametrize("m", [1, 3, 17])
-def test_gemm_writes_nothing_past_its_outputs(cuda_lib, m):
+def test_gemm_writes_nothing_past_its_outputs(cuda_lib, kernel, m):
     """Guard bands: with n inside the last 16-row tile (rows past n exist in
     the packed planes) and ldy > n, every column past n and every row past m
     keeps its sentinel."""
@@ -387,7 +413,7 @@ def test_gemm_writes_nothing_past_its_outputs(cuda_lib, m):
 
 
 @pytest.mark.parametrize("m", [1, 8, 32])
-def test_gemm_small_weights(cuda_lib, m):
+def test_gemm_small_weights(cuda_lib, kernel, m):
     """Weights of std 1e-4: half-block scales d around 6e-4, so the products
     fp16(c * d) of the smallest centroid fall near the bottom of the fp16
     normal range (6.1e-5), and some below it."""

@@ -100,8 +100,11 @@ def test_static_scratch_timeout_is_reported_and_recovers(cuda_lib):
 
 def test_static_scratch_rejects_oversized_problems(cuda_lib):
     tq = cuda_lib
-    n, k = 1 << 20, 4096  # partial sums alone exceed the fixed scratch
+    # the pre-rotated activation alone (2 bytes per column) exceeds the fixed
+    # scratch, whichever kernel would run the product
+    n, k = 16, 1 << 22
     assert tq.tq_gemm_workspace_bytes(1, n, k) > (4 << 20)
+    assert 2 * k > (4 << 20)
     st = tq.tq_gemv_static_scratch(1 << 20, 1 << 20, n, k, 1 << 20, tq.TQ_BF16, 1 << 20, tq.TQ_F32,
                                    torch.cuda.current_stream().cuda_stream)
     assert st == 2  # TQ_ERR_SHAPE, returned before anything is launched
