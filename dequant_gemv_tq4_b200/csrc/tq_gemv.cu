@@ -110,6 +110,7 @@ constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusLayout = 2u;
 constexpr uint64_t kTimeoutNs = 1000000000ull;     // 1 s
 constexpr uint64_t kDebugTimeoutNs = 5000000ull;   // 5 ms under fault injection
+constexpr uint64_t kStealAfterNs = 50000ull;       // 50 us (later contributors store at the start of their ranges)
 
 
 // Dynamic shared memory to request for a dynamic base of `base` bytes.
@@ -140,7 +141,9 @@ struct GroupParams {
     uint64_t *partials;  // tagged partial sums (value bits | call tag << 32)
     unsigned *header;    // workspace header: status word, call tag
     uint64_t timeout_ns;
+    uint64_t steal_after_ns;  // a split tile's first warp computes a contribution missing for this long
     int inject_skip;
+    int steal_all;            // test hook: compute every later contribution instead of reading it
     double inv_units;  // 1.0 / units and 1.0 / total_warps (host-computed):
     double inv_warps;  // the split arithmetic divides without 64-bit integer division
 };
@@ -433,112 +436,6 @@ __device__ __forceinline__ int lane_xrow(int a, int g, int m) {
     else return min(g / (8 / CM), m - 1);
 }
 
-// The first contributor of a split tile: its own sums plus those of warps
-// gw+1 .. last, the owner of the tile's last unit (the largest w with
-// floor(w*U/W) <= x), added in warp order once each word carries the tag.
-template <int NT, int CM, int OT>
-__device__ __noinline__ void reduce_first(const GroupParams &P, int q, int r, int tile_hi, int gw, uint32_t tag,
-                                          AccTile<NT> acc) {
-    constexpr int kMcap = 8 * NT;
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const DevProblem &pr = P.prob[q];
-    const int64_t gt = pr.tile_begin + r;
-    const int U = (int)P.units, W = P.total_warps;
-    const int last = (int)div_floor((int64_t)tile_hi * W - 1, U, P.inv_units);
-    const uint64_t *base = P.partials + (gt + gw + 1) * (int64_t)(16 * kMcap);
-    uint64_t t0 = 0;
-    bool timed_out = false;
-#pragma unroll
-    for (int a = 0; a < NT; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int xrow = acc_xrow<CM>(a, b, t);
-            const int wl = g + ((b & 2) ? 8 : 0);
-            if (xrow >= P.m) continue;
-            const uint64_t *src = base + xrow * 16 + wl;
-            float sum = acc.v[a][b];
-            for (int w0 = gw + 1; w0 <= last; w0 += 8) {
-                const int cnt = min(8, last - w0 + 1);
-                uint64_t v[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)  // up to eight loads in flight
-                    if (i < cnt) v[i] = ld_relaxed_u64(src + (int64_t)(w0 - gw - 1 + i) * (16 * kMcap));
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (i >= cnt) break;
-                    for (uint32_t it = 0; (uint32_t)(v[i] >> 32) != tag && !timed_out; ++it) {
-                        if (t0 == 0) t0 = global_ns();
-                        if ((it & 63u) == 63u && (global_ns() - t0 > P.timeout_ns || it >= (1u << 30)))
-                            timed_out = true;
-                        v[i] = ld_relaxed_u64(src + (int64_t)(w0 - gw - 1 + i) * (16 * kMcap));
-                    }
-                    sum += __uint_as_float((uint32_t)v[i]);
-                }
-            }
-            const int wrow = r * 16 + wl;
-            if (!timed_out && wrow < pr.n) store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum);
-        }
-    if (timed_out) atomicOr(P.header + kHeaderStatus, kStatusTimeout);
-}
-
-// Write the accumulators of a finished tile segment: straight to Y when this
-// warp covered the whole tile, else through the tagged partial sums.
-//
-// A tile split over warps gw0 < ... < gwk: the tile starts in gw0's range and
-// is that warp's last segment, reached at the end of its work; for every
-// later contributor it is the first segment, reached at the start.  So the
-// later contributors store their sums, each as one 64-bit word (fp32 value,
-// call tag), with no fence and no atomic, and gw0 adds them (own part first,
-// then warp order: deterministic), polling until each word carries this
-// call's tag.  The wait is bounded in time and reports a timeout.
-template <int NT, int CM, int OT>
-__device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
-                                           int u1, int gw, uint32_t tag, const float (&acc_in)[NT][4]) {
-    constexpr int kMcap = 8 * NT;
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const DevProblem &pr = P.prob[q];
-    float acc[NT][4];
-    const float ts = pr.tscale ? __ldg(pr.tscale) : 1.0f;  // NVFP4 tensor scale
-#pragma unroll
-    for (int a = 0; a < NT; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = acc_in[a][b] * ts;
-    const int64_t gt = pr.tile_begin + r;
-    const int row_g = r * 16 + g, row_g8 = row_g + 8;
-    if (u0 <= tile_lo && tile_hi <= u1) {
-#pragma unroll
-        for (int a = 0; a < NT; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int xrow = acc_xrow<CM>(a, b, t);
-                const int wrow = (b & 2) ? row_g8 : row_g;
-                if (xrow < P.m && wrow < pr.n)
-                    store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, acc[a][b]);
-            }
-        return;
-    }
-    const uint64_t tag_hi = (uint64_t)tag << 32;
-    if (tile_lo < u0) {  // a later contributor: store the tagged sums and go on
-        uint64_t *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
-#pragma unroll
-        for (int a = 0; a < NT; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int xrow = acc_xrow<CM>(a, b, t);
-                const int wrow = g + ((b & 2) ? 8 : 0);
-                if (xrow < P.m) st_relaxed_u64(slot + xrow * 16 + wrow, tag_hi | __float_as_uint(acc[a][b]));
-            }
-        return;
-    }
-    // the first contributor (kept out of line: rare, and register hungry)
-    AccTile<NT> own;
-#pragma unroll
-    for (int a = 0; a < NT; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) own.v[a][b] = acc[a][b];
-    reduce_first<NT, CM, OT>(P, q, r, tile_hi, gw, tag, own);
-}
-
 // Products of one unit (16 rows x 128 columns) accumulated into acc: the
 // unit's codes at shared address sc, its scales at ss, the activation
 // fragments at xcur[a] + xoff.
@@ -740,16 +637,22 @@ __device__ __forceinline__ void unit_any(uint32_t sc, uint32_t ss, const uint16_
     }
 }
 
-// The tile segment ending at unit u is complete: write it out, reset the
-// accumulators and move the segment state to the tile of unit u.
-template <int NT, int CM, int OT, int CODEC>
-__device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0, int u1, int gw, int g, int t,
-                                         uint32_t tag, int &q,
-                                         int &prob_end, int &nsb, int &r, int &tile_lo, int &seg_end,
-                                         const uint16_t *(&xcur)[NT], float (&acc)[NT][4]) {
+// What the first contributor of a split tile needs to compute a missing
+// contribution itself: a free shared-memory stage of its ring and its lane
+// constants for the unit products.
+struct StealCtx {
+    uint32_t smem;
+    uint32_t lut_lane;
+    uint32_t off_c;
+    uint32_t off_x;
+};
+
+// Half-block-combination kernels: add the two halves of every weight row,
+// then the blocks the lanes of one activation row share (as when a tile
+// segment ends).
+template <int NT, int CM>
+__device__ __forceinline__ void combine_rows(float (&acc)[NT][4]) {
     if constexpr (CM > 0) {
-        // weight rows g, g + 8: add the two halves, then the blocks the lanes
-        // of one activation row share (four lanes for CM = 1, two for CM = 2)
         float vg = acc[0][0] + acc[0][1], vg8 = acc[0][2] + acc[0][3];
         if constexpr (CM <= 2) {
             vg += __shfl_xor_sync(kFull, vg, 1);
@@ -762,6 +665,191 @@ __device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0,
         acc[0][0] = vg;
         acc[0][2] = vg8;
     }
+}
+
+// The sums warp w would store for its part [va, vb) of tile (q, r),
+// recomputed by this warp (same units, same order, same arithmetic: the
+// result is bit-identical).  Each unit is copied into the free stage with
+// plain loads and multiplied as in the main loop.
+template <int NT, int CM, int CODEC>
+__device__ __noinline__ AccTile<NT> steal_partial(const GroupParams &P, int q, int va, int vb, const StealCtx &cx) {
+    using CT = CodecTraits<CODEC>;
+    constexpr int SB = CT::kScaleBytes;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const DevProblem &pr = P.prob[q];
+    float acc[NT][4];
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    for (int v = va; v < vb; ++v) {
+        const int local = v - (int)pr.unit_begin;
+        const int sb = local % pr.nsb;
+        const uint8_t *c = pr.codes + (int64_t)local * kUnitCodeBytes;
+        const uint8_t *sc = pr.scales + (int64_t)local * SB;
+        const uint4 c0 = ldg_keep(c + 32 * lane), c1 = ldg_keep(c + 32 * lane + 16);
+        __syncwarp();  // the previous unit's products have read the stage
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(cx.smem + 32 * lane), "r"(c0.x), "r"(c0.y),
+                     "r"(c0.z), "r"(c0.w)
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(cx.smem + 32 * lane + 16), "r"(c1.x), "r"(c1.y),
+                     "r"(c1.z), "r"(c1.w)
+                     : "memory");
+        if (lane < SB / 16) {
+            const uint4 s4 = ldg_keep(sc + 16 * lane);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(cx.smem + kUnitCodeBytes + 16 * lane),
+                         "r"(s4.x), "r"(s4.y), "r"(s4.z), "r"(s4.w)
+                         : "memory");
+        }
+        __syncwarp();
+        const uint16_t *xcur[NT];
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+            xcur[a] = pr.xrot + ((int64_t)lane_xrow<CM>(a, g, P.m) * pr.nsb + sb) * 128 + t * 8;
+        unit_any<NT, CM, CT>(cx.smem, cx.smem + kUnitCodeBytes, xcur, 0, cx.lut_lane, cx.off_c, cx.off_x, g, t, acc);
+    }
+    __syncwarp();
+    combine_rows<NT, CM>(acc);
+    const float ts = pr.tscale ? __ldg(pr.tscale) : 1.0f;  // NVFP4 tensor scale
+    AccTile<NT> out;
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) out.v[a][b] = acc[a][b] * ts;
+    return out;
+}
+
+// The first contributor of a split tile: its own sums plus those of warps
+// gw+1 .. last (the owner of the tile's last unit), added in warp order.
+// The later contributors store their sums at the start of their ranges, so
+// normally every word already carries this call's tag; a contribution still
+// missing after a short bounded poll (its warp may not have been able to
+// start: nothing guarantees that the grid is resident at once) is computed
+// here from the packed weights instead.  Nothing waits unboundedly for
+// another CTA, and the result is the same bits either way.
+template <int NT, int CM, int OT, int CODEC>
+__device__ __noinline__ void reduce_first(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int gw,
+                                          uint32_t tag, AccTile<NT> acc, uint32_t smem, uint32_t lut_lane,
+                                          uint32_t off_c, uint32_t off_x) {
+    constexpr int kMcap = 8 * NT;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const DevProblem &pr = P.prob[q];
+    const int64_t gt = pr.tile_begin + r;
+    const int U = (int)P.units, W = P.total_warps;
+    const int last = (int)div_floor((int64_t)tile_hi * W - 1, U, P.inv_units);
+    const StealCtx cx = {smem, lut_lane, off_c, off_x};
+    const float ts = pr.tscale ? __ldg(pr.tscale) : 1.0f;  // NVFP4 tensor scale
+    AccTile<NT> sum;
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) sum.v[a][b] = acc.v[a][b] * ts;
+    uint64_t t0 = 0;
+    for (int w = gw + 1; w <= last; ++w) {
+        const uint64_t *slot = P.partials + (gt + w) * (int64_t)(16 * kMcap);
+        bool present = false;
+        AccTile<NT> part;
+        for (uint32_t it = 0;; ++it) {  // bounded poll for the tagged words
+            bool ok = !P.steal_all;
+#pragma unroll
+            for (int a = 0; a < NT; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int xrow = acc_xrow<CM>(a, b, t);
+                    part.v[a][b] = 0.f;
+                    if (xrow >= P.m) continue;
+                    const uint64_t v = ld_relaxed_u64(slot + xrow * 16 + g + ((b & 2) ? 8 : 0));
+                    ok = ok && (uint32_t)(v >> 32) == tag;
+                    part.v[a][b] = __uint_as_float((uint32_t)v);
+                }
+            present = __all_sync(kFull, ok);
+            if (present || P.steal_all) break;
+            if (t0 == 0) t0 = global_ns();
+            if (global_ns() - t0 > P.steal_after_ns || it >= (1u << 24)) break;
+        }
+        if (!present) {
+            const int64_t wa = div_floor((int64_t)w * U, W, P.inv_warps), wb = div_floor((int64_t)(w + 1) * U, W, P.inv_warps);
+            part = steal_partial<NT, CM, CODEC>(P, q, (int)max(wa, (int64_t)tile_lo), (int)min(wb, (int64_t)tile_hi),
+                                                cx);
+        }
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) sum.v[a][b] += part.v[a][b];
+    }
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int xrow = acc_xrow<CM>(a, b, t);
+            const int wrow = r * 16 + g + ((b & 2) ? 8 : 0);
+            if (xrow < P.m && wrow < pr.n)
+                store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, sum.v[a][b]);
+        }
+}
+
+// Write the accumulators of a finished tile segment: straight to Y when this
+// warp covered the whole tile, else (a later contributor of a split tile)
+// through the tagged partial sums.
+//
+// A tile split over warps gw0 < ... < gwk: the tile starts in gw0's range and
+// is that warp's last segment, reached at the end of its work; for every
+// later contributor it is the first segment, reached at the start.  So the
+// later contributors store their sums, each as one 64-bit word (fp32 value,
+// call tag), with no fence and no atomic, and gw0 adds them (own part first,
+// then warp order: deterministic) in reduce_first, after its main loop.
+template <int NT, int CM, int OT>
+__device__ __forceinline__ void flush_segment(const GroupParams &P, int q, int r, int tile_lo, int tile_hi, int u0,
+                                           int u1, int gw, uint32_t tag, const float (&acc_in)[NT][4]) {
+    constexpr int kMcap = 8 * NT;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const DevProblem &pr = P.prob[q];
+    float acc[NT][4];
+    const float ts = pr.tscale ? __ldg(pr.tscale) : 1.0f;  // NVFP4 tensor scale
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = acc_in[a][b] * ts;
+    const int64_t gt = pr.tile_begin + r;
+    const int row_g = r * 16 + g, row_g8 = row_g + 8;
+    if (u0 <= tile_lo && tile_hi <= u1) {
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int xrow = acc_xrow<CM>(a, b, t);
+                const int wrow = (b & 2) ? row_g8 : row_g;
+                if (xrow < P.m && wrow < pr.n)
+                    store1<OT>(pr.y + ((int64_t)xrow * pr.ldy + wrow) * ElemSize<OT>::value, acc[a][b]);
+            }
+        return;
+    }
+    // a later contributor: store the tagged sums and go on
+    const uint64_t tag_hi = (uint64_t)tag << 32;
+    uint64_t *slot = P.partials + (gt + gw) * (int64_t)(16 * kMcap);
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int xrow = acc_xrow<CM>(a, b, t);
+            const int wrow = g + ((b & 2) ? 8 : 0);
+            if (xrow < P.m) st_relaxed_u64(slot + xrow * 16 + wrow, tag_hi | __float_as_uint(acc[a][b]));
+        }
+}
+
+// The tile segment ending at unit u is complete: write it out, reset the
+// accumulators and move the segment state to the tile of unit u.
+template <int NT, int CM, int OT, int CODEC>
+__device__ __forceinline__ void end_segment(const GroupParams &P, int u, int u0, int u1, int gw, int g, int t,
+                                         uint32_t tag, int &q,
+                                         int &prob_end, int &nsb, int &r, int &tile_lo, int &seg_end,
+                                         const uint16_t *(&xcur)[NT], float (&acc)[NT][4]) {
+    // weight rows g, g + 8: add the two halves, then the blocks the lanes of
+    // one activation row share (four lanes for CM = 1, two for CM = 2)
+    combine_rows<NT, CM>(acc);
+    // the first contributor of a split tile meets it at the end of its range
+    // (u == u1): its sums stay in acc for reduce_first after the main loop
+    if (tile_lo >= u0 && tile_lo + nsb > u1) return;
     flush_segment<NT, CM, OT>(P, q, r, tile_lo, tile_lo + nsb, u0, u1, gw, tag, acc);
 #pragma unroll
     for (int a = 0; a < NT; ++a)
@@ -953,6 +1041,16 @@ __global__ void __launch_bounds__(warps_for(CM > 0, NT) * 32, 1) gemv_group_kern
         stage = (stage == kStages - 1) ? 0 : stage + 1;
         parity ^= (stage == 0) ? 1u : 0u;
     }
+    // the first contributor of a split tile (its last segment, still in acc);
+    // no copy is in flight any more, so the ring may serve as scratch
+    if (tile_lo >= u0 && tile_lo + nsb > u1) {
+        AccTile<NT> own;
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) own.v[a][b] = acc[a][b];
+        reduce_first<NT, CM, OT, CODEC>(P, q, r, tile_lo, tile_lo + nsb, gw, tag, own, ring, lut_lane, off_c, off_x);
+    }
 }
 
 // Base offset of dynamic shared memory in a CTA's shared window (the
@@ -982,17 +1080,14 @@ cudaError_t launch_nt(const GroupParams &prm, int dtype, int grid, bool programm
     cfg.blockDim = dim3(G::kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
-    // Cooperative: the whole grid (at most one CTA per SM) is resident at
-    // once, which the split-tile reduction relies on (a tile's first warp
-    // polls for the partial sums of later CTAs; a CTA that could not start
-    // until the first one exited would make that poll run out).
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    // (no warp depends on another CTA being resident: a split tile's first warp
+    // computes a contribution that does not arrive, so a plain launch, which
+    // may start on the SMs that the previous kernel frees, is enough)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = programmatic ? 2 : 1;
+    cfg.numAttrs = programmatic ? 1 : 0;
     cudaError_t err;
     switch (dtype) {
         case kF32:
@@ -1073,6 +1168,8 @@ cudaError_t launch_group_codec(const GemvProblem *probs, int count, int64_t m, i
     prm.inv_units = 1.0 / (double)prm.units;
     prm.inv_warps = 1.0 / (double)prm.total_warps;
     prm.timeout_ns = prm.inject_skip ? kDebugTimeoutNs : kTimeoutNs;
+    prm.steal_after_ns = kStealAfterNs;
+    prm.steal_all = (g_debug_flags & kDebugStealAll) ? 1 : 0;
     // the partial-slot stride is 16 * 8 * NT floats: NT must match plan.mcap
     const int nt = plan.mcap / 8;
     const int cm = nt == 1 ? combo_rows(m) : 0;

@@ -112,6 +112,10 @@ constexpr uint32_t kDebugSkipPrefillCopy = 2u;
 // tests and measurements cover both kernels at every m)
 constexpr uint32_t kDebugUseTmem = 4u;
 constexpr uint32_t kDebugUseMmaSync = 8u;
+// bit 4: in the mma.sync kernel, the first warp of every split tile computes
+// the later contributions itself instead of reading them (the path taken
+// when a contributor cannot run)
+constexpr uint32_t kDebugStealAll = 16u;
 void set_debug_flags(uint32_t flags);
 uint32_t debug_flags();
 

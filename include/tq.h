@@ -289,7 +289,12 @@ TQ_API tq_status tq_workspace_status(void *workspace, int clear, void *stream);
  * issued, so its bounded wait expires after ~5 ms and the timeout path runs
  * (status word set, kernel returns normally; no fault, no trap).  Bits 2 and
  * 3: every product with m <= 32 runs on the tensor-memory kernel (bit 2) or
- * on the mma.sync kernel (bit 3) instead of the kernel chosen by m.  Bit 1:
+ * on the mma.sync kernel (bit 3) instead of the kernel chosen by m.  Bit 4:
+ * in the mma.sync kernel the first warp of every split tile recomputes the
+ * later warps' contributions from the packed weights instead of reading
+ * them (the path it takes when a contribution does not arrive within 50 us,
+ * e.g. because another kernel holds the SMs its CTA needs); the result is
+ * bit-identical.  Bit 1:
  * the same for the tensor-core prefill product (tq_gemm_prefill and m > 32):
  * the first CTA never issues its second activation-tile copy (nor counts its
  * bytes), its waits expire after ~5 ms, every tensor-memory column is still

@@ -426,3 +426,46 @@ def test_gemm_small_weights(cuda_lib, kernel, m):
     Y = cuda_lib.gemm(codes, scales, n, k, X.to(DEV))
     torch.cuda.synchronize()
     assert _rel_l2(Y.cpu().numpy(), Y_ref).max() <= REL_L2_TOL
+
+
+STEAL_ALL = 16  # tq_debug_set_flags bit 4: split tiles' first warps compute every later contribution
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 8, 16, 24, 32])
+def test_split_tiles_recomputed_contributions_are_bit_identical(cuda_lib, m):
+    """The mma.sync kernel needs no co-resident grid: a split tile's first
+    warp computes a later contribution that does not arrive in time from the
+    packed weights.  Forced on every split tile (test hook), the products are
+    bit-identical to the normal path, which reads those contributions."""
+    shapes = [(4096, 4096), (300, 14336), (1000, 1056)]
+    for n, k in shapes:
+        W = _w(n, k, BF16, seed=50 + m)
+        X = _w(m, k, BF16, seed=51 + m, std=1.0)
+        codes, scales = cuda_lib.quantize(W.to(DEV))
+        try:
+            cuda_lib.tq_debug_set_flags(USE_MMA_SYNC)
+            ref = cuda_lib.gemm(codes, scales, n, k, X.to(DEV)).clone()
+            cuda_lib.tq_debug_set_flags(USE_MMA_SYNC | STEAL_ALL)
+            got = cuda_lib.gemm(codes, scales, n, k, X.to(DEV))
+        finally:
+            cuda_lib.tq_debug_set_flags(0)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref), (m, n, k)
+
+
+def test_split_tiles_recomputed_nvfp4(cuda_lib):
+    """The same for the NVFP4 product (its tensor scale applies to the
+    recomputed contributions too)."""
+    for m in (1, 16):
+        n, k = 4096, 4096
+        W = _w(n, k, BF16, seed=60 + m)
+        X = _w(m, k, BF16, seed=61 + m, std=1.0).to(DEV)
+        c, s, t = cuda_lib.nvfp4_quantize(W.to(DEV))
+        ref = cuda_lib.nvfp4_gemm(c, s, t, n, k, X).clone()
+        try:
+            cuda_lib.tq_debug_set_flags(STEAL_ALL)
+            got = cuda_lib.nvfp4_gemm(c, s, t, n, k, X)
+        finally:
+            cuda_lib.tq_debug_set_flags(0)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref), m
