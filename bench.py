@@ -48,6 +48,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -74,6 +76,10 @@ def parse_args(argv=None):
     p.add_argument("--skip-codec-comparison", action="store_true",
                    help="skip the NVFP4 vs TQ4_1S comparison on the Llama-3-8B layer shapes")
     p.add_argument("--skip-prefill", action="store_true", help="omit the large-M tensor-core product line")
+    p.add_argument("--skip-ffn", action="store_true", help="omit the 70B-class FFN skinny sweep")
+    p.add_argument("--skip-single", action="store_true", help="omit the single 2048x2048 matrix line")
+    p.add_argument("--skip-comparators", action="store_true",
+                   help="omit dequantise+matmul and dense bf16 GEMV on the same layer")
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     p.add_argument("--cpu-sample-rows", type=int, default=None,
                    help="rows per matrix for the CPU oracle sample (default: half of each matrix)")
@@ -110,6 +116,26 @@ PROFILE_FILES = {  # phase -> committed ncu summary and the sources its kernel i
     "dequantize": ("dequantize_kernel_llama3_8b_down.md", ("tq_device.cuh", "tq_codec.cu")),
     "gemv": ("gemv_group_kernel_llama3_8b_layer.md", ("tq_device.cuh", "tq_gemv.cu")),
 }
+
+
+def profile_field(phase: str, field: str):
+    """A `field: value` line of the phase's committed ncu summary, or None when
+    the kernel source changed since the capture."""
+    import hashlib
+
+    name, sources = PROFILE_FILES[phase]
+    try:
+        text = open(os.path.join(ROOT, "profiles", name)).read()
+        fields = dict(ln.split(": ", 1) for ln in text.splitlines() if ": " in ln)
+        h = hashlib.sha256()
+        for src in sources:
+            with open(os.path.join(ROOT, "dequant_gemv_tq4_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != fields["source_sha256"].strip():
+            return None
+        return fields[field].strip()
+    except Exception:
+        return None
 
 
 def profile_traffic(phase: str, weights: int):
@@ -333,6 +359,23 @@ def time_replays(run, reps: int, flush=None):
     return sum(s.elapsed_time(e) for s, e in zip(starts, ends))
 
 
+def replay_stats(run, reps: int, per_replay: int, flush=None):
+    """CUDA-event time of each of `reps` calls of `run` (each `per_replay`
+    passes), per pass in microseconds: (mean, median, min, max)."""
+    stream = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        if flush is not None:
+            flush()
+        starts[i].record(stream)
+        run()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    us = sorted(1e3 * s.elapsed_time(e) / per_replay for s, e in zip(starts, ends))
+    return statistics.fmean(us), statistics.median(us), us[0], us[-1]
+
+
 def rank_seed(rank: int) -> int:
     """Layer seed of a rank: every rank quantises and multiplies its own layer
     (independent problems, weak scaling, no collective on the data path)."""
@@ -365,36 +408,73 @@ def barrier(world):
         torch.cuda.synchronize()
 
 
-def cpu_oracle_sample(path, rows_per_matrix=None):
-    """The CPU oracle, as it stands, on the first rows of every matrix."""
-    import numpy as np
+CPU_SAMPLE_FRACTION = 8  # the CPU sample: the first 1/8 of every matrix's rows
+
+
+def cpu_sample_rows(n: int, rows_per_matrix=None) -> int:
+    return min(n, rows_per_matrix) if rows_per_matrix else max(16, n // CPU_SAMPLE_FRACTION)
+
+
+def oracle_pass(mats, threads: int):
+    """One pass of the CPU oracle, as it stands, over `mats` (list of
+    (W fp32 numpy [r, k], x fp64 numpy [1, k])): quantise, dequantise and the
+    fp64 GEMV.  With threads > 1 the rows are partitioned into `threads`
+    slices (multiples of 16 rows) run concurrently (the oracle's C routines
+    release the GIL); each slice is the oracle applied to those rows.
+    Returns seconds per phase and the packed bytes produced."""
+    from concurrent.futures import ThreadPoolExecutor
 
     import oracle
 
+    def slices(r):
+        per = max(16, -(-r // threads) // 16 * 16)
+        return [(a, min(r, a + per)) for a in range(0, r, per)]
+
+    tq_s = td_s = tg_s = 0.0
+    packed = 0
+    with ThreadPoolExecutor(max_workers=max(1, threads)) as ex:
+        for W, x in mats:
+            r, k = W.shape
+            parts = slices(r)
+            t0 = time.perf_counter()
+            q = list(ex.map(lambda ab: oracle.quantize(np.ascontiguousarray(W[ab[0]:ab[1]])), parts))
+            t1 = time.perf_counter()
+            list(ex.map(lambda a: oracle.dequantize(a[1][0], a[1][1], a[0][1] - a[0][0], k), zip(parts, q)))
+            t2 = time.perf_counter()
+            list(ex.map(lambda a: oracle.gemm(a[1][0], a[1][1], a[0][1] - a[0][0], k, x), zip(parts, q)))
+            t3 = time.perf_counter()
+            tq_s += t1 - t0
+            td_s += t2 - t1
+            tg_s += t3 - t2
+            packed += sum(c.nbytes + sc.nbytes for c, sc in q)
+    return tq_s, td_s, tg_s, packed
+
+
+def cpu_oracle_sample(path, rows_per_matrix=None):
+    """The CPU oracle, as it stands, on the first rows of every matrix: one
+    core, then the same rows partitioned over every host core."""
+    import oracle
+
     oracle.build()
-    tq_w = tg = td = 0.0
-    weights = packed = 0
+    mats = []
+    weights = 0
     for it in path.items:
         n, k = it["n"], it["k"]
-        r = min(n, rows_per_matrix) if rows_per_matrix else max(1, n // 2)
-        W = it["W"][:r].float().cpu().numpy()
-        x = it["x"].float().cpu().numpy().reshape(1, -1).astype(np.float64)
-        t0 = time.perf_counter()
-        c, s = oracle.quantize(W)
-        t1 = time.perf_counter()
-        oracle.dequantize(c, s, r, k)
-        t2 = time.perf_counter()
-        oracle.gemm(c, s, r, k, x)
-        t3 = time.perf_counter()
-        tq_w += t1 - t0
-        td += t2 - t1
-        tg += t3 - t2
+        r = cpu_sample_rows(n, rows_per_matrix)
+        mats.append((it["W"][:r].float().cpu().numpy(),
+                     it["x"].float().cpu().numpy().reshape(1, -1).astype(np.float64)))
         weights += r * k
-        packed += c.nbytes + s.nbytes
-    return {"gemv_gbs": packed / tg / 1e9, "quantize_gweights_per_s": weights / tq_w / 1e9,
-            "dequantize_gweights_per_s": weights / td / 1e9, "seconds": tq_w + td + tg,
-            "sample": f"first {rows_per_matrix or 'half of the'} rows of each of the {len(path.items)} matrices "
-                      f"({weights / 1e6:.1f} M weights): quantise, dequantise, GEMV"}
+    cores = os.cpu_count() or 1
+    res = {}
+    for label, threads in (("single_core", 1), ("all_cores", cores)):
+        tq_s, td_s, tg_s, packed = oracle_pass(mats, threads)
+        res[label] = {"threads": threads, "gemv_gbs": packed / tg_s / 1e9,
+                      "quantize_gweights_per_s": weights / tq_s / 1e9,
+                      "dequantize_gweights_per_s": weights / td_s / 1e9, "seconds": tq_s + td_s + tg_s}
+    res["sample"] = (f"first {rows_per_matrix or f'1/{CPU_SAMPLE_FRACTION} of the'} rows of each of the "
+                     f"{len(path.items)} matrices ({weights / 1e6:.1f} M weights): quantise, dequantise, GEMV")
+    res["weights"] = weights
+    return res
 
 
 def run_ours(args, world, rank, local):
@@ -447,14 +527,15 @@ def run_ours(args, world, rank, local):
     sampler.start()
     time.sleep(0.4)
     barrier(world)
-    t_step = time_replays(step_run, steps)
+    st_step = replay_stats(step_run, steps, R)
     barrier(world)
-    t_q = time_replays(q_run, steps, flush)
-    t_d = time_replays(d_run, steps, flush)
+    st_q = replay_stats(q_run, steps, R, flush)
+    st_d = replay_stats(d_run, steps, R, flush)
     # the GEMV passes alternate between two layers whose packed weights
     # together exceed L2, so they need no flush (a write flush would leave
     # 126 MB of dirty lines for the first pass to write back)
-    t_g = time_replays(g_run, steps)
+    st_g = replay_stats(g_run, steps, R)
+    t_step, t_q, t_d, t_g = (1e-3 * x[0] * steps * R for x in (st_step, st_q, st_d, st_g))
     per_matrix = {}
     for i, it in enumerate(path.items):
         run_i = capture(path.gemv_one(i), use_graph)
@@ -501,6 +582,12 @@ def run_ours(args, world, rank, local):
                                  "ops_per_weight": round(QUANT_OPS_PER_WEIGHT, 4), "ms": round(ms_q, 5),
                                  "peak_note": f"{props.multi_processor_count} SMs x {LANES_PER_SM} lanes x "
                                               f"{max_mhz:.0f} MHz, one operation per lane per cycle"}
+    ipw = profile_field("quantize", "thread_instructions_per_weight")
+    rooflines["quantize_alu"]["measured_instructions_per_weight"] = float(ipw) if ipw is not None else None
+    rooflines["quantize_alu"]["instructions_note"] = (
+        "ops_per_weight counts the codec's defined operations; measured_instructions_per_weight is ncu's "
+        "thread-instruction count per weight for the same kernel (committed summary), null if the kernel "
+        "changed since")
     top = rooflines["quantize_alu"] if dominant == "quantize" else rooflines[dominant]
 
     line = {
@@ -519,6 +606,10 @@ def run_ours(args, world, rank, local):
         "quantize_gweights_per_s": round(quant_gw, 2),
         "phases_ms": {"quantize": round(ms_q, 5), "dequantize": round(ms_d, 5), "gemv": round(ms_g, 5)},
         "gemv_single_matrix": per_matrix,
+        "phase_stats_us": {ph: {"mean": round(v[0], 3), "median": round(v[1], 3), "min": round(v[2], 3),
+                                "max": round(v[3], 3)}
+                           for ph, v in (("step", st_step), ("quantize", st_q), ("dequantize", st_d),
+                                         ("gemv", st_g))},
         "roofline": dict(top, kernel=dominant, **({} if dominant == "quantize" else
                                                   {"peak_note": f"{hbm_kind} HBM copy bandwidth"})),
         "rooflines": rooflines,
@@ -536,12 +627,32 @@ def run_ours(args, world, rank, local):
     if args.workload == "llama3_8b_layer" and not args.skip_codec_comparison:
         line["codec_comparison"] = codec_comparison(tq, path, rank, device, min(steps, 10), warmup, flush, use_graph,
                                                     world)
+    if args.workload == "llama3_8b_layer" and not args.skip_comparators:
+        cmp = comparators(tq, path, device, min(steps, 10), warmup, use_graph, world, hbm)
+        fused_us = 1e3 * ms_g
+        for key in ("dequant_then_matmul", "dense_bf16_gemv"):
+            cmp[key]["vs_fused"] = round(cmp[key]["us_mean"] / fused_us, 2)
+        cmp["fused_us"] = round(fused_us, 2)
+        line["comparators"] = cmp
+    if args.workload == "llama3_8b_layer" and not args.skip_ffn:
+        line["ffn_70b"] = ffn70b_sweep(tq, rank, device, min(steps, 10), warmup, use_graph, world, hbm)
+    if args.workload == "llama3_8b_layer" and not args.skip_single:
+        line["single_matrix"] = single_matrix_measure(tq, device, min(steps, 10), warmup, use_graph, hbm)
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         cb = cpu_oracle_sample(path, args.cpu_sample_rows)
-        line["cpu_baseline"] = {"value": round(cb["gemv_gbs"], 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": cb["sample"],
-                                "quantize_gweights_per_s": round(cb["quantize_gweights_per_s"], 5),
-                                "seconds": round(cb["seconds"], 1)}
+        allc, one = cb["all_cores"], cb["single_core"]
+        line["cpu_baseline"] = {"value": round(allc["gemv_gbs"], 4), "unit": UNIT, "cores": allc["threads"],
+                                "kind": "oracle", "sample": cb["sample"],
+                                "quantize_gweights_per_s": round(allc["quantize_gweights_per_s"], 5),
+                                "dequantize_gweights_per_s": round(allc["dequantize_gweights_per_s"], 5),
+                                "seconds": round(allc["seconds"], 2),
+                                "partition": "rows split into one slice per core (multiples of 16), the oracle "
+                                             "as it stands applied to each slice on its own thread",
+                                "single_core": {"value": round(one["gemv_gbs"], 4), "cores": 1,
+                                                "quantize_gweights_per_s": round(one["quantize_gweights_per_s"], 5),
+                                                "dequantize_gweights_per_s":
+                                                    round(one["dequantize_gweights_per_s"], 5),
+                                                "seconds": round(one["seconds"], 2)}}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -655,6 +766,151 @@ def codec_comparison(tq, path, rank, device, steps, warmup, flush, use_graph, wo
         entry["packed_bytes"] = packed
         result[codec] = entry
     return result
+
+
+def ffn70b_sweep(tq, rank, device, steps, warmup, use_graph, world, hbm):
+    """The 70B-class FFN (gate, up 28672 x 8192; down 8192 x 28672; bf16
+    ~N(0, 0.015^2)) at m = 1, 2, 4, 8, 16, 32 activation rows (bf16 ~N(0, 1)):
+    one batched product over the three matrices per pass (gate and up share
+    their input, down has its own), 440 MB of packed weights per pass (> L2,
+    no flush needed), with the kernel the library picks for m; from m = 9 the
+    mma.sync kernel forced by the test hook is timed beside it for context."""
+    from dequant_gemv_tq4_b200 import inputs
+
+    R = 5
+    packs, shapes = [], []
+    for tid, (label, (n, k)) in enumerate(inputs.FFN_70B.items()):
+        W = inputs.gaussian_matrix(2 + rank_seed(rank), tid, n, k, 0.015, torch.bfloat16, device)
+        packs.append(tq.quantize(W))
+        shapes.append((label, n, k))
+        del W
+    packed = sum(c.numel() + 2 * s.numel() for c, s in packs)
+    weights = sum(n * k for _, n, k in shapes)
+    xs = {k: inputs.gaussian_matrix(1, 200 + i, 32, k, 1.0, torch.bfloat16, device)
+          for i, k in enumerate(sorted({k for _, _, k in shapes}))}
+    res = {"workload": "ffn_70b: gate, up 28672x8192 and down 8192x28672, bf16 ~N(0,0.015^2), X bf16 ~N(0,1)",
+           "packed_bytes": packed, "passes_per_replay": R, "sweep": {}}
+    for m in (1, 2, 4, 8, 16, 32):
+        entry = {}
+        for label, flag in (("default", 0), ("mma_sync", 8)):
+            if label == "mma_sync" and m < 9:
+                continue
+            tq.tq_debug_set_flags(flag)
+            try:
+                items = [(c, s, n, k, xs[k][:m], torch.empty((m, n), dtype=torch.float32, device=device))
+                         for (c, s), (_, n, k) in zip(packs, shapes)]
+                descs = tq.batch_descs(items)
+                ws = tq.batch_workspace(items, m, device)
+                run = capture(lambda: tq.gemm_batch(items, m=m, ws=ws, descs=descs), use_graph, R)
+                for _ in range(warmup):
+                    run()
+                mean, med, mn, mx = replay_stats(run, steps, R)
+                st = tq.workspace_status(ws)
+            finally:
+                tq.tq_debug_set_flags(0)
+            (mean,) = max_over_ranks([mean], world)
+            gbs = job_gbs(packed, world, mean * 1e-3)
+            entry[label] = {"us_mean": round(mean, 2), "us_median": round(med, 2), "us_min": round(mn, 2),
+                            "us_max": round(mx, 2), "gbs": round(gbs, 1), "pct_of_hbm": round(100 * gbs / world / hbm, 1),
+                            "tflops": round(2.0 * m * weights * world / (mean * 1e-6) / 1e12, 2), "status": int(st)}
+            if label == "default":
+                entry[label]["kernel"] = "tcgen05 (tensor memory)" if m >= 9 else "mma.sync"
+        res["sweep"][f"m{m}"] = entry
+    del packs
+    return res
+
+
+def single_matrix_measure(tq, device, steps, warmup, use_graph, hbm):
+    """The single 2048 x 2048 fp32 matrix (~N(0, 0.02^2), seed 0) with an fp32
+    activation (~N(0,1), seed 1): quantise, dequantise and the GEMV.  Its
+    packed weights (2.6 MB) fit in L2, so the GEMV passes cycle through 64
+    independently packed copies (168 MB > L2) to read from HBM; the quantise
+    passes read the fp32 weights after a 256 MB L2 flush."""
+    from dequant_gemv_tq4_b200 import inputs
+
+    W, x = inputs.single_matrix(device=device)
+    n, k = W.shape
+    copies = []
+    for i in range(64):
+        Wi = W if i == 0 else (W * (1.0 + 2.0 ** -10 * i))
+        copies.append(tq.quantize(Wi))
+    ys = torch.empty((1, n), dtype=torch.float32, device=device)
+    xs = x.view(1, -1)
+    wss = [tq.workspace(1, n, k, device) for _ in range(8)]
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def gemv_all():
+        for i, (c, s) in enumerate(copies):
+            tq.gemm(c, s, n, k, xs, out=ys, ws=wss[i % 8])
+
+    run = capture(gemv_all, use_graph)
+    for _ in range(warmup):
+        run()
+    mean, med, mn, mx = replay_stats(run, steps, len(copies))
+    packed = copies[0][0].numel() + 2 * copies[0][1].numel()
+    codes, scales = tq.tq_codes_bytes(n, k), tq.tq_scales_bytes(n, k)
+    c0 = torch.empty(codes, dtype=torch.uint8, device=device)
+    s0 = torch.empty(scales // 2, dtype=torch.int16, device=device)
+    qrun = capture(lambda: tq.quantize(W, c0, s0), use_graph)
+    for _ in range(warmup):
+        qrun()
+    qmean, qmed, _, _ = replay_stats(qrun, steps, 1, flush=lambda: flush_buf.zero_())
+    return {"workload": "single_matrix_2048: W 2048x2048 fp32 ~N(0,0.02^2) (seed 0), x fp32 ~N(0,1) (seed 1)",
+            "gemv_us_mean": round(mean, 2), "gemv_us_median": round(med, 2), "gemv_us_min": round(mn, 2),
+            "gemv_us_max": round(mx, 2), "gemv_gbs": round(packed / (mean * 1e-6) / 1e9, 1),
+            "gemv_pct_of_hbm": round(100 * packed / (mean * 1e-6) / 1e9 / hbm, 1),
+            "gemv_note": "one tq_gemm call per pass (pre-rotation + product), 64 packed copies cycled (> L2); "
+                         "a 2.6 MB matrix is bound by launch latency, not HBM",
+            "quantize_us": round(qmean, 2), "quantize_gweights_per_s": round(n * k / (qmean * 1e-6) / 1e9, 1)}
+
+
+def comparators(tq, path, device, steps, warmup, use_graph, world, hbm):
+    """Two ways to run the same batch-1 layer without the fused kernel
+    (TQ4_1S page, TQ4_1S 是什么 / 解码速度 sections: the CUDA port converts
+    TQ4_1S to q8_0 at load time and runs a plain kernel):
+      * dequant_then_matmul: tq_dequantize every matrix to bf16, then a
+        cuBLAS bf16 GEMV (torch.matmul) on it, every pass;
+      * dense_bf16_gemv: cuBLAS bf16 GEMV on the unquantised bf16 weights
+        (the weights converted once; 3.2 x the bytes of the packed form),
+        alternating two copies of the layer (2 x 436 MB > L2).
+    GB/s is counted for each method's own weight bytes; `vs_fused` is the
+    method's time over the fused product's time on the same layer."""
+    R = 4
+    deq = [torch.empty((it["n"], it["k"]), dtype=torch.bfloat16, device=device) for it in path.items]
+    outs = [torch.empty((1, it["n"]), dtype=torch.bfloat16, device=device) for it in path.items]
+
+    def dq_mm():
+        for it, d, o in zip(path.items, deq, outs):
+            tq.dequantize(it["codes"], it["scales"], it["n"], it["k"], out=d)
+            torch.matmul(it["x"], d.t(), out=o)
+
+    run = capture(dq_mm, use_graph, R)
+    for _ in range(warmup):
+        run()
+    dq_mean, dq_med, dq_min, dq_max = replay_stats(run, steps, R)
+    shadow_w = [it["W"].clone() for it in path.items]  # a second dense copy: two layers > L2
+
+    def dense():
+        for it, o in zip(path.items, outs):
+            torch.matmul(it["x"], it["W"].t(), out=o)
+        for it, w, o in zip(path.items, shadow_w, outs):
+            torch.matmul(it["x"], w.t(), out=o)
+
+    run2 = capture(dense, use_graph, R)
+    for _ in range(warmup):
+        run2()
+    de_mean, de_med, de_min, de_max = replay_stats(run2, steps, 2 * R)
+    del shadow_w
+    packed, dense_bytes = path.packed_bytes(), path.in_bytes()
+    return {"workload": "llama3_8b_layer at m = 1 (bf16 x, bf16 y)",
+            "dequant_then_matmul": {"us_mean": round(dq_mean, 2), "us_median": round(dq_med, 2),
+                                    "us_min": round(dq_min, 2), "us_max": round(dq_max, 2),
+                                    "packed_gbs": round(packed / (dq_mean * 1e-6) / 1e9, 1)},
+            "dense_bf16_gemv": {"us_mean": round(de_mean, 2), "us_median": round(de_med, 2),
+                                "us_min": round(de_min, 2), "us_max": round(de_max, 2),
+                                "bf16_gbs": round(dense_bytes / (de_mean * 1e-6) / 1e9, 1),
+                                "pct_of_hbm": round(100 * dense_bytes / (de_mean * 1e-6) / 1e9 / hbm, 1)},
+            "bytes": {"packed": packed, "bf16": dense_bytes}}
 
 
 PREFILL_PROFILE = ("prefill_kernel_8192x8192_m2048.md", ("tq_device.cuh", "tq_prefill.cu"))
@@ -772,64 +1028,64 @@ def run_e2e(tq, path, steps, world):
 # reference arm: the CPU oracle on the host cores
 # ---------------------------------------------------------------------------
 def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the host cores --
+    the same row sample as the GPU line's cpu_baseline (the first 1/8 of every
+    matrix's rows), partitioned over every core -- one oracle pass per step
+    (quantise, dequantise, GEMV); the metric is the GEMV phase's GB/s of
+    packed weights, as for the GPU line."""
     if rank != 0:
         return
-    import numpy as np
 
     import oracle
     from dequant_gemv_tq4_b200 import inputs
 
     oracle.build()
-    # same workload, one row sample per step: the first 1/64 of every matrix's rows
     if args.workload == "llama3_8b_layer":
         shapes = [(lbl, n, k, seed) for seed, (lbl, (n, k)) in enumerate(inputs.LLAMA3_8B_LAYER.items())]
     elif args.workload == "single_matrix":
         shapes = [("w", 2048, 2048, 0)]
     else:
         shapes = [(lbl, n, k, tid) for tid, (lbl, (n, k)) in enumerate(inputs.FFN_70B.items())]
-    sample = []
+    mats = []
+    weights = 0
     for lbl, n, k, seed in shapes:
-        r = max(1, n // 64)
+        r = cpu_sample_rows(n, args.cpu_sample_rows)
         # the generator is row-major, so r rows are exactly the matrix's first r rows
         if args.workload == "llama3_8b_layer":
             W = inputs.llama_weight(seed, 0, r, k)
+            x = inputs.gaussian_matrix(1, 7, 1, k, 1.0, torch.bfloat16)
         elif args.workload == "single_matrix":
             W = inputs.gaussian_matrix(0, 0, r, k, 0.02, torch.float32)
+            x = inputs.gaussian_matrix(1, 0, 1, k, 1.0, torch.float32)
         else:
             W = inputs.gaussian_matrix(2, seed, r, k, 0.015, torch.bfloat16)
-        x = inputs.gaussian_matrix(1, 7, 1, k, 1.0, torch.bfloat16).float().numpy().astype(np.float64)
-        sample.append((W.float().numpy(), x, r, k))
-
-    def step():
-        tg = 0.0
-        packed = 0
-        for W, x, r, k in sample:
-            c, s = oracle.quantize(W)
-            oracle.dequantize(c, s, r, k)
-            t0 = time.perf_counter()
-            oracle.gemm(c, s, r, k, x)
-            tg += time.perf_counter() - t0
-            packed += c.nbytes + s.nbytes
-        return packed, tg
-
+            x = inputs.gaussian_matrix(1, 7, 1, k, 1.0, torch.bfloat16)
+        mats.append((W.float().numpy(), x.float().numpy().astype(np.float64)))
+        weights += r * k
+    cores = os.cpu_count() or 1
     for _ in range(max(3, args.warmup)):
-        step()
-    tot_b = tot_t = 0.0
+        oracle_pass(mats, cores)
+    tot_b = tot_t = tot_q = 0.0
     t0 = time.perf_counter()
     for _ in range(max(1, args.steps)):
-        b, t = step()
-        tot_b += b
-        tot_t += t
+        tq_s, td_s, tg_s, packed = oracle_pass(mats, cores)
+        tot_b += packed
+        tot_t += tg_s
+        tot_q += tq_s
     wall = time.perf_counter() - t0
     value = tot_b / tot_t / 1e9
+    sample = (f"first {args.cpu_sample_rows or f'1/{CPU_SAMPLE_FRACTION} of the'} rows of every matrix "
+              f"({weights / 1e6:.1f} M weights) per step, rows split over {cores} threads: quantise, dequantise, GEMV")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
             "steps": max(1, args.steps), "warmup": max(3, args.warmup),
             "ms_per_step": round(1e3 * wall / max(1, args.steps), 2), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "dtype_detail": "CPU oracle: f32 codec in the codec order, f64 product",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "dtype_detail": "CPU oracle: f32 codec in the codec order, f64 product",
             "data": "synthetic (seeded counter-based generator; no checkpoints)",
-            "config": {"workload": args.workload, "sample": "first 1/64 of the rows of every matrix per step"},
-            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": "first 1/64 of the rows of every matrix, quantise + dequantise + GEMV"},
+            "config": {"workload": args.workload, "sample": sample},
+            "quantize_gweights_per_s": round(weights * max(1, args.steps) / tot_q / 1e9, 5),
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

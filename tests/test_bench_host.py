@@ -83,3 +83,21 @@ def test_quantise_alu_operation_count():
     assert block == 434
     assert bench.QUANT_OPS_PER_WEIGHT == pytest.approx(block / 32)
     assert bench.LANES_PER_SM == 128
+
+
+def test_cpu_sample_and_row_partitioned_oracle():
+    """The CPU baseline's sample is the first 1/8 of each matrix's rows
+    (at least 16), and the row-partitioned run applies the oracle to slices
+    of whole 16-row tiles: it produces exactly the packed bytes of the
+    single-threaded run."""
+    import numpy as np
+
+    assert bench.cpu_sample_rows(4096) == 512
+    assert bench.cpu_sample_rows(40) == 16
+    assert bench.cpu_sample_rows(4096, 100) == 100
+    rng = np.random.default_rng(3)
+    mats = [(rng.standard_normal((50, 96)).astype(np.float32) * 0.02, rng.standard_normal((1, 96))),
+            (rng.standard_normal((33, 160)).astype(np.float32) * 0.02, rng.standard_normal((1, 160)))]
+    one = bench.oracle_pass(mats, 1)
+    three = bench.oracle_pass(mats, 3)
+    assert one[3] == three[3] > 0
