@@ -25,18 +25,6 @@ constexpr int kCodecThreads = kCodecWarps * 32;
 __constant__ uint32_t c_thr_bits[7] = TQ_THR_F32_INIT;
 __constant__ uint32_t c_mag_bits[8] = TQ_MAG_F32_INIT;
 
-// Full 32-point transform of the warp's four blocks (see file comment).
-__device__ __forceinline__ void fwht32_warp(float (&v)[4], int p) {
-    butterfly_local4(v);
-#pragma unroll
-    for (int s = 0; s < 3; ++s) {
-        const int x = 1 << s;
-        const bool upper = (p & x) != 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = butterfly_xlane(v[i], x, upper);
-    }
-}
-
 // Index of a row's 64-byte code slot (and 16-byte scale slot) for superblock
 // sb in the tile-major layout [tile][sb][16 rows].
 __device__ __forceinline__ size_t unit_row(int row, int sb, int nsb) {
@@ -363,25 +351,11 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     const RotInput &in = prm.in[q];
     const int64_t local = unit - in.unit_begin;
     const int row = (int)(local / in.nsb), sb = (int)(local % in.nsb);
-    const bool valid = sb * kSbBlocks + j < in.nb && row < prm.m;
     const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (valid) load4<DT>(in.x + ((int64_t)row * in.ldx + col0) * ElemSize<DT>::value, v);
-    if (ROTATE) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = flip(v[i], sign_mask(col0 + i));
-        fwht32_warp(v, p);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = __fmul_rn(v[i], 0.03125f);
-    }
-    const __half2 lo = __floats2half2_rn(v[0], v[1]);
-    const __half2 hi = __floats2half2_rn(v[2], v[3]);
+    __half2 lo, hi;
+    rotate_unit_lane<DT, ROTATE>(in.x, in.ldx, in.nb, prm.m, row, sb, lane, lo, hi);
     if constexpr (LAYOUT == kRotFragment) {
-        // elements 4p, 4p+1 -> t = 2(p&1), q = 2(p>>1) + {0,1}; 4p+2, 4p+3 -> t + 1
-        const size_t blk_words = ((size_t)local * kSbBlocks + j) * 16;  // 32 halves per block
-        const int t0 = 2 * (p & 1), q0 = 2 * (p >> 1);
-        in.xrot[blk_words + (t0 * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&lo);
-        in.xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
+        store_fragment(in.xrot, local, lane, lo, hi);
     } else {
         size_t half_off;
         if constexpr (LAYOUT == kRotPlain) {

@@ -239,4 +239,56 @@ __device__ __forceinline__ void decode_word(uint32_t w, uint32_t (&o)[4]) {
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
+// ---------------------------------------------------------------------------
+// Activation pre-rotation (TQ page, section 解码速度: the activation is
+// rotated once per call with the weights' sign pattern and transform, scaled
+// by 1/32, and stored as fp16).  One warp rotates the 128 columns of one
+// (row, superblock) "rotation unit": lane = 8*j + p holds elements 4p..4p+3 of
+// block j; stages h = 1, 2 run in registers, h = 4, 8, 16 across lanes.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwht32_warp(float (&v)[4], int p) {
+    butterfly_local4(v);
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        const int x = 1 << s;
+        const bool upper = (p & x) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = butterfly_xlane(v[i], x, upper);
+    }
+}
+
+// This lane's four rotated (or, without ROTATE, only converted) values of
+// rotation unit (row, sb) of an activation with nb blocks per row, as two
+// fp16 pairs; blocks past nb and rows >= m give zeros.
+template <int DT, bool ROTATE>
+__device__ __forceinline__ void rotate_unit_lane(const char *x, int64_t ldx, int nb, int m, int row, int sb, int lane,
+                                                 __half2 &lo, __half2 &hi) {
+    const int j = lane >> 3, p = lane & 7;
+    const bool valid = sb * kSbBlocks + j < nb && row < m;
+    const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (valid) load4<DT>(x + ((int64_t)row * ldx + col0) * ElemSize<DT>::value, v);
+    if (ROTATE) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = flip(v[i], sign_mask(col0 + i));
+        fwht32_warp(v, p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = __fmul_rn(v[i], 0.03125f);
+    }
+    lo = __floats2half2_rn(v[0], v[1]);
+    hi = __floats2half2_rn(v[2], v[3]);
+}
+
+// Store of one lane's values in the mma.sync kernel's fragment order: element
+// e of a block goes to slot t*8 + q with t = (e%8)/2, q = 2*(e/8) + e%2
+// (`local` = row * nsb + sb within the input).
+__device__ __forceinline__ void store_fragment(uint32_t *xrot, int64_t local, int lane, __half2 lo, __half2 hi) {
+    const int j = lane >> 3, p = lane & 7;
+    const size_t blk_words = ((size_t)local * kSbBlocks + j) * 16;  // 32 halves per block
+    // elements 4p, 4p+1 -> t = 2(p&1), q = 2(p>>1) + {0,1}; 4p+2, 4p+3 -> t + 1
+    const int t0 = 2 * (p & 1), q0 = 2 * (p >> 1);
+    xrot[blk_words + (t0 * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&lo);
+    xrot[blk_words + ((t0 + 1) * 8 + q0) / 2] = *reinterpret_cast<const uint32_t *>(&hi);
+}
+
 }  // namespace tq

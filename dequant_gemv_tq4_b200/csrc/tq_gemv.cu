@@ -764,8 +764,10 @@ __device__ __noinline__ void reduce_first(const GroupParams &P, int q, int r, in
                 }
             present = __all_sync(kFull, ok);
             if (present || P.steal_all) break;
-            if (t0 == 0) t0 = global_ns();
-            if (global_ns() - t0 > P.steal_after_ns || it >= (1u << 24)) break;
+            if (t0 == 0) t0 = __shfl_sync(kFull, global_ns(), 0);
+            // a vote, so that all 32 lanes stop polling together (a lane that
+            // left alone would leave the others in the next full-warp vote)
+            if (__any_sync(kFull, global_ns() - t0 > P.steal_after_ns || it >= (1u << 24))) break;
         }
         if (!present) {
             const int64_t wa = div_floor((int64_t)w * U, W, P.inv_warps), wb = div_floor((int64_t)(w + 1) * U, W, P.inv_warps);
