@@ -68,16 +68,54 @@ __device__ __forceinline__ void packed_sign_words(uint32_t bits, uint32_t (&ps)[
     for (int i = 0; i < 16; ++i) ps[i] = (((bits >> (2 * i)) & 1u) << 15) | (((bits >> (2 * i + 1)) & 1u) << 31);
 }
 
+// Packed fp32 pairs (sm_100 add/sub.rn.f32x2): each half is one IEEE fp32
+// operation rounded to nearest even, exactly the scalar __fadd_rn/__fsub_rn.
+// Their operands here are loads or scalar products, never a packed product
+// (a packed multiply feeding a packed add may be contracted into an FMA).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t r, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// The 32-point transform in the codec's stage order h = 1, 2, 4, 8, 16.
+// Element t and element t + 16 share one packed register: stages h < 16 pair
+// register t with register t + h (both halves at once), stage 16 combines
+// the two halves of each register in scalar.  Every element sees the same
+// operations on the same operands as the sequential definition.
 __device__ __forceinline__ void fwht32_regs(float (&v)[32]) {
+    uint64_t P[16];
 #pragma unroll
-    for (int h = 1; h < 32; h <<= 1)
+    for (int t = 0; t < 16; ++t) P[t] = pack2(v[t], v[t + 16]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
             if ((i & h) == 0) {
-                const float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
+                const uint64_t a = P[i], b = P[i + h];
+                P[i] = add2(a, b);
+                P[i + h] = sub2(a, b);
             }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+        float lo, hi;
+        unpack2(P[t], lo, hi);
+        v[t] = __fadd_rn(lo, hi);
+        v[t + 16] = __fsub_rn(lo, hi);
+    }
 }
 
 // 32 input elements -> fp32 with the sign flip applied (exact).
@@ -218,64 +256,65 @@ __global__ void __launch_bounds__(kCodecThreads) quantize_kernel(const char *__r
 // -------------------------------------------------------------------------
 // Dequantise: w~ = s .* (H c) / 32, fp32, rounded to the output dtype.
 // The 1/32 is folded into the fp16 scale (exact power-of-two scaling).
+// A warp writes one row segment of 32 blocks per step: each lane's block goes
+// through a per-warp shared-memory stage (16-byte chunks, XOR-placed so that
+// neither side has bank conflicts) and leaves as fully coalesced 512-byte
+// stores; the next row's codes and scales are loaded one step ahead.
 // -------------------------------------------------------------------------
 template <int DT>
-__device__ __forceinline__ void store_block(char *p, uint32_t bits, const uint32_t (&ps)[16], const float (&v)[32]);
+struct DeqOut {
+    static constexpr int kWords = DT == kF32 ? 32 : 16;  // 32-bit output words per block
+    static constexpr int kChunks = kWords / 4;            // 16-byte chunks per block
+};
+
+// A block's output words: elements rounded to DT, sign flip applied.
+template <int DT>
+__device__ __forceinline__ void block_words(uint32_t bits, const uint32_t (&ps)[16], const float (&v)[32],
+                                            uint32_t (&o)[DeqOut<DT>::kWords]);
 
 template <>
-__device__ __forceinline__ void store_block<kF32>(char *p, uint32_t bits, const uint32_t (&)[16],
-                                                  const float (&v)[32]) {
-    uint4 *q = reinterpret_cast<uint4 *>(p);
+__device__ __forceinline__ void block_words<kF32>(uint32_t bits, const uint32_t (&)[16], const float (&v)[32],
+                                                  uint32_t (&o)[32]) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t o[4];
+    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(v[e]) ^ ((bits << (31 - e)) & 0x80000000u);
+}
+
+template <>
+__device__ __forceinline__ void block_words<kBF16>(uint32_t, const uint32_t (&ps)[16], const float (&v)[32],
+                                                   uint32_t (&o)[16]) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int e = 4 * i + c;
-            o[c] = __float_as_uint(v[e]) ^ ((bits << (31 - e)) & 0x80000000u);
-        }
-        q[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int i = 0; i < 16; ++i) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        o[i] = *reinterpret_cast<uint32_t *>(&h) ^ ps[i];
     }
 }
 
 template <>
-__device__ __forceinline__ void store_block<kBF16>(char *p, uint32_t, const uint32_t (&ps)[16],
-                                                   const float (&v)[32]) {
-    uint4 *q = reinterpret_cast<uint4 *>(p);
+__device__ __forceinline__ void block_words<kF16>(uint32_t, const uint32_t (&ps)[16], const float (&v)[32],
+                                                  uint32_t (&o)[16]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t o[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * c], v[8 * i + 2 * c + 1]);
-            o[c] = *reinterpret_cast<uint32_t *>(&h) ^ ps[4 * i + c];
-        }
-        q[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int i = 0; i < 16; ++i) {
+        __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+        o[i] = *reinterpret_cast<uint32_t *>(&h) ^ ps[i];
     }
 }
 
-template <>
-__device__ __forceinline__ void store_block<kF16>(char *p, uint32_t, const uint32_t (&ps)[16],
-                                                  const float (&v)[32]) {
-    uint4 *q = reinterpret_cast<uint4 *>(p);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t o[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            __half2 h = __floats2half2_rn(v[8 * i + 2 * c], v[8 * i + 2 * c + 1]);
-            o[c] = *reinterpret_cast<uint32_t *>(&h) ^ ps[4 * i + c];
-        }
-        q[i] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
+// Stage slot of chunk i of lane l's block: l * C + (i ^ key(l)); within any
+// 8 consecutive lanes writing chunk i, and within any 8 consecutive chunks
+// read back, the slots fall in 8 different 16-byte bank groups.
+template <int C>
+__device__ __forceinline__ int stage_key(int l) {
+    return C == 8 ? (l & 7) : ((l >> 1) & 3);
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_t *__restrict__ codes,
+__global__ void __launch_bounds__(kCodecThreads, DT == kF32 ? 2 : 3) dequantize_kernel(const uint32_t *__restrict__ codes,
                                                                      const uint32_t *__restrict__ scales, int n,
                                                                      int nb, int nsb, char *__restrict__ out,
                                                                      int64_t ldo) {
+    constexpr int C = DeqOut<DT>::kChunks;
     __shared__ float cent[16];  // signed centroids c(code)
+    __shared__ __align__(16) uint4 stage[kCodecWarps * 32 * C];
     if (threadIdx.x < 16) {
         const float m = __uint_as_float(c_mag_bits[threadIdx.x & 7]);
         cent[threadIdx.x] = (threadIdx.x & 8) ? -m : m;
@@ -286,30 +325,65 @@ __global__ void __launch_bounds__(kCodecThreads) dequantize_kernel(const uint32_
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int blk = blockIdx.x * 32 + lane;
     const bool valid = blk < nb;
+    const int nvalid = min(32, nb - (int)blockIdx.x * 32);  // blocks of this column segment
     const int sb = blk >> 2, j = blk & 3;
     const uint32_t k0 = (uint32_t)blk * kBlock;
     const uint32_t bits = block_sign_bits(k0);
     uint32_t ps[16];
     packed_sign_words(bits, ps);
+    uint4 *st = stage + warp * 32 * C;
+    const int key = stage_key<C>(lane);
+    const int64_t seg_col = (int64_t)blockIdx.x * 32 * kBlock;
 
-    for (int row = blockIdx.y * kCodecWarps + warp; row < n; row += gridDim.y * kCodecWarps) {
-        if (!valid) continue;
+    const int rstep = gridDim.y * kCodecWarps;
+    int row = blockIdx.y * kCodecWarps + warp;
+    uint32_t nsw[4] = {0u, 0u, 0u, 0u}, nsc = 0u;  // codes and scales of the next row
+    if (valid && row < n) {
         const size_t slot = unit_row(row, sb, nsb);
-        uint32_t sw[4], lw[4];
 #pragma unroll
-        for (int tt = 0; tt < 4; ++tt) sw[tt] = __ldg(codes + slot * 16 + 4 * tt + j);
-        transpose_bytes(sw, lw);  // the transpose is its own inverse
-        const uint32_t sc = __ldg(scales + slot * 4 + j);
-        const float2 D = __half22float2(*reinterpret_cast<const __half2 *>(&sc));
-        const float Ds[2] = {__fmul_rn(D.x, 0.03125f), __fmul_rn(D.y, 0.03125f)};
+        for (int tt = 0; tt < 4; ++tt) nsw[tt] = __ldg(codes + slot * 16 + 4 * tt + j);
+        nsc = __ldg(scales + slot * 4 + j);
+    }
+    for (; row < n; row += rstep) {
         float v[32];
+        if (valid) {
+            uint32_t sw[4], lw[4];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const uint32_t code = (lw[e >> 3] >> (4 * (e & 7))) & 15u;
-            v[e] = __fmul_rn(lds_f32(cent_base + 4 * code), Ds[e >> 4]);
+            for (int tt = 0; tt < 4; ++tt) sw[tt] = nsw[tt];
+            const uint32_t sc = nsc;
+            if (row + rstep < n) {
+                const size_t slot = unit_row(row + rstep, sb, nsb);
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) nsw[tt] = __ldg(codes + slot * 16 + 4 * tt + j);
+                nsc = __ldg(scales + slot * 4 + j);
+            }
+            transpose_bytes(sw, lw);  // the transpose is its own inverse
+            const float2 D = __half22float2(*reinterpret_cast<const __half2 *>(&sc));
+            const float Ds[2] = {__fmul_rn(D.x, 0.03125f), __fmul_rn(D.y, 0.03125f)};
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const uint32_t code = (lw[e >> 3] >> (4 * (e & 7))) & 15u;
+                v[e] = __fmul_rn(lds_f32(cent_base + 4 * code), Ds[e >> 4]);
+            }
+            fwht32_regs(v);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0.f;
         }
-        fwht32_regs(v);
-        store_block<DT>(out + ((int64_t)row * ldo + k0) * ElemSize<DT>::value, bits, ps, v);
+        uint32_t o[DeqOut<DT>::kWords];
+        block_words<DT>(bits, ps, v, o);
+#pragma unroll
+        for (int i = 0; i < C; ++i) st[lane * C + (i ^ key)] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        __syncwarp();
+        uint4 *rowp = reinterpret_cast<uint4 *>(out + ((int64_t)row * ldo + seg_col) * ElemSize<DT>::value);
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+            const int c = i * 32 + lane;  // 16-byte chunk of the warp's row segment
+            const int L = c / C;          // the lane (block) it belongs to
+            const uint4 val = st[L * C + ((c % C) ^ stage_key<C>(L))];
+            if (L < nvalid) rowp[c] = val;
+        }
+        __syncwarp();
     }
 }
 
