@@ -256,6 +256,8 @@ class Path:
                                    ws=tq.workspace(1, n, k, device)))
         self.batch = [(it["codes"], it["scales"], it["n"], it["k"], it["x"], it["y"]) for it in self.items]
         self.descs = tq.batch_descs(self.batch)
+        self.deq_batch = [(it["codes"], it["scales"], it["n"], it["k"], it["deq"]) for it in self.items]
+        self.deq_descs = tq.dequant_descs(self.deq_batch)
         self.ws = tq.batch_workspace(self.batch, 1, device)
 
     def quantize(self):
@@ -263,8 +265,8 @@ class Path:
             self.tq.quantize(it["W"], it["codes"], it["scales"])
 
     def dequantize(self):
-        for it in self.items:
-            self.tq.dequantize(it["codes"], it["scales"], it["n"], it["k"], out=it["deq"])
+        """All matrices in one launch."""
+        self.tq.dequantize_batch(self.deq_batch, descs=self.deq_descs)
 
     def gemv(self):
         """All matrices in one batch: one pre-rotation launch for the distinct
@@ -489,7 +491,7 @@ def run_ours(args, world, rank, local):
     path.add_shadow(smats, sacts, device)
     del smats, sacts
     nmat = len(path.items)
-    launches_per_step = 2 * nmat + 2  # quantize + dequantize per matrix; one pre-rotation + one fused product
+    launches_per_step = nmat + 3  # quantize per matrix; one dequantise; one pre-rotation + one fused product
     warmup = max(3, args.warmup)
     steps = max(1, args.steps)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
@@ -559,7 +561,7 @@ def run_ours(args, world, rank, local):
     # algorithmic bytes per phase (one GPU)
     alg = {
         "quantize": (path.in_bytes() + packed, ms_q, nmat),
-        "dequantize": (packed + 2 * weights, ms_d, nmat),
+        "dequantize": (packed + 2 * weights, ms_d, 1),
         "gemv": (packed + path.act_bytes() + path.out_bytes(), ms_g, 2),
     }
     rooflines = {}
@@ -868,8 +870,9 @@ def comparators(tq, path, device, steps, warmup, use_graph, world, hbm):
     """Two ways to run the same batch-1 layer without the fused kernel
     (TQ4_1S page, TQ4_1S 是什么 / 解码速度 sections: the CUDA port converts
     TQ4_1S to q8_0 at load time and runs a plain kernel):
-      * dequant_then_matmul: tq_dequantize every matrix to bf16, then a
-        cuBLAS bf16 GEMV (torch.matmul) on it, every pass;
+      * dequant_then_matmul: tq_dequantize_batch of every matrix to bf16
+        (one launch), then a cuBLAS bf16 GEMV (torch.matmul) per matrix,
+        every pass;
       * dense_bf16_gemv: cuBLAS bf16 GEMV on the unquantised bf16 weights
         (the weights converted once; 3.2 x the bytes of the packed form),
         alternating two copies of the layer (2 x 436 MB > L2).
@@ -879,9 +882,12 @@ def comparators(tq, path, device, steps, warmup, use_graph, world, hbm):
     deq = [torch.empty((it["n"], it["k"]), dtype=torch.bfloat16, device=device) for it in path.items]
     outs = [torch.empty((1, it["n"]), dtype=torch.bfloat16, device=device) for it in path.items]
 
+    dq_items = [(it["codes"], it["scales"], it["n"], it["k"], d) for it, d in zip(path.items, deq)]
+    dq_descs = tq.dequant_descs(dq_items)
+
     def dq_mm():
+        tq.dequantize_batch(dq_items, descs=dq_descs)
         for it, d, o in zip(path.items, deq, outs):
-            tq.dequantize(it["codes"], it["scales"], it["n"], it["k"], out=d)
             torch.matmul(it["x"], d.t(), out=o)
 
     run = capture(dq_mm, use_graph, R)

@@ -39,6 +39,12 @@ class GemmDesc(ctypes.Structure):
                 ("ldy", ctypes.c_int64)]
 
 
+class DequantDesc(ctypes.Structure):
+    """Mirror of ``tq_dequant_desc`` in include/tq.h."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("n", ctypes.c_int64),
+                ("k", ctypes.c_int64), ("w_out", ctypes.c_void_p), ("ldo", ctypes.c_int64)]
+
+
 class Nvfp4GemmDesc(ctypes.Structure):
     """Mirror of ``tq_nvfp4_gemm_desc`` in include/tq.h."""
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
@@ -76,6 +82,7 @@ def load_library() -> ctypes.CDLL:
             "tq_gemm_workspace_bytes": ([I64, I64, I64], SZ),
             "tq_quantize": ([P, I, I64, I64, I64, P, P, P], I),
             "tq_dequantize": ([P, P, I64, I64, P, I, I64, P], I),
+            "tq_dequantize_batch": ([ctypes.POINTER(DequantDesc), I, I, P], I),
             "tq_prerotate": ([P, I, I64, I64, I64, P, P], I),
             "tq_gemm": ([P, P, I64, I64, P, I, I64, I64, P, I, I64, P, SZ, P], I),
             "tq_gemv": ([P, P, I64, I64, P, I, P, I, P, SZ, P], I),
@@ -140,6 +147,10 @@ def tq_quantize(w, wt, n, k, ldw, codes, scales, stream) -> int:
 
 def tq_dequantize(codes, scales, n, k, w_out, ot, ldo, stream) -> int:
     return load_library().tq_dequantize(codes, scales, n, k, w_out, ot, ldo, stream)
+
+
+def tq_dequantize_batch(descs, count, ot, stream) -> int:
+    return load_library().tq_dequantize_batch(descs, count, ot, stream)
 
 
 def tq_prerotate(X, xt, m, k, ldx, xrot, stream) -> int:
@@ -290,6 +301,24 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, n: int, k: int, dtype=
     _check(tq_dequantize(codes.data_ptr(), scales.data_ptr(), n, k, out.data_ptr(), _dt(out.dtype), _ld(out),
                          _stream(stream)), "tq_dequantize")
     return out
+
+
+def dequant_descs(items):
+    """items: sequence of (codes, scales, n, k, out [n, k]) -> ctypes array."""
+    arr = (DequantDesc * len(items))()
+    for i, (codes, scales, n, k, out) in enumerate(items):
+        arr[i] = DequantDesc(codes.data_ptr(), scales.data_ptr(), n, k, out.data_ptr(), _ld(out))
+    return arr
+
+
+def dequantize_batch(items, stream=None, descs=None):
+    """Dequantise every (codes, scales, n, k, out) in one launch (outputs of one dtype)."""
+    dts = {it[4].dtype for it in items}
+    if len(dts) != 1:
+        raise ValueError("dequantize_batch: every output needs the same dtype")
+    if descs is None:
+        descs = dequant_descs(items)
+    _check(tq_dequantize_batch(descs, len(items), _dt(dts.pop()), _stream(stream)), "tq_dequantize_batch")
 
 
 def prerotate(X: torch.Tensor, xrot: torch.Tensor | None = None, stream=None) -> torch.Tensor:

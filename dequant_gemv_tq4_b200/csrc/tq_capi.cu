@@ -195,6 +195,25 @@ tq_status tq_dequantize(const uint8_t *codes, const uint16_t *scales, int64_t n,
     return from_cuda(tq::launch_dequantize(codes, scales, n, k, w_out, ot, ldo, (cudaStream_t)stream));
 }
 
+tq_status tq_dequantize_batch(const tq_dequant_desc *descs, int count, tq_dtype ot, void *stream) {
+    if (!descs) return TQ_ERR_INVALID_ARG;
+    if (count < 1 || count > TQ_MAX_BATCH) return TQ_ERR_SHAPE;
+    if (!valid_dtype(ot)) return TQ_ERR_DTYPE;
+    tq::DequantJob jobs[TQ_MAX_BATCH];
+    int rows = 0;  // descriptors with rows
+    for (int i = 0; i < count; ++i) {
+        const tq_dequant_desc &d = descs[i];
+        tq_status st = check_nk(d.n, d.k);
+        if (st != TQ_OK) return st;
+        if (d.n == 0) continue;
+        if ((st = check_planes(d.codes, d.scales)) != TQ_OK) return st;
+        if ((st = check_matrix_operand(d.w_out, d.ldo, d.k)) != TQ_OK) return st;
+        jobs[rows++] = {d.codes, d.scales, d.n, d.k, d.w_out, d.ldo};
+    }
+    if (rows == 0) return TQ_OK;  // nothing to launch
+    return from_cuda(tq::launch_dequantize_batch(jobs, rows, ot, (cudaStream_t)stream));
+}
+
 tq_status tq_prerotate(const void *X, tq_dtype xt, int64_t m, int64_t k, int64_t ldx, uint16_t *xrot,
                        void *stream) {
     tq_status st = check_nk(m, k);

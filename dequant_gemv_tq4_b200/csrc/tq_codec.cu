@@ -307,11 +307,41 @@ __device__ __forceinline__ int stage_key(int l) {
     return C == 8 ? (l & 7) : ((l >> 1) & 3);
 }
 
+// Work items of a (batched) dequantise launch: (matrix, 1024-column segment,
+// 8-row group), numbered matrix by matrix and, within a matrix, segment by
+// segment; each CTA takes one contiguous range of items, so its lanes'
+// sign patterns change only where the segment does.  Warp w of a CTA
+// writes row 8 * group + w of each item.
+struct DeqProblem {
+    const uint32_t *codes;
+    const uint32_t *scales;
+    char *out;
+    int64_t ldo;
+    int64_t item_begin;
+    int n, nb, nsb, segs, groups;
+};
+struct DeqParams {
+    DeqProblem p[kMaxProblems];
+    int count;
+    int64_t items;
+};
+
+struct DeqItem {
+    int q, seg, group;
+};
+
+__device__ __forceinline__ void next_item(const DeqParams &P, DeqItem &it) {
+    if (++it.group == P.p[it.q].groups) {
+        it.group = 0;
+        if (++it.seg == P.p[it.q].segs) {
+            it.seg = 0;
+            ++it.q;
+        }
+    }
+}
+
 template <int DT>
-__global__ void __launch_bounds__(kCodecThreads, DT == kF32 ? 2 : 3) dequantize_kernel(const uint32_t *__restrict__ codes,
-                                                                     const uint32_t *__restrict__ scales, int n,
-                                                                     int nb, int nsb, char *__restrict__ out,
-                                                                     int64_t ldo) {
+__global__ void __launch_bounds__(kCodecThreads, DT == kF32 ? 2 : 3) dequantize_kernel(const __grid_constant__ DeqParams P) {
     constexpr int C = DeqOut<DT>::kChunks;
     __shared__ float cent[16];  // signed centroids c(code)
     __shared__ __align__(16) uint4 stage[kCodecWarps * 32 * C];
@@ -321,42 +351,52 @@ __global__ void __launch_bounds__(kCodecThreads, DT == kF32 ? 2 : 3) dequantize_
     }
     __syncthreads();
     const uint32_t cent_base = (uint32_t)__cvta_generic_to_shared(cent);
-
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int blk = blockIdx.x * 32 + lane;
-    const bool valid = blk < nb;
-    const int nvalid = min(32, nb - (int)blockIdx.x * 32);  // blocks of this column segment
-    const int sb = blk >> 2, j = blk & 3;
-    const uint32_t k0 = (uint32_t)blk * kBlock;
-    const uint32_t bits = block_sign_bits(k0);
-    uint32_t ps[16];
-    packed_sign_words(bits, ps);
     uint4 *st = stage + warp * 32 * C;
     const int key = stage_key<C>(lane);
-    const int64_t seg_col = (int64_t)blockIdx.x * 32 * kBlock;
 
-    const int rstep = gridDim.y * kCodecWarps;
-    int row = blockIdx.y * kCodecWarps + warp;
-    uint32_t nsw[4] = {0u, 0u, 0u, 0u}, nsc = 0u;  // codes and scales of the next row
-    if (valid && row < n) {
-        const size_t slot = unit_row(row, sb, nsb);
-#pragma unroll
-        for (int tt = 0; tt < 4; ++tt) nsw[tt] = __ldg(codes + slot * 16 + 4 * tt + j);
-        nsc = __ldg(scales + slot * 4 + j);
+    const int64_t i0 = P.items * blockIdx.x / gridDim.x, i1 = P.items * (blockIdx.x + 1) / gridDim.x;
+    if (i0 >= i1) return;
+    DeqItem cur;
+    cur.q = 0;
+    while (cur.q + 1 < P.count && i0 >= P.p[cur.q + 1].item_begin) ++cur.q;
+    {
+        const int64_t local = i0 - P.p[cur.q].item_begin;
+        cur.seg = (int)(local / P.p[cur.q].groups);
+        cur.group = (int)(local % P.p[cur.q].groups);
     }
-    for (; row < n; row += rstep) {
+    // codes and scales of this warp's row of an item (nothing past the matrix)
+    auto load_row = [&](const DeqItem &it, uint32_t (&w)[4], uint32_t &sc) {
+        const DeqProblem &pr = P.p[it.q];
+        const int row = it.group * kCodecWarps + warp, blk = it.seg * 32 + lane;
+        if (row < pr.n && blk < pr.nb) {
+            const size_t slot = unit_row(row, blk >> 2, pr.nsb);
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) w[tt] = __ldg(pr.codes + slot * 16 + 4 * tt + (blk & 3));
+            sc = __ldg(pr.scales + slot * 4 + (blk & 3));
+        }
+    };
+    int seg_bits = -1;  // segment whose sign pattern `bits` / `ps` hold
+    uint32_t bits = 0, ps[16];
+    uint32_t nsw[4] = {0u, 0u, 0u, 0u}, nsc = 0u;  // the next item's row, loaded one step ahead
+    load_row(cur, nsw, nsc);
+    for (int64_t i = i0; i < i1; ++i) {
+        const DeqProblem &pr = P.p[cur.q];
+        const int row = cur.group * kCodecWarps + warp, blk = cur.seg * 32 + lane;
+        if (cur.seg != seg_bits) {
+            seg_bits = cur.seg;
+            bits = block_sign_bits((uint32_t)blk * kBlock);
+            packed_sign_words(bits, ps);
+        }
+        uint32_t sw[4], sc = nsc;
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) sw[tt] = nsw[tt];
+        DeqItem nx = cur;
+        next_item(P, nx);
+        if (i + 1 < i1) load_row(nx, nsw, nsc);
         float v[32];
-        if (valid) {
-            uint32_t sw[4], lw[4];
-#pragma unroll
-            for (int tt = 0; tt < 4; ++tt) sw[tt] = nsw[tt];
-            const uint32_t sc = nsc;
-            if (row + rstep < n) {
-                const size_t slot = unit_row(row + rstep, sb, nsb);
-#pragma unroll
-                for (int tt = 0; tt < 4; ++tt) nsw[tt] = __ldg(codes + slot * 16 + 4 * tt + j);
-                nsc = __ldg(scales + slot * 4 + j);
-            }
+        if (row < pr.n && blk < pr.nb) {
+            uint32_t lw[4];
             transpose_bytes(sw, lw);  // the transpose is its own inverse
             const float2 D = __half22float2(*reinterpret_cast<const __half2 *>(&sc));
             const float Ds[2] = {__fmul_rn(D.x, 0.03125f), __fmul_rn(D.y, 0.03125f)};
@@ -373,17 +413,22 @@ __global__ void __launch_bounds__(kCodecThreads, DT == kF32 ? 2 : 3) dequantize_
         uint32_t o[DeqOut<DT>::kWords];
         block_words<DT>(bits, ps, v, o);
 #pragma unroll
-        for (int i = 0; i < C; ++i) st[lane * C + (i ^ key)] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        for (int c = 0; c < C; ++c) st[lane * C + (c ^ key)] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
         __syncwarp();
-        uint4 *rowp = reinterpret_cast<uint4 *>(out + ((int64_t)row * ldo + seg_col) * ElemSize<DT>::value);
+        if (row < pr.n) {
+            const int nvalid = min(32, pr.nb - cur.seg * 32);  // blocks of this segment
+            uint4 *rowp = reinterpret_cast<uint4 *>(pr.out + ((int64_t)row * pr.ldo + (int64_t)cur.seg * 32 * kBlock) *
+                                                                 ElemSize<DT>::value);
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            const int c = i * 32 + lane;  // 16-byte chunk of the warp's row segment
-            const int L = c / C;          // the lane (block) it belongs to
-            const uint4 val = st[L * C + ((c % C) ^ stage_key<C>(L))];
-            if (L < nvalid) rowp[c] = val;
+            for (int c0 = 0; c0 < C; ++c0) {
+                const int c = c0 * 32 + lane;  // 16-byte chunk of the warp's row segment
+                const int L = c / C;           // the lane (block) it belongs to
+                const uint4 val = st[L * C + ((c % C) ^ stage_key<C>(L))];
+                if (L < nvalid) rowp[c] = val;
+            }
         }
         __syncwarp();
+        cur = nx;
     }
 }
 
@@ -504,26 +549,49 @@ cudaError_t launch_quantize(const void *w, int dtype, int64_t n, int64_t k, int6
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, void *w_out,
-                              int dtype, int64_t ldo, cudaStream_t stream) {
+cudaError_t launch_dequantize_batch(const DequantJob *jobs, int count, int dtype, cudaStream_t stream) {
+    if (count < 1 || count > kMaxProblems) return cudaErrorInvalidValue;
     DeviceInfo di;
     cudaError_t err = device_info(&di);
     if (err != cudaSuccess) return err;
-    const int64_t nb = k / 32, nsb = superblocks(k);
-    const int64_t segs = (nb + 31) / 32;
+    DeqParams prm = {};
+    int64_t items = 0;
+    int used = 0;  // matrices with rows (an empty one has no items to walk)
+    for (int i = 0; i < count; ++i) {
+        if (jobs[i].n <= 0) continue;
+        DeqProblem &d = prm.p[used++];
+        d.codes = reinterpret_cast<const uint32_t *>(jobs[i].codes);
+        d.scales = reinterpret_cast<const uint32_t *>(jobs[i].scales);
+        d.out = static_cast<char *>(jobs[i].out);
+        d.ldo = jobs[i].ldo;
+        d.item_begin = items;
+        d.n = (int)jobs[i].n;
+        d.nb = (int)(jobs[i].k / 32);
+        d.nsb = (int)superblocks(jobs[i].k);
+        d.segs = (d.nb + 31) / 32;
+        d.groups = (int)((jobs[i].n + kCodecWarps - 1) / kCodecWarps);
+        items += (int64_t)d.segs * d.groups;
+    }
+    prm.count = used;
+    prm.items = items;
+    if (items == 0) return cudaSuccess;
     const int per_sm = dtype == kF32 ? dequantize_per_sm<kF32>() : dtype == kBF16 ? dequantize_per_sm<kBF16>()
                                                                                    : dequantize_per_sm<kF16>();
-    dim3 grid((unsigned)segs, (unsigned)rows_grid(n, segs, di.sm_count, per_sm));
-    auto *c = reinterpret_cast<const uint32_t *>(codes);
-    auto *s = reinterpret_cast<const uint32_t *>(scales);
-    char *o = static_cast<char *>(w_out);
+    int64_t grid = (int64_t)di.sm_count * per_sm;  // one wave, persistent
+    if (grid > items) grid = items;
     switch (dtype) {
-        case kF32: dequantize_kernel<kF32><<<grid, kCodecThreads, 0, stream>>>(c, s, (int)n, (int)nb, (int)nsb, o, ldo); break;
-        case kBF16: dequantize_kernel<kBF16><<<grid, kCodecThreads, 0, stream>>>(c, s, (int)n, (int)nb, (int)nsb, o, ldo); break;
-        case kF16: dequantize_kernel<kF16><<<grid, kCodecThreads, 0, stream>>>(c, s, (int)n, (int)nb, (int)nsb, o, ldo); break;
+        case kF32: dequantize_kernel<kF32><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
+        case kBF16: dequantize_kernel<kBF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
+        case kF16: dequantize_kernel<kF16><<<(unsigned)grid, kCodecThreads, 0, stream>>>(prm); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, void *w_out,
+                              int dtype, int64_t ldo, cudaStream_t stream) {
+    const DequantJob job = {codes, scales, n, k, w_out, ldo};
+    return launch_dequantize_batch(&job, 1, dtype, stream);
 }
 
 namespace {

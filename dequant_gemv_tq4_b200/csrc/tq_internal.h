@@ -29,6 +29,17 @@ cudaError_t launch_quantize(const void *w, int dtype, int64_t n, int64_t k, int6
 cudaError_t launch_dequantize(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, void *w_out,
                               int dtype, int64_t ldo, cudaStream_t stream);
 
+// Several matrices dequantised by one launch (all outputs of one dtype).
+struct DequantJob {
+    const uint8_t *codes;
+    const uint16_t *scales;
+    int64_t n;
+    int64_t k;
+    void *out;
+    int64_t ldo;
+};
+cudaError_t launch_dequantize_batch(const DequantJob *jobs, int count, int dtype, cudaStream_t stream);
+
 // ---- pre-rotation ----------------------------------------------------------
 struct RotInput {  // device-side description of one activation matrix
     const char *x;

@@ -121,6 +121,23 @@ TQ_API tq_status tq_dequantize(const uint8_t *codes, const uint16_t *scales, int
                         tq_dtype ot, int64_t ldo, void *stream);
 
 /*
+ * tq_dequantize_batch -- tq_dequantize of count (1..TQ_MAX_BATCH) matrices in
+ * one launch, every output of dtype ot (e.g. all seven matrices of a layer;
+ * one launch has one ramp and one tail instead of seven).  The same argument
+ * rules as tq_dequantize per descriptor; descriptors with n == 0 are skipped.
+ * Outputs must not overlap one another or any codes/scales.
+ */
+typedef struct {
+    const uint8_t *codes;   /* device, packed planes of an n x k matrix (tq_quantize) */
+    const uint16_t *scales;
+    int64_t n;              /* >= 0 */
+    int64_t k;              /* positive multiple of 32 */
+    void *w_out;            /* device, n x k of dtype ot, row stride ldo (ldo >= k, ldo % 8 == 0, 16-byte aligned) */
+    int64_t ldo;
+} tq_dequant_desc;
+TQ_API tq_status tq_dequantize_batch(const tq_dequant_desc *descs, int count, tq_dtype ot, void *stream);
+
+/*
  * Pre-rotated activations (TQ page, 解码速度 section: the activation is
  * rotated once and shared, so the per-weight work is lookup x scale).
  * xrot holds fp16 values H(s .* x)/32 per 32-block, in the order the fused

@@ -96,6 +96,25 @@ def test_dequantize_and_prerotate_argument_errors(lib):
     assert d(FAKE, FAKE, 4, 64, None, 0, 64, None) == INVALID
     assert d(FAKE, FAKE, 4, 64, FAKE + 8, 0, 64, None) == ALIGN
     assert d(FAKE, FAKE, 0, 64, FAKE, 0, 64, None) == OK
+    from dequant_gemv_tq4_b200 import DequantDesc
+    b = lib.tq_dequantize_batch
+
+    def descs(*rows):
+        arr = (DequantDesc * len(rows))()
+        for i, r in enumerate(rows):
+            arr[i] = DequantDesc(*r)
+        return arr
+
+    good = (FAKE, FAKE, 4, 64, FAKE, 64)
+    assert b(None, 1, 0, None) == INVALID
+    assert b(descs(good), 0, 0, None) == SHAPE
+    assert b(descs(*[good] * 9), 9, 0, None) == SHAPE
+    assert b(descs(good), 1, 5, None) == DTYPE
+    assert b(descs(good, (FAKE, FAKE, 4, 40, FAKE, 64)), 2, 0, None) == SHAPE
+    assert b(descs(good, (None, FAKE, 4, 64, FAKE, 64)), 2, 0, None) == INVALID
+    assert b(descs(good, (FAKE, FAKE, 4, 64, FAKE + 8, 64)), 2, 0, None) == ALIGN
+    assert b(descs(good, (FAKE, FAKE, 4, 64, FAKE, 60)), 2, 0, None) == INVALID  # ldo < k
+    assert b(descs((FAKE, FAKE, 0, 64, FAKE, 64), (None, None, 0, 96, None, 0)), 2, 0, None) == OK  # no rows
     p = lib.tq_prerotate
     assert p(FAKE, 0, 1, 33, 40, FAKE, None) == SHAPE
     assert p(FAKE, 3, 1, 64, 64, FAKE, None) == DTYPE

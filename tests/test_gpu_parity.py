@@ -140,6 +140,52 @@ def test_dequantize_strided_output(cuda_lib):
     assert np.all(np.abs(o[:, :k] - w64) <= _dequant_bound(c_ref, s_ref, n, k, w64, F32))
 
 
+@pytest.mark.parametrize("out_dtype", [BF16, F32, F16])
+def test_dequantize_batch_matches_single_launches(cuda_lib, out_dtype):
+    """tq_dequantize_batch (one launch over several matrices, work items
+    spread over persistent CTAs) writes exactly what one tq_dequantize per
+    matrix writes: ragged k, rows not a multiple of 8 or 16, an empty matrix,
+    strided outputs whose padding columns stay untouched."""
+    shapes = [(64, 1056), (17, 96), (0, 128), (300, 4160), (33, 160), (1000, 1024), (9, 32)]
+    items, expect = [], []
+    for i, (n, k) in enumerate(shapes):
+        W = _w(max(n, 1), k, BF16, seed=120 + i)[:n]
+        codes, scales = cuda_lib.quantize(W.to(DEV).contiguous())
+        ld = k + (8 if i % 2 else 0)
+        out = torch.full((n, ld), 7.0, dtype=out_dtype, device=DEV)
+        items.append((codes, scales, n, k, out[:, :k]))
+        expect.append(cuda_lib.dequantize(codes, scales, n, k, dtype=out_dtype) if n else None)
+    cuda_lib.dequantize_batch(items)
+    torch.cuda.synchronize()
+    for (codes, scales, n, k, o), ref in zip(items, expect):
+        if n == 0:
+            continue
+        assert torch.equal(o, ref), (n, k)
+        full = o.as_strided((n, o.stride(0)), (o.stride(0), 1))
+        assert bool((full[:, k:] == 7.0).all()), (n, k)
+
+
+def test_dequantize_batch_layer_against_oracle(cuda_lib):
+    """Eight matrices (the batch limit) in one launch; sampled rows checked
+    against the oracle within the arithmetic bound."""
+    shapes = [(256, 1024), (64, 1024), (64, 1024), (256, 1024), (512, 1024), (512, 1024), (256, 3584), (40, 2080)]
+    items, packed = [], []
+    for i, (n, k) in enumerate(shapes):
+        W = _w(n, k, BF16, seed=140 + i)
+        c_ref, s_ref = _oracle_quantize(W)
+        codes = torch.tensor(c_ref, device=DEV)
+        scales = torch.tensor(s_ref.view(np.int16), device=DEV)
+        items.append((codes, scales, n, k, torch.empty((n, k), dtype=F32, device=DEV)))
+        packed.append((c_ref, s_ref))
+    cuda_lib.dequantize_batch(items)
+    torch.cuda.synchronize()
+    for (codes, scales, n, k, o), (c_ref, s_ref) in zip(items, packed):
+        w64 = oracle.dequantize(c_ref, s_ref, n, k)
+        got = o.cpu().numpy().astype(np.float64)
+        bound = _dequant_bound(c_ref, s_ref, n, k, w64, F32)
+        assert np.all(np.abs(got - w64) <= bound), (n, k)
+
+
 @pytest.mark.parametrize("m,k", [(1, 32), (1, 4096), (3, 96), (5, 160)])
 def test_prerotate_values_and_layout(cuda_lib, m, k):
     X = _w(m, k, BF16, seed=7, std=1.0)
