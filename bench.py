@@ -113,7 +113,7 @@ LANES_PER_SM = 128  # fp32 / integer lanes of one SM (4 partitions x 32)
 
 PROFILE_FILES = {  # phase -> committed ncu summary and the sources its kernel is built from
     "quantize": ("quantize_kernel_llama3_8b_down.md", ("tq_device.cuh", "tq_codec.cu")),
-    "dequantize": ("dequantize_kernel_llama3_8b_down.md", ("tq_device.cuh", "tq_codec.cu")),
+    "dequantize": ("dequantize_kernel_llama3_8b_layer.md", ("tq_device.cuh", "tq_codec.cu")),
     "gemv": ("gemv_group_kernel_llama3_8b_layer.md", ("tq_device.cuh", "tq_gemv.cu")),
 }
 
