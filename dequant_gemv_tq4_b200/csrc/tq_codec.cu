@@ -454,23 +454,29 @@ __global__ void __launch_bounds__(kCodecThreads) prerotate_kernel(const __grid_c
     // written by a quantise launch that completed before this kernel could
     // start), so its CTAs can take the SMs that the previous product frees
     // in its tail.  Then wait until every earlier kernel has completed.
-    grid_dependents_launch();
-    grid_dependency_wait();
-    if (prm.header && blockIdx.x == 0 && threadIdx.x == 0) {
-        prm.header[kHeaderStatus] = 0u;
-        prm.header[kHeaderTag] += 1u;  // the previous call (and its product) has completed
-    }
-
+    //
+    // The activation lines this lane will read are prefetched into L2 before
+    // the wait (L2 is where writes meet, so a line a still-running kernel
+    // rewrites is current there when the load after the wait reads it): the
+    // loads then do not queue behind the product's weight prefetch in DRAM.
     const int lane = threadIdx.x & 31;
     const int j = lane >> 3, p = lane & 7;
     const int64_t unit = (int64_t)blockIdx.x * kCodecWarps + (threadIdx.x >> 5);
-    if (unit >= prm.units) return;
     int q = 0;
     while (q + 1 < prm.count && unit >= prm.in[q + 1].unit_begin) ++q;
     const RotInput &in = prm.in[q];
     const int64_t local = unit - in.unit_begin;
     const int row = (int)(local / in.nsb), sb = (int)(local % in.nsb);
     const uint32_t col0 = (uint32_t)sb * kSbElems + 32u * j + 4u * p;
+    if (unit < prm.units && sb * kSbBlocks + j < in.nb && row < prm.m)
+        prefetch_l2(in.x + ((int64_t)row * in.ldx + col0) * ElemSize<DT>::value);
+    grid_dependents_launch();
+    grid_dependency_wait();
+    if (prm.header && blockIdx.x == 0 && threadIdx.x == 0) {
+        prm.header[kHeaderStatus] = 0u;
+        prm.header[kHeaderTag] += 1u;  // the previous call (and its product) has completed
+    }
+    if (unit >= prm.units) return;
     __half2 lo, hi;
     rotate_unit_lane<DT, ROTATE>(in.x, in.ldx, in.nb, prm.m, row, sb, lane, lo, hi);
     if constexpr (LAYOUT == kRotFragment) {

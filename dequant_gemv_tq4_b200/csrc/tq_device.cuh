@@ -234,6 +234,10 @@ __device__ __forceinline__ void decode_word(uint32_t w, uint32_t (&o)[4]) {
     o[3] = prmt(lo47, hi47, 0x7362u);  // elements 6, 7
 }
 
+// L2 prefetch hint for the line holding p (no data returned, no fault on a
+// valid address).
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // Programmatic dependent launch: wait for the preceding grid's results / let
 // the next grid start its prologue.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -902,8 +902,10 @@ __global__ void __launch_bounds__(warps_for(CM > 0, NT) * 32, 1) gemv_group_kern
     const int u1 = active ? (int)div_floor((int64_t)(gw + 1) * U, W, P.inv_warps) : 0;
 
     // ---- prologue: barriers, first bulk copies, lookup table -------------
-    // (the packed weights never depend on the preceding grid, so the copies
-    // start before the programmatic-dependency wait)
+    // (the packed weights never depend on the preceding grid, so the first
+    // stage's copies start before the programmatic-dependency wait; the
+    // other stages follow it: a smaller burst ahead of the wait lets the
+    // pre-rotation's activation loads, which run meanwhile, come back sooner)
     Cursor cu = {nullptr, nullptr, 0, 0, 0};
     int pv = u0;  // next unit to copy
     if (active) {
@@ -913,10 +915,10 @@ __global__ void __launch_bounds__(warps_for(CM > 0, NT) * 32, 1) gemv_group_kern
         }
         __syncwarp();
         cu = cursor_at<SB>(P, u0);
-        for (int i = 0; i < kStages && pv < u1; ++i) {
+        if (pv < u1) {
             const int cnt = min(kPerStage, u1 - pv);
-            const bool skip = P.inject_skip && gw == 0 && i == 0;
-            issue_stage<SB, kStageScaleOff>(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0 && !skip);
+            const bool skip = P.inject_skip && gw == 0;
+            issue_stage<SB, kStageScaleOff>(P, cu, cnt, ring, bars, lane == 0 && !skip);
             pv += cnt;
         }
     }
@@ -936,6 +938,11 @@ __global__ void __launch_bounds__(warps_for(CM > 0, NT) * 32, 1) gemv_group_kern
     // wait (it waits for this grid's completion before writing anything)
     grid_dependents_launch();
     if (!active) return;
+    for (int i = 1; i < kStages && pv < u1; ++i) {  // the ring's other stages
+        const int cnt = min(kPerStage, u1 - pv);
+        issue_stage<SB, kStageScaleOff>(P, cu, cnt, ring + i * kStageBytes, bars + 8 * i, lane == 0);
+        pv += cnt;
+    }
     // this call's tag (advanced by the launch that prepared the header)
     const uint32_t tag = *reinterpret_cast<volatile const unsigned *>(P.header + kHeaderTag);
 
