@@ -25,11 +25,13 @@
 //  * The weight tile (256 rows x 64 columns per stage) is decoded by sixteen
 //    warps, one row and one 32-column block per thread: each thread reads its
 //    row's 64-byte superblock slot with 16-byte loads (neighbouring threads,
-//    neighbouring slots), three superblocks ahead in registers; a 4x4 byte
-//    transpose restores element order; byte permutes against register tables
-//    of the fp16 magnitudes, with the sign bits merged in by two more
-//    permutes, give fp16 centroid pairs; one fp16 multiply applies the
-//    half-block scale and 16-byte stores write the swizzled rows.  A proxy
+//    neighbouring slots), three superblocks ahead in registers; byte
+//    permutes against register tables of the fp16 magnitudes, with the sign
+//    bits merged in by two more permutes, turn each stored word into four
+//    fp16 centroid pairs (each byte holds two neighbouring elements, so the
+//    stored byte order needs no transpose, only a choice of output chunk);
+//    one fp16 multiply applies the half-block scale and 16-byte stores write
+//    the swizzled rows.  A proxy
 //    fence then publishes them to the tensor cores.  Three stages.
 //  * One thread issues the MMAs; tcgen05.commit releases each stage to its
 //    producers and finally signals the epilogue.  The sixteen decode warps
@@ -257,24 +259,28 @@ __device__ __forceinline__ BlockWords block_of(const RowSlot &r, int j) {
 }
 
 // Decode one row's 32-column block jj of the stage into the swizzled weight
-// tile.  In a row's 64-byte superblock slot, logical byte L of block j sits at
-// chunk L % 4, word j, byte L / 4; so the block's four chunk words, byte-
-// transposed, give logical words i = 0..3, each holding elements 8i .. 8i+7.
-// The half-block scale multiplies in fp16.  Logical word i lands in 16-byte
-// chunk 4 jj + i of the tile row, stored at chunk (4 jj + i) xor (row % 8)
+// tile.  In a row's 64-byte superblock slot, logical byte L of block j
+// (elements 2L, 2L + 1) sits at chunk L % 4, word j, byte L / 4; so byte k of
+// chunk word b holds elements 8k + 2b, 8k + 2b + 1, and each chunk word is
+// decoded as it stands into fp16 pairs, k = 0..3.  The half-block scale
+// multiplies in fp16.  Elements 8k .. 8k + 7 (pairs b = 0..3) form 16-byte
+// chunk 4 jj + k of the tile row, stored at chunk (4 jj + k) xor (row % 8)
 // (the 128-byte swizzle).
 __device__ __forceinline__ void decode_block(const BlockWords &w, int row, int jj, uint32_t atile) {
     const uint32_t rbase = atile + (uint32_t)row * 128u;
-    uint32_t L[4];
-    transpose4(w.c, L);
     const uint32_t d0 = prmt(w.s, w.s, 0x1010u), d1 = prmt(w.s, w.s, 0x3232u);  // (d, d) of each half
+    uint32_t o[4][4];  // o[k][b]: elements 8k + 2b, 8k + 2b + 1
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t d = i < 2 ? d0 : d1;  // elements 0..15 take d0, 16..31 d1
+    for (int b = 0; b < 4; ++b) {
         uint32_t v[4];
-        decode_word(L[i], v);
-        const uint32_t chunk = (uint32_t)(4 * jj + i) ^ (uint32_t)(row & 7);
-        p_sts128(rbase + chunk * 16u, p_hmul2(v[0], d), p_hmul2(v[1], d), p_hmul2(v[2], d), p_hmul2(v[3], d));
+        decode_word(w.c[b], v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[k][b] = p_hmul2(v[k], k < 2 ? d0 : d1);  // elements 0..15: d0, 16..31: d1
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t chunk = (uint32_t)(4 * jj + k) ^ (uint32_t)(row & 7);
+        p_sts128(rbase + chunk * 16u, o[k][0], o[k][1], o[k][2], o[k][3]);
     }
 }
 

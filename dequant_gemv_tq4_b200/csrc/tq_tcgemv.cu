@@ -333,26 +333,24 @@ __device__ __forceinline__ TcSeg tc_seg_at(const TcParams &P, int u, int u1) {
 }
 
 // Decoded operands of one row's 32-column block j (the row's 64-byte
-// superblock slot in four 16-byte chunks c[0..3]; chunk b, word j holds byte
-// b of the block's logical words): a byte transpose gives logical words i =
-// 0..3 (elements 8i .. 8i+7), register byte tables give their fp16 centroid
-// pairs, and the half-block scale multiplies them (elements 0..15: d0,
-// 16..31: d1).  o[4i + e] = elements 8i + 2e, 8i + 2e + 1: tensor-memory
-// column 16 j + 4 i + e.
+// superblock slot in four 16-byte chunks c[0..3]; chunk b, word j holds
+// logical bytes b, b + 4, b + 8, b + 12 of the block, logical byte L holding
+// elements 2L and 2L + 1).  Each chunk word is decoded as it stands: register
+// byte tables give the fp16 centroid pairs of its four bytes, k = 0..3 being
+// elements 8k + 2b, 8k + 2b + 1, and the half-block scale multiplies them
+// (elements 0..15: d0, 16..31: d1).  o[4k + b] = elements 8k + 2b, 8k + 2b +
+// 1: tensor-memory column 16 j + 4 k + b.
 __device__ __forceinline__ void tc_decode_block(const uint4 (&c)[4], uint32_t sw, uint32_t (&o)[16], int j) {
-    const uint32_t w[4] = {j == 0 ? c[0].x : j == 1 ? c[0].y : j == 2 ? c[0].z : c[0].w,
-                           j == 0 ? c[1].x : j == 1 ? c[1].y : j == 2 ? c[1].z : c[1].w,
-                           j == 0 ? c[2].x : j == 1 ? c[2].y : j == 2 ? c[2].z : c[2].w,
-                           j == 0 ? c[3].x : j == 1 ? c[3].y : j == 2 ? c[3].z : c[3].w};
-    uint32_t L[4];
-    transpose4(w, L);
     const uint32_t d0 = prmt(sw, sw, 0x1010u), d1 = prmt(sw, sw, 0x3232u);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int b = 0; b < 4; ++b) {
+        const uint32_t w = j == 0 ? c[b].x : j == 1 ? c[b].y : j == 2 ? c[b].z : c[b].w;
         uint32_t v[4];
-        decode_word(L[i], v);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[4 * i + e] = tc_hmul2(v[e], i < 2 ? d0 : d1);
+        decode_word(w, v);
+        o[b] = tc_hmul2(v[0], d0);
+        o[4 + b] = tc_hmul2(v[1], d0);
+        o[8 + b] = tc_hmul2(v[2], d1);
+        o[12 + b] = tc_hmul2(v[3], d1);
     }
 }
 
