@@ -173,17 +173,6 @@ __device__ __forceinline__ void load_block<kF16>(const char *p, uint32_t, const 
     }
 }
 
-// Logical words W0..W3 (bytes 0-3, 4-7, 8-11, 12-15 of a block) <-> stored
-// words T0..T3 (T_t = logical bytes t, t+4, t+8, t+12): a 4x4 byte transpose.
-__device__ __forceinline__ void transpose_bytes(const uint32_t (&w)[4], uint32_t (&o)[4]) {
-    const uint32_t a = prmt(w[0], w[1], 0x5140u), b = prmt(w[2], w[3], 0x5140u);
-    const uint32_t c = prmt(w[0], w[1], 0x7362u), d = prmt(w[2], w[3], 0x7362u);
-    o[0] = prmt(a, b, 0x5410u);
-    o[1] = prmt(a, b, 0x7632u);
-    o[2] = prmt(c, d, 0x5410u);
-    o[3] = prmt(c, d, 0x7632u);
-}
-
 // -------------------------------------------------------------------------
 // Quantise.  grid.x = 1024-column segment (32 blocks, one per lane),
 // grid.y * 8 warps stride the rows (padded to a multiple of 16).
@@ -244,7 +233,7 @@ __global__ void __launch_bounds__(kCodecThreads) quantize_kernel(const char *__r
         }
         if (exists) {
             uint32_t sw[4];
-            transpose_bytes(lw, sw);
+            transpose4(lw, sw);
             const size_t slot = unit_row(row, sb, nsb);
 #pragma unroll
             for (int tt = 0; tt < 4; ++tt) codes[slot * 16 + 4 * tt + j] = sw[tt];
@@ -397,7 +386,7 @@ __global__ void __launch_bounds__(kCodecThreads, DT == kF32 ? 2 : 3) dequantize_
         float v[32];
         if (row < pr.n && blk < pr.nb) {
             uint32_t lw[4];
-            transpose_bytes(sw, lw);  // the transpose is its own inverse
+            transpose4(sw, lw);  // the transpose is its own inverse
             const float2 D = __half22float2(*reinterpret_cast<const __half2 *>(&sc));
             const float Ds[2] = {__fmul_rn(D.x, 0.03125f), __fmul_rn(D.y, 0.03125f)};
 #pragma unroll

@@ -29,8 +29,6 @@ constexpr unsigned kFull = 0xffffffffu;
 // Element dtypes, same numbering as tq_dtype in tq.h.
 enum Dtype : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 
-__device__ __forceinline__ uint32_t f32_bits(float v) { return __float_as_uint(v); }
-
 // Sign pattern of global column k: golden-ratio multiplicative hash followed by
 // one MurmurHash3-style mixing round; -1 where bit 31 is set.  Returned as the
 // mask to XOR into an fp32 bit pattern (0x80000000 = negate, 0 = keep).
@@ -140,15 +138,6 @@ struct ElemSize {
 // PTX wrappers
 // ---------------------------------------------------------------------------
 
-// Streaming 128-bit global load: read-only, not kept in L1.
-__device__ __forceinline__ uint4 ldg_stream(const void *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 // 128-bit global load that may stay in L1 (small, reused operands).
 __device__ __forceinline__ uint4 ldg_keep(const void *p) {
     uint4 r;
@@ -169,27 +158,13 @@ __device__ __forceinline__ float lds_f32(uint32_t saddr) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
-    return v;
-}
-
-// D = A(16x16 f16, row) * B(16x8 f16, col) with a zero accumulator; fp32 out.
-__device__ __forceinline__ void mma_16816_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
-}
-
 // ---------------------------------------------------------------------------
 // Register-table decode of TQ4_1S codes (no shared-memory table): the eight
 // fp16 Lloyd-Max magnitudes as byte tables for PRMT.
 // ---------------------------------------------------------------------------
-// 4x4 byte transpose: out[i] byte b = in[b] byte i.
+// 4x4 byte transpose: out[i] byte b = in[b] byte i (its own inverse).  Logical
+// code words W0..W3 (bytes 0-3, 4-7, 8-11, 12-15 of a block) <-> stored words
+// T0..T3 (T_t = logical bytes t, t+4, t+8, t+12).
 __device__ __forceinline__ void transpose4(const uint32_t (&w)[4], uint32_t (&o)[4]) {
     const uint32_t a = prmt(w[0], w[1], 0x5140u), b = prmt(w[2], w[3], 0x5140u);
     const uint32_t c = prmt(w[0], w[1], 0x7362u), d = prmt(w[2], w[3], 0x7362u);

@@ -63,16 +63,6 @@ __device__ __forceinline__ uint32_t unsign_zero_nibbles(uint32_t w) {
     return mag | (w & (nz << 3));
 }
 
-// 4x4 byte transpose between logical code words and stored words (self-inverse).
-__device__ __forceinline__ void transpose4(const uint32_t (&w)[4], uint32_t (&o)[4]) {
-    const uint32_t a = prmt(w[0], w[1], 0x5140u), b = prmt(w[2], w[3], 0x5140u);
-    const uint32_t c = prmt(w[0], w[1], 0x7362u), d = prmt(w[2], w[3], 0x7362u);
-    o[0] = prmt(a, b, 0x5410u);
-    o[1] = prmt(a, b, 0x7632u);
-    o[2] = prmt(c, d, 0x5410u);
-    o[3] = prmt(c, d, 0x7632u);
-}
-
 template <int DT>
 __device__ __forceinline__ void load32(const char *p, float (&v)[32]) {
 #pragma unroll
