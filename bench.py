@@ -398,6 +398,18 @@ def max_over_ranks(values, world):
     return t.tolist()
 
 
+def timed_launches(nmat: int, steps: int, passes: int, gemv_passes: int) -> dict:
+    """Kernel launches of this library inside the timed regions of the main
+    line, per phase: the step loop (a quantise launch per matrix, one batched
+    dequantise, one pre-rotation and one fused product), the quantise and
+    dequantise phases, the GEMV phase (pre-rotation and product per pass) and
+    the per-matrix GEMV timings (one tq_gemv each: pre-rotation and product)."""
+    per = {"step": (nmat + 3) * steps * passes, "quantize": nmat * steps * passes, "dequantize": steps * passes,
+           "gemv": 2 * steps * gemv_passes, "gemv_single_matrix": 2 * steps * nmat}
+    per["total"] = sum(per.values())
+    return per
+
+
 def job_gbs(bytes_per_rank: int, world: int, ms: float) -> float:
     """Whole-job throughput: the bytes all ranks processed / the slowest rank's time."""
     return world * bytes_per_rank / (ms * 1e-3) / 1e9
@@ -493,7 +505,6 @@ def run_ours(args, world, rank, local):
     path.add_shadow(smats, sacts, device)
     del smats, sacts
     nmat = len(path.items)
-    launches_per_step = nmat + 3  # quantize per matrix; one dequantise; one pre-rotation + one fused product
     warmup = max(3, args.warmup)
     steps = max(1, args.steps)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > 126 MB L2
@@ -624,7 +635,8 @@ def run_ours(args, world, rank, local):
                                                   {"peak_note": f"{hbm_kind} HBM copy bandwidth"})),
         "rooflines": rooflines,
         "clocks": clocks,
-        "gpu_launches": launches_per_step * steps * R,
+        "gpu_launches": timed_launches(nmat, steps, R, RG)["total"],
+        "gpu_launches_by_phase": timed_launches(nmat, steps, R, RG),
         "timing": {"passes_per_replay": R, "gemv_passes_per_replay": RG, "replays": steps,
                    "gemv": f"{RG} passes per graph replay (one token through the 32 decoder layers of Llama-3-8B), "
                            "alternating between the layer and an independent shadow layer (2 x packed bytes > L2)",

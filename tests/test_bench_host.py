@@ -1,6 +1,7 @@
 """Host-side logic of bench.py (no GPU): the ncu-traffic lookup that fills
 `roofline.traffic`, its invalidation when a kernel source changes, the
-whole-job throughput arithmetic and the quantise ALU-roofline constants."""
+whole-job throughput arithmetic, the launch count of the timed regions and
+the quantise ALU-roofline constants."""
 import os
 import shutil
 
@@ -73,6 +74,16 @@ def test_job_throughput_is_all_ranks_over_the_slowest():
     assert bench.job_gbs(1_000_000_000, 1, 1000.0) == pytest.approx(1.0)
     assert bench.job_gbs(1_000_000_000, 4, 1000.0) == pytest.approx(4.0)
     assert bench.max_over_ranks([1.0, 2.0], 1) == [1.0, 2.0]
+
+
+def test_timed_launch_count():
+    """The Llama layer (7 matrices), 20 replays of 10 step / quantise /
+    dequantise passes and of 32 GEMV passes."""
+    got = bench.timed_launches(7, 20, 10, 32)
+    assert got["step"] == 10 * 20 * 10  # 7 quantise + 1 dequantise + pre-rotation + product per step
+    assert got["quantize"] == 7 * 200 and got["dequantize"] == 200
+    assert got["gemv"] == 2 * 20 * 32 and got["gemv_single_matrix"] == 2 * 20 * 7
+    assert got["total"] == sum(v for k, v in got.items() if k != "total") == 5160
 
 
 def test_quantise_alu_operation_count():
